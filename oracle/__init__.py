@@ -1,0 +1,217 @@
+"""Float64 CPU oracle for causal sliding-window RoPE attention (forward and backward).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. It shares no code
+with the CUDA library and never imports it; the only thing both sides take in
+common is the seeded input generator.
+
+The arithmetic lives in ``oracle.c`` (plain C, float64, OpenMP over rows);
+this module compiles it with gcc and marshals numpy float64 arrays. Every
+step cites the page "5만원으로 나만의 ChatGPT 훈련하는 방법" (apidog.com),
+section "1. GPT 모델 (nanochat/gpt.py)" (architecture list and the value
+embedding code) and section "5. 플래시 어텐션 통합" (the causal windowed
+attention call); see the header of ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+NO_NORM = 1
+NO_ROPE = 2
+
+
+class _Layer(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+        ("Hk", ctypes.c_int), ("D", ctypes.c_int), ("W", ctypes.c_int),
+        ("has_ve", ctypes.c_int), ("flags", ctypes.c_int), ("pos_offset", ctypes.c_int),
+        ("rope_base", ctypes.c_double), ("eps", ctypes.c_double), ("scale", ctypes.c_double),
+    ]
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c to liboracle.so with gcc (-O2 -fopenmp)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        L = ctypes.POINTER(_Layer)
+        _lib.oracle_prologue.argtypes = [L] + [dp] * 10
+        _lib.oracle_attn_fwd.argtypes = [L] + [dp] * 5
+        _lib.oracle_fwd_rows.argtypes = [L, dp, dp, dp, ctypes.c_int, ip, dp, dp]
+        _lib.oracle_attn_bwd.argtypes = [L] + [dp] * 9
+        _lib.oracle_dq_rows.argtypes = [L, dp, dp, dp, dp, ctypes.c_int, ip, dp]
+        _lib.oracle_dkv_rows.argtypes = [L, dp, dp, dp, dp, ctypes.c_int, ip, dp, dp]
+        _lib.oracle_prologue_bwd.argtypes = [L] + [dp] * 12
+        _lib.oracle_probs_row.argtypes = [L, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp]
+        _lib.oracle_probs_row.restype = ctypes.c_double
+    return _lib
+
+
+class Layer:
+    """Shape and switches of one attention layer.
+
+    W is the number of visible keys, the query itself included; W >= T is
+    plain causal attention. ``scale`` defaults to 1/sqrt(D). ``flags`` and
+    ``pos_offset`` are test hooks (skip the norm / the rotation, shift the
+    position origin).
+    """
+
+    def __init__(self, B, T, H, Hk, D, W, has_ve, rope_base=10000.0, eps=1e-6,
+                 scale=None, flags=0, pos_offset=0):
+        if H % Hk != 0:
+            raise ValueError("n_head must be a multiple of n_kv_head")
+        if D % 2 != 0 or D > 1024:
+            raise ValueError("head_dim must be even and at most 1024")
+        if W < 1:
+            raise ValueError("window must be >= 1")
+        self.B, self.T, self.H, self.Hk, self.D, self.W = B, T, H, Hk, D, W
+        self.has_ve = bool(has_ve)
+        self.rope_base, self.eps = float(rope_base), float(eps)
+        self.scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+        self.flags, self.pos_offset = int(flags), int(pos_offset)
+
+    def c(self):
+        return _Layer(self.B, self.T, self.H, self.Hk, self.D, min(self.W, 2**31 - 1),
+                      int(self.has_ve), self.flags, self.pos_offset,
+                      self.rope_base, self.eps, self.scale)
+
+
+def _f64(x, shape=None):
+    if x is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if shape is not None and a.shape != tuple(shape):
+        raise ValueError(f"expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def _p(a):
+    if a is None:
+        return ctypes.cast(0, ctypes.POINTER(ctypes.c_double))
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _rows(rows):
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    return r, r.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def prologue(L: Layer, q, k, v, ve=None, gate=None):
+    """q~, k~, v_eff, rstd_q, rstd_k."""
+    lib = _get()
+    sq, skv = (L.B, L.T, L.H, L.D), (L.B, L.T, L.Hk, L.D)
+    q, k, v = _f64(q, sq), _f64(k, skv), _f64(v, skv)
+    ve = _f64(ve, skv) if L.has_ve else None
+    gate = _f64(gate, (L.B, L.T, L.Hk)) if L.has_ve else None
+    qt, kt, veff = np.empty(sq), np.empty(skv), np.empty(skv)
+    rq, rk = np.empty((L.B, L.T, L.H)), np.empty((L.B, L.T, L.Hk))
+    lib.oracle_prologue(ctypes.byref(L.c()), _p(q), _p(k), _p(v), _p(ve), _p(gate),
+                        _p(qt), _p(kt), _p(veff), _p(rq), _p(rk))
+    return qt, kt, veff, rq, rk
+
+
+def attn_fwd(L: Layer, qt, kt, veff):
+    """O (B,T,H,D) and lse (B,H,T), natural log."""
+    lib = _get()
+    qt, kt, veff = _f64(qt), _f64(kt), _f64(veff)
+    O, lse = np.empty((L.B, L.T, L.H, L.D)), np.empty((L.B, L.H, L.T))
+    lib.oracle_attn_fwd(ctypes.byref(L.c()), _p(qt), _p(kt), _p(veff), _p(O), _p(lse))
+    return O, lse
+
+
+def fwd_rows(L: Layer, qt, kt, veff, rows):
+    """O and lse of selected rows; rows is a sequence of (b, h, i)."""
+    lib = _get()
+    qt, kt, veff = _f64(qt), _f64(kt), _f64(veff)
+    r, rp = _rows(rows)
+    O, lse = np.empty((len(r), L.D)), np.empty(len(r))
+    lib.oracle_fwd_rows(ctypes.byref(L.c()), _p(qt), _p(kt), _p(veff), len(r), rp, _p(O), _p(lse))
+    return O, lse
+
+
+def attn_bwd(L: Layer, qt, kt, veff, O, lse, dO):
+    """dq~ (B,T,H,D), dk~ and dv_eff (B,T,Hk,D)."""
+    lib = _get()
+    args = [_f64(a) for a in (qt, kt, veff, O, lse, dO)]
+    dqt = np.empty((L.B, L.T, L.H, L.D))
+    dkt, dveff = np.empty((L.B, L.T, L.Hk, L.D)), np.empty((L.B, L.T, L.Hk, L.D))
+    lib.oracle_attn_bwd(ctypes.byref(L.c()), *[_p(a) for a in args], _p(dqt), _p(dkt), _p(dveff))
+    return dqt, dkt, dveff
+
+
+def dq_rows(L: Layer, qt, kt, veff, dO, rows):
+    """dq~ of selected query rows (b, h, i), computed from scratch."""
+    lib = _get()
+    qt, kt, veff, dO = _f64(qt), _f64(kt), _f64(veff), _f64(dO)
+    r, rp = _rows(rows)
+    out = np.empty((len(r), L.D))
+    lib.oracle_dq_rows(ctypes.byref(L.c()), _p(qt), _p(kt), _p(veff), _p(dO), len(r), rp, _p(out))
+    return out
+
+
+def dkv_rows(L: Layer, qt, kt, veff, dO, rows):
+    """dk~ and dv_eff of selected key rows (b, hk, j), computed from scratch."""
+    lib = _get()
+    qt, kt, veff, dO = _f64(qt), _f64(kt), _f64(veff), _f64(dO)
+    r, rp = _rows(rows)
+    dk, dv = np.empty((len(r), L.D)), np.empty((len(r), L.D))
+    lib.oracle_dkv_rows(ctypes.byref(L.c()), _p(qt), _p(kt), _p(veff), _p(dO), len(r), rp,
+                        _p(dk), _p(dv))
+    return dk, dv
+
+
+def prologue_bwd(L: Layer, q, k, ve, gate, dqt, dkt, dveff):
+    """dQ, dK, dV, dve, dgate (dve/dgate are None without a value embedding)."""
+    lib = _get()
+    q, k, dqt, dkt, dveff = (_f64(a) for a in (q, k, dqt, dkt, dveff))
+    ve = _f64(ve) if L.has_ve else None
+    gate = _f64(gate) if L.has_ve else None
+    dq, dk, dv = np.empty(q.shape), np.empty(k.shape), np.empty(k.shape)
+    dve = np.empty(k.shape) if L.has_ve else None
+    dgate = np.empty((L.B, L.T, L.Hk)) if L.has_ve else None
+    lib.oracle_prologue_bwd(ctypes.byref(L.c()), _p(q), _p(k), _p(ve), _p(gate), _p(dqt),
+                            _p(dkt), _p(dveff), _p(dq), _p(dk), _p(dv), _p(dve), _p(dgate))
+    return dq, dk, dv, dve, dgate
+
+
+def probs_row(L: Layer, qt, kt, b, h, i):
+    """Softmax row p_i. (length T, zeros where masked) and lse_i."""
+    lib = _get()
+    qt, kt = _f64(qt), _f64(kt)
+    p = np.empty(L.T)
+    lse = lib.oracle_probs_row(ctypes.byref(L.c()), _p(qt), _p(kt), b, h, i, _p(p))
+    return p, lse
+
+
+def layer(L: Layer, q, k, v, ve, gate, dO):
+    """Whole layer, forward and backward. Returns a dict of float64 arrays."""
+    qt, kt, veff, rq, rk = prologue(L, q, k, v, ve, gate)
+    O, lse = attn_fwd(L, qt, kt, veff)
+    dqt, dkt, dveff = attn_bwd(L, qt, kt, veff, O, lse, dO)
+    dq, dk, dv, dve, dgate = prologue_bwd(L, q, k, ve, gate, dqt, dkt, dveff)
+    return dict(qt=qt, kt=kt, veff=veff, rstd_q=rq, rstd_k=rk, O=O, lse=lse,
+                dqt=dqt, dkt=dkt, dveff=dveff, dq=dq, dk=dk, dv=dv, dve=dve, dgate=dgate)

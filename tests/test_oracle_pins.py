@@ -1,0 +1,303 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test ties one step of the oracle to a library routine, a closed form, an
+invariant of the definition or finite differences, so that a dropped term, a
+wrong sign or index, or a transposed operand fails at least one of them.
+Definition followed: page "5만원으로 나만의 ChatGPT 훈련하는 방법"
+(apidog.com), section "1. GPT 모델 (nanochat/gpt.py)" (RoPE, QK normalisation,
+GQA, sliding window, value embedding code) and section "5. 플래시 어텐션 통합"
+(causal attention call with a window size).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def inputs(L, seed=0):
+    q = rnd((L.B, L.T, L.H, L.D), seed)
+    k = rnd((L.B, L.T, L.Hk, L.D), seed + 1)
+    v = rnd((L.B, L.T, L.Hk, L.D), seed + 2)
+    ve = rnd((L.B, L.T, L.Hk, L.D), seed + 3)
+    gate = rnd((L.B, L.T, L.Hk), seed + 4)
+    dO = rnd((L.B, L.T, L.H, L.D), seed + 5)
+    return q, k, v, ve, gate, dO
+
+
+def band_mask(T, W):
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    return (j <= i) & (j > i - W)
+
+
+# ---------------------------------------------------------------- attention core
+
+@pytest.mark.parametrize("T,W,H,Hk,D", [(9, 9, 2, 2, 4), (9, 3, 2, 1, 4), (13, 1, 4, 2, 6),
+                                        (16, 5, 6, 2, 8), (7, 100, 3, 3, 2)])
+def test_core_matches_torch_sdpa_and_autograd(T, W, H, Hk, D):
+    """With the norm and rotation switched off, the core is plain banded causal
+    softmax attention: torch's SDPA (float64, explicit band mask, repeat
+    -interleave GQA) and its autograd must agree with the oracle."""
+    L = oracle.Layer(2, T, H, Hk, D, W, has_ve=False, flags=oracle.NO_NORM | oracle.NO_ROPE)
+    q, k, v, _, _, dO = inputs(L, seed=T * 7 + W)
+    qt, kt, veff, rq, rk = oracle.prologue(L, q, k, v)
+    assert np.array_equal(qt, q) and np.array_equal(kt, k) and np.array_equal(veff, v)
+    O, lse = oracle.attn_fwd(L, qt, kt, veff)
+    dqt, dkt, dveff = oracle.attn_bwd(L, qt, kt, veff, O, lse, dO)
+
+    tq = torch.tensor(q).transpose(1, 2).requires_grad_()
+    tk = torch.tensor(k).transpose(1, 2).requires_grad_()
+    tv = torch.tensor(v).transpose(1, 2).requires_grad_()
+    ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=band_mask(T, W), enable_gqa=True)
+    ref.backward(torch.tensor(dO).transpose(1, 2))
+    np.testing.assert_allclose(O, ref.detach().transpose(1, 2).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dqt, tq.grad.transpose(1, 2).numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dkt, tk.grad.transpose(1, 2).numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dveff, tv.grad.transpose(1, 2).numpy(), rtol=0, atol=1e-11)
+
+    # lse against torch.logsumexp of the masked score matrix (library routine)
+    qh = torch.tensor(q).transpose(1, 2)
+    kh = torch.tensor(k).transpose(1, 2).repeat_interleave(H // Hk, dim=1)
+    s = qh @ kh.transpose(-1, -2) / math.sqrt(D)
+    s = s.masked_fill(~band_mask(T, W), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_and_respect_band():
+    L = oracle.Layer(1, 12, 2, 1, 4, 5, has_ve=False)
+    q, k, v, *_ = inputs(L, 3)
+    qt, kt, *_ = oracle.prologue(L, q, k, v)
+    for h in range(2):
+        for i in range(12):
+            p, lse = oracle.probs_row(L, qt, kt, 0, h, i)
+            assert abs(p.sum() - 1.0) < 1e-12
+            visible = [(j <= i and j > i - 5) for j in range(12)]
+            assert all((p[j] > 0) == visible[j] for j in range(12))
+
+
+def test_output_in_convex_hull_of_visible_values():
+    L = oracle.Layer(1, 20, 2, 2, 4, 6, has_ve=True)
+    q, k, v, ve, gate, _ = inputs(L, 4)
+    qt, kt, veff, *_ = oracle.prologue(L, q, k, v, ve, gate)
+    O, _ = oracle.attn_fwd(L, qt, kt, veff)
+    for h in range(2):
+        for i in range(20):
+            win = veff[0, max(0, i - 5): i + 1, h]
+            assert np.all(O[0, i, h] <= win.max(0) + 1e-12)
+            assert np.all(O[0, i, h] >= win.min(0) - 1e-12)
+
+
+def test_window_at_least_T_is_full_causal():
+    args = dict(B=2, T=11, H=4, Hk=2, D=6, has_ve=True)
+    Lw = oracle.Layer(W=11, **args)
+    Lbig = oracle.Layer(W=10**6, **args)
+    data = inputs(Lw, 5)
+    a = oracle.layer(Lw, *data)
+    b = oracle.layer(Lbig, *data)
+    for key in ("O", "lse", "dq", "dk", "dv", "dve", "dgate"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_window_one_gives_value_and_zero_qk_grads():
+    """W = 1: every query sees only itself, so O = v_eff, lse = s_ii and
+    ds = p (dp - Delta) = 0 exactly (p = 1, Delta = dp)."""
+    L = oracle.Layer(2, 9, 4, 2, 8, 1, has_ve=True)
+    q, k, v, ve, gate, dO = inputs(L, 6)
+    r = oracle.layer(L, q, k, v, ve, gate, dO)
+    veff_rep = np.repeat(r["veff"], 2, axis=2)
+    np.testing.assert_allclose(r["O"], veff_rep, rtol=0, atol=1e-14)
+    kt_rep = np.repeat(r["kt"], 2, axis=2)
+    s = (r["qt"] * kt_rep).sum(-1) / math.sqrt(8)
+    np.testing.assert_allclose(r["lse"], s.transpose(0, 2, 1), rtol=0, atol=1e-13)
+    assert np.abs(r["dq"]).max() < 1e-13 and np.abs(r["dk"]).max() < 1e-13
+    np.testing.assert_allclose(r["dveff"], dO.reshape(2, 9, 2, 2, 8).sum(3), atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    Lg = oracle.Layer(2, 10, 6, 2, 4, 4, has_ve=False)
+    Lm = oracle.Layer(2, 10, 6, 6, 4, 4, has_ve=False)
+    q, k, v, _, _, dO = inputs(Lg, 7)
+    g = oracle.layer(Lg, q, k, v, None, None, dO)
+    m = oracle.layer(Lm, q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), None, None, dO)
+    np.testing.assert_allclose(g["O"], m["O"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(g["dq"], m["dq"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g["dk"], m["dk"].reshape(2, 10, 2, 3, 4).sum(3), atol=1e-12)
+    np.testing.assert_allclose(g["dv"], m["dv"].reshape(2, 10, 2, 3, 4).sum(3), atol=1e-12)
+
+
+# ---------------------------------------------------------------- prologue
+
+def test_rope_matches_complex_rotation_and_preserves_norm():
+    """RoPE on half-split pairs is multiplication of x_i + 1j*x_{i+D/2} by
+    exp(1j * t * base^(-2i/D)); it keeps the norm and is the identity at t=0."""
+    D, T = 8, 6
+    L = oracle.Layer(1, T, 1, 1, D, T, has_ve=False, flags=oracle.NO_NORM, rope_base=500.0)
+    q, k, v, *_ = inputs(L, 8)
+    qt, *_ = oracle.prologue(L, q, k, v)
+    z = q[0, :, 0, : D // 2] + 1j * q[0, :, 0, D // 2:]
+    w = 500.0 ** (-2.0 * np.arange(D // 2) / D)
+    zr = z * np.exp(1j * np.arange(T)[:, None] * w[None, :])
+    np.testing.assert_allclose(qt[0, :, 0, : D // 2], zr.real, atol=1e-13)
+    np.testing.assert_allclose(qt[0, :, 0, D // 2:], zr.imag, atol=1e-13)
+    np.testing.assert_allclose(np.linalg.norm(qt, axis=-1), np.linalg.norm(q, axis=-1), rtol=1e-13)
+    np.testing.assert_array_equal(qt[0, 0], q[0, 0])
+
+
+def test_rmsnorm_matches_torch_and_closed_form():
+    L = oracle.Layer(2, 5, 3, 1, 16, 5, has_ve=False, flags=oracle.NO_ROPE, eps=1e-3)
+    q, k, v, *_ = inputs(L, 9)
+    qt, kt, _, rq, rk = oracle.prologue(L, q, k, v)
+    ref = F.rms_norm(torch.tensor(q), (16,), eps=1e-3).numpy()
+    np.testing.assert_allclose(qt, ref, rtol=1e-13, atol=1e-14)
+    ms = (q ** 2).mean(-1)
+    np.testing.assert_allclose((qt ** 2).mean(-1), ms / (ms + 1e-3), rtol=1e-12)
+    np.testing.assert_allclose(rq, 1.0 / np.sqrt(ms + 1e-3), rtol=1e-13)
+
+
+def test_norm_and_rope_commute():
+    base = dict(B=1, T=7, H=2, Hk=1, D=8, W=7, has_ve=False)
+    q, k, v, *_ = inputs(oracle.Layer(**base), 10)
+    both = oracle.prologue(oracle.Layer(**base), q, k, v)[0]
+    rope_only = oracle.prologue(oracle.Layer(**base, flags=oracle.NO_NORM), q, k, v)[0]
+    normed = F.rms_norm(torch.tensor(rope_only), (8,), eps=1e-6).numpy()
+    np.testing.assert_allclose(both, normed, rtol=0, atol=1e-14)
+
+
+def test_scores_depend_only_on_relative_position():
+    base = dict(B=1, T=10, H=2, Hk=2, D=8, W=4, has_ve=True)
+    data = inputs(oracle.Layer(**base), 11)
+    a = oracle.layer(oracle.Layer(**base), *data)
+    b = oracle.layer(oracle.Layer(**base, pos_offset=37), *data)
+    for key in ("O", "lse", "dq", "dk", "dv", "dve", "dgate"):
+        np.testing.assert_allclose(a[key], b[key], rtol=0, atol=1e-11, err_msg=key)
+    assert not np.allclose(a["qt"], b["qt"])  # the rotation itself did change
+
+
+def test_value_residual_gate_limits():
+    """v_eff = v + 3 sigmoid(gate) ve (value-embedding code on the page):
+    gate -> -inf gives v, gate = 0 gives v + 1.5 ve, gate -> +inf gives v + 3 ve."""
+    L = oracle.Layer(1, 3, 2, 2, 4, 3, has_ve=True)
+    q, k, v, ve, *_ = inputs(L, 12)
+    for g, coef in ((-1e4, 0.0), (0.0, 1.5), (1e4, 3.0)):
+        _, _, veff, *_ = oracle.prologue(L, q, k, v, ve, np.full((1, 3, 2), g))
+        np.testing.assert_allclose(veff, v + coef * ve, rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- gradients
+
+def _loss(L, q, k, v, ve, gate, dO):
+    qt, kt, veff, *_ = oracle.prologue(L, q, k, v, ve, gate)
+    O, _ = oracle.attn_fwd(L, qt, kt, veff)
+    return float((O * dO).sum())
+
+
+@pytest.mark.parametrize("W", [1, 3, 16])
+def test_gradients_match_central_differences(W):
+    """Every input of the layer against central differences of L = sum(O * dO)."""
+    L = oracle.Layer(1, 16, 4, 2, 6, W, has_ve=True)
+    q, k, v, ve, gate, dO = inputs(L, 13 + W)
+    r = oracle.layer(L, q, k, v, ve, gate, dO)
+    grads = dict(q=r["dq"], k=r["dk"], v=r["dv"], ve=r["dve"], gate=r["dgate"])
+    data = dict(q=q, k=k, v=v, ve=ve, gate=gate)
+    rng = np.random.default_rng(W)
+    h = 1e-6
+    for name, x in data.items():
+        for _ in range(12):
+            idx = tuple(rng.integers(0, s) for s in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            fp = _loss(L, **{**data, name: xp}, dO=dO)
+            fm = _loss(L, **{**data, name: xm}, dO=dO)
+            fd = (fp - fm) / (2 * h)
+            an = grads[name][idx]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, idx, fd, an)
+
+
+def test_layer_matches_torch_autograd_restatement():
+    """The full layer written with torch library routines (rms_norm, a complex
+    rotation, SDPA with a band mask and GQA), differentiated by autograd."""
+    B, T, H, Hk, D, W = 2, 12, 6, 2, 8, 5
+    L = oracle.Layer(B, T, H, Hk, D, W, has_ve=True, rope_base=10000.0, eps=1e-6)
+    q, k, v, ve, gate, dO = inputs(L, 14)
+    r = oracle.layer(L, q, k, v, ve, gate, dO)
+
+    tq, tk, tv, tve, tg = (torch.tensor(a, requires_grad=True) for a in (q, k, v, ve, gate))
+
+    def rope(x):
+        z = torch.complex(x[..., : D // 2], x[..., D // 2:])
+        w = 10000.0 ** (-2.0 * torch.arange(D // 2, dtype=torch.float64) / D)
+        ang = torch.arange(T, dtype=torch.float64)[:, None] * w[None, :]
+        z = z * torch.polar(torch.ones_like(ang), ang)[None, :, None, :]
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    qn = rope(F.rms_norm(tq, (D,), eps=1e-6))
+    kn = rope(F.rms_norm(tk, (D,), eps=1e-6))
+    vv = tv + 3 * torch.sigmoid(tg)[..., None] * tve
+    o = F.scaled_dot_product_attention(qn.transpose(1, 2), kn.transpose(1, 2), vv.transpose(1, 2),
+                                       attn_mask=band_mask(T, W), enable_gqa=True).transpose(1, 2)
+    o.backward(torch.tensor(dO))
+    np.testing.assert_allclose(r["O"], o.detach().numpy(), atol=1e-12)
+    for name, t in (("dq", tq), ("dk", tk), ("dv", tv), ("dve", tve), ("dgate", tg)):
+        np.testing.assert_allclose(r[name], t.grad.numpy(), atol=1e-11, err_msg=name)
+
+
+# ---------------------------------------------------------------- row entry points
+
+def test_row_functions_match_full_layer():
+    L = oracle.Layer(2, 40, 6, 2, 8, 9, has_ve=True)
+    q, k, v, ve, gate, dO = inputs(L, 15)
+    r = oracle.layer(L, q, k, v, ve, gate, dO)
+    rows = [(0, 0, 0), (1, 5, 39), (0, 3, 17), (1, 2, 8)]
+    O, lse = oracle.fwd_rows(L, r["qt"], r["kt"], r["veff"], rows)
+    dq = oracle.dq_rows(L, r["qt"], r["kt"], r["veff"], dO, rows)
+    for n, (b, h, i) in enumerate(rows):
+        np.testing.assert_allclose(O[n], r["O"][b, i, h], atol=1e-14)
+        assert abs(lse[n] - r["lse"][b, h, i]) < 1e-14
+        np.testing.assert_allclose(dq[n], r["dqt"][b, i, h], atol=1e-13)
+    krows = [(0, 0, 0), (1, 1, 39), (0, 1, 20), (1, 0, 31)]
+    dk, dv = oracle.dkv_rows(L, r["qt"], r["kt"], r["veff"], dO, krows)
+    for n, (b, hk, j) in enumerate(krows):
+        np.testing.assert_allclose(dk[n], r["dkt"][b, j, hk], atol=1e-13)
+        np.testing.assert_allclose(dv[n], r["dveff"][b, j, hk], atol=1e-13)
+
+
+# ---------------------------------------------------------------- golden values
+
+def test_hand_worked_example():
+    """A two-token case worked by hand (derivation in the fixture)."""
+    with open(os.path.join(GOLDEN, "two_token_by_hand.json")) as f:
+        g = json.load(f)
+    L = oracle.Layer(1, 2, 1, 1, 2, 2, has_ve=False, flags=oracle.NO_NORM | oracle.NO_ROPE)
+    q = np.array(g["q"]).reshape(1, 2, 1, 2)
+    k = np.array(g["k"]).reshape(1, 2, 1, 2)
+    v = np.array(g["v"]).reshape(1, 2, 1, 2)
+    O, lse = oracle.attn_fwd(L, q, k, v)
+    np.testing.assert_allclose(O.reshape(2, 2), np.array(g["O"]), atol=1e-15)
+    np.testing.assert_allclose(lse.reshape(2), np.array(g["lse"]), atol=1e-15)
+
+
+def test_oracle_regression_fixture():
+    """Oracle outputs on a small seeded case, written by tests/golden/make_golden.py
+    (which calls only the oracle). Guards against unintended oracle changes."""
+    with open(os.path.join(GOLDEN, "oracle_small_case.json")) as f:
+        g = json.load(f)
+    c = g["case"]
+    L = oracle.Layer(c["B"], c["T"], c["H"], c["Hk"], c["D"], c["W"], has_ve=True)
+    data = inputs(L, c["seed"])
+    r = oracle.layer(L, *data)
+    for key, val in g["checksums"].items():
+        assert abs(float(np.sum(r[key] * np.cos(np.arange(r[key].size)).reshape(r[key].shape))) - val) \
+            <= 1e-9 * max(1.0, abs(val)), key
