@@ -1,0 +1,409 @@
+"""Benchmark: attention forward+backward TFLOP/s of the d24 GQA SSSL layer stack.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    (N > 1: python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...)
+
+One step is the whole hot path over one batch of synthetic input: for each of
+the four layers (windows S, S, S, L) the fused prologue, the forward and the
+backward through the C ABI. FLOPs count only the unmasked causal/window pairs:
+12*D per pair per (batch, head) (forward 4*D, backward 8*D, no credit for the
+backward's recomputation). Every rank runs its own batch (weak scaling, no
+collective on the data path); the time is the max over ranks.
+
+Prints one JSON line on rank 0. ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd+bwd TFLOP/s (bf16, causal/windowed) and % of B200 dense BF16 peak"
+NOMINAL_BF16_TFLOPS = 2250.0  # NVIDIA B200 dense BF16 (HGX B200 datasheet: 36 PF sparse per 8 GPUs)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CONFIG_ID = 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(w):
+    return (f"{w.name}: B={w.B} T={w.T} H={w.H} Hk={w.Hk} D={w.D} windows={w.windows} "
+            f"ve={['on' if v else 'off' for v in w.ve]} rope_base={w.rope_base:g} eps={w.eps:g}")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, indices):
+        self.indices = set(indices)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                idx = int(parts[0])
+            except ValueError:
+                continue
+            if self.indices and idx not in self.indices:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def visible_gpu_indices(n_local):
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if cvd:
+        try:
+            return [int(x) for x in cvd.split(",")][:n_local]
+        except ValueError:
+            return []
+    return list(range(n_local))
+
+
+# ---------------------------------------------------------------------- ours
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import causal_sliding_window_rope_b200 as cs
+    from causal_sliding_window_rope_b200 import synth
+    from causal_sliding_window_rope_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    w = cs.WORKLOADS[CONFIG_ID]
+    specs = [cs.LayerSpec(w.B, w.T, w.H, w.Hk, w.D, W, has_ve=ve, dtype=w.dtype,
+                          rope_base=w.rope_base, eps=w.eps)
+             for W, ve in zip(w.windows, w.ve)]
+    # Per-rank shard: its own batch, seeded by rank (config id offset).
+    host = [synth.layer_inputs(w.B, w.T, w.H, w.Hk, w.D, ve, torch.bfloat16,
+                               config=CONFIG_ID + 1000 * rank, layer=i, dO_std=w.dO_std)
+            for i, ve in enumerate(w.ve)]
+    names = ("q", "k", "v", "ve", "gate", "dO")
+    pinned = [{k: (v.pin_memory() if v is not None else None) for k, v in h.items()} for h in host]
+    inp = [{k: (v.to(dev) if v is not None else None) for k, v in h.items()} for h in host]
+    bufs = [cs.LayerBuffers(s, device=dev) for s in specs]
+    stream = torch.cuda.current_stream(dev)
+    l2_flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        for s, x, b in zip(specs, inp, bufs):
+            cs.layer_forward(s, b, x["q"], x["k"], x["v"], x["ve"], x["gate"])
+            cs.layer_backward(s, b, x["q"], x["k"], x["ve"], x["gate"], x["dO"])
+
+    out_names = ("O", "dQ", "dK", "dV", "dve", "dgate")
+    host_out = [{n: torch.empty_like(getattr(b, n), device="cpu").pin_memory()
+                 for n in out_names if getattr(b, n) is not None} for b in bufs]
+    h2d = sum(v.numel() * v.element_size() for p in pinned for v in p.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for o in host_out for v in o.values())
+
+    def step_e2e():
+        for x, p in zip(inp, pinned):
+            for n in names:
+                if p[n] is not None:
+                    x[n].copy_(p[n], non_blocking=True)
+        step()
+        for b, o in zip(bufs, host_out):
+            for n, t in o.items():
+                t.copy_(getattr(b, n), non_blocking=True)
+
+    flops_layer = [12.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
+    flops_fwd = [4.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
+    flops_bwd = [8.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
+    flops_step = sum(flops_layer)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    cs.cswattn_sync_status()
+
+    def timed(fn, k, flush):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(k)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        for a, b in evs:
+            if flush:
+                l2_flush.zero_()  # outside the events: L2 holds nothing of the next step
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    clocks = ClockSampler(visible_gpu_indices(world if world > 1 else 1) if rank == 0 else [])
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    cs.cswattn_set_timing(True)
+    cs.cswattn_kernel_times()
+    total_ms = timed(step, args.steps, flush=True)
+    ktimes = cs.cswattn_kernel_times()
+    cs.cswattn_set_timing(False)
+    clk = clocks.stop() if rank == 0 else None
+    cs.cswattn_sync_status()
+
+    # e2e: host buffers in, results out, copies inside the timed region
+    for _ in range(2):
+        step_e2e()
+    torch.cuda.synchronize(dev)
+    e2e_ms = timed(step_e2e, max(1, min(args.steps, 5)), flush=False)
+    e2e_steps = max(1, min(args.steps, 5))
+    cs.cswattn_sync_status()
+
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+    e2e_value = flops_step * world / (e2e_ms / e2e_steps * 1e-3) / 1e12
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        launches = sum(n for _, n in ktimes.values())
+        # dominant kernel: the kind with the most device time
+        dom = max(ktimes, key=lambda k: ktimes[k][0])
+        dom_ms, dom_n = ktimes[dom]
+        if dom in ("fwd", "bwd"):
+            fl = (flops_fwd if dom == "fwd" else flops_bwd)
+            achieved = sum(fl) * args.steps / (dom_ms * 1e-3) / 1e12
+            peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+            roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_source": f"{peak_src} bf16_tflops_sustained",
+                    "launches": dom_n, "avg_launch_us": round(dom_ms / max(dom_n, 1) * 1e3, 2),
+                    "traffic": traffic_for(dom)}
+        else:
+            roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": None, "traffic": traffic_for(dom)}
+        kern = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches": v[1]}
+                for k, v in ktimes.items()}
+        for k, fl in (("fwd", flops_fwd), ("bwd", flops_bwd)):
+            if ktimes[k][0] > 0:
+                kern[k]["tflops"] = round(sum(fl) * args.steps / (ktimes[k][0] * 1e-3) / 1e12, 2)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) d24-layer-shaped tensors)",
+            "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.T,
+                       "parallelism": f"dp{world} (independent batch per GPU, no collective)",
+                       "l2": "256 MiB buffer written between timed steps, outside the events",
+                       "flops_per_step_per_gpu": flops_step, "flop_convention": "12*D per unmasked pair"},
+            "pct_of_peak": {
+                "measured_burst": round(value / world / peaks.get("bf16_tflops", 1590.0), 4),
+                "measured_sustained": round(value / world / peaks.get("bf16_tflops_sustained", 1400.0), 4),
+                "nominal_dense": round(value / world / NOMINAL_BF16_TFLOPS, 4),
+                "peak_source": peak_src},
+            "roofline": roof,
+            "kernels": kern,
+            "gpu_launches": launches,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms / e2e_steps, 3)},
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def traffic_for(kind):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's
+    source still matches the one the counters were taken on; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d.get(kind)
+        if not ent:
+            return None
+        if ent.get("source_sha") != kernel_source_sha(kind):
+            return None
+        return ent.get("bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+def kernel_source_sha(kind):
+    import hashlib
+    files = {"fwd": ["fwd_sm100.cuh", "common.cuh"], "bwd": ["bwd_sm100.cuh", "common.cuh"],
+             "prologue": ["prologue.cuh"], "bwd_pre": ["bwd_aux.cuh"], "bwd_epi": ["bwd_aux.cuh"]}
+    h = hashlib.sha256()
+    for fn in files.get(kind, []):
+        with open(os.path.join(ROOT, "causal_sliding_window_rope_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(w):
+    """A bounded slice of the workload for the float64 CPU oracle: batch 1, one
+    KV head and its query group, all four layers' windows, full T."""
+    import numpy as np
+    return dict(B=1, T=w.T, H=w.H // w.Hk, Hk=1, D=w.D, windows=w.windows, ve=w.ve,
+                flops=sum(12.0 * w.D * w.pairs(W) * 1 * (w.H // w.Hk) for W in w.windows),
+                rng=np.random.default_rng(0))
+
+
+def time_oracle_sample(w, n_layers=None):
+    import numpy as np
+
+    import oracle
+    s = oracle_sample(w)
+    layers = list(zip(s["windows"], s["ve"]))[: n_layers or len(s["windows"])]
+    rng = s["rng"]
+    t0 = time.perf_counter()
+    flops = 0.0
+    for W, ve in layers:
+        L = oracle.Layer(s["B"], s["T"], s["H"], s["Hk"], s["D"], W, ve, rope_base=w.rope_base, eps=w.eps)
+        q = rng.standard_normal((1, s["T"], s["H"], s["D"]))
+        k = rng.standard_normal((1, s["T"], 1, s["D"]))
+        v = rng.standard_normal((1, s["T"], 1, s["D"]))
+        vee = rng.standard_normal((1, s["T"], 1, s["D"])) if ve else None
+        g = rng.standard_normal((1, s["T"], 1)) if ve else None
+        dO = rng.standard_normal((1, s["T"], s["H"], s["D"]))
+        oracle.layer(L, q, k, v, vee, g, dO)
+        flops += 12.0 * w.D * w.pairs(W) * s["H"]
+    dt = time.perf_counter() - t0
+    return flops, dt, len(layers)
+
+
+def cpu_baseline(w, budget_s=20.0):
+    import oracle
+    oracle.build()
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    flops, dt, n = time_oracle_sample(w, n_layers=1)
+    if dt < budget_s / 4:
+        f2, d2, n2 = time_oracle_sample(w, n_layers=None)
+        flops, dt, n = f2, d2, n2
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"float64 C oracle (prologue+fwd+bwd+chain rule), batch 1, one KV head "
+                      f"with its {w.H // w.Hk} query heads, T={w.T}, first {n} of the layer windows "
+                      f"{w.windows}; FLOPs counted as 12*D per unmasked pair"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import causal_sliding_window_rope_b200 as cs
+    import oracle
+    oracle.build()
+    w = cs.WORKLOADS[CONFIG_ID]
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    for _ in range(args.warmup and 1):
+        time_oracle_sample(w, n_layers=1)
+    tot_f, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, t, _ = time_oracle_sample(w, n_layers=1)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_t / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(w), "sample": "one KV head group, batch 1, first layer (S window)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": "float64 C oracle, batch 1, one KV head group, one S layer per step"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

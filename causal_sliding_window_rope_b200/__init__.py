@@ -1,0 +1,220 @@
+"""B200-native causal sliding-window RoPE attention (forward and backward).
+
+A thin ctypes binding over libcswattn.so, the C ABI declared in
+``include/cswattn.h``. Every step of the computation runs in the library's
+CUDA kernels; this module only marshals pointers, sizes and the stream.
+PyTorch provides device memory and streams.
+
+The layer is the attention of a nanochat-style GPT block (page
+"5만원으로 나만의 ChatGPT 훈련하는 방법", section "1. GPT 모델"): RoPE,
+parameter-free QK RMSNorm, GQA, a per-layer sliding window ("SSSL") and the
+value-embedding residual v + 3*sigmoid(gate)*ve.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+from .configs import WORKLOADS, Workload, alternating_ve, window_pattern  # noqa: F401
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcswattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+F32, BF16 = 0, 1
+
+# Every symbol the header declares; the CPU tests check the library exports them.
+EXPORTS = ("attn_prologue", "attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd",
+           "cswattn_sync_status", "cswattn_set_wait_limit_ns", "cswattn_set_timing",
+           "cswattn_kernel_times", "cswattn_last_error", "cswattn_version")
+KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi")
+
+
+class CswattnLayer(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("n_head", ctypes.c_int),
+        ("n_kv_head", ctypes.c_int), ("head_dim", ctypes.c_int), ("window", ctypes.c_int),
+        ("rope_base", ctypes.c_float), ("eps", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+        ("has_ve", ctypes.c_int), ("dtype", ctypes.c_int),
+    ]
+
+
+class CswattnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"cswattn status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library. Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m causal_sliding_window_rope_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+        lp = ctypes.POINTER(CswattnLayer)
+        L.attn_prologue.argtypes = [lp] + [vp] * 8 + [fp, fp, vp]
+        L.attn_fwd.argtypes = [lp, vp, vp, vp, vp, fp, vp]
+        L.attn_bwd_workspace_bytes.argtypes = [lp]
+        L.attn_bwd_workspace_bytes.restype = sz
+        L.attn_bwd.argtypes = [lp] + [vp] * 7 + [fp, fp, vp, fp, vp] + [vp] * 6 + [sz, vp]
+        L.cswattn_sync_status.argtypes = [vp]
+        L.cswattn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.cswattn_set_wait_limit_ns.restype = None
+        L.cswattn_last_error.restype = ctypes.c_char_p
+        L.cswattn_set_timing.argtypes = [ctypes.c_int]
+        L.cswattn_set_timing.restype = None
+        L.cswattn_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                           ctypes.POINTER(ctypes.c_int)]
+        L.cswattn_kernel_times.restype = ctypes.c_int
+        for name in ("attn_prologue", "attn_fwd", "attn_bwd", "cswattn_sync_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+@dataclass
+class LayerSpec:
+    """Arguments of one layer, as in the C struct ``cswattn_layer``."""
+    B: int
+    T: int
+    n_head: int
+    n_kv_head: int
+    head_dim: int
+    window: int
+    has_ve: bool = True
+    dtype: str = "bf16"          # "bf16" or "f32"
+    rope_base: float = 10000.0
+    eps: float = 1e-6
+    softmax_scale: float = 0.0   # 0: 1/sqrt(head_dim)
+
+    def c(self) -> CswattnLayer:
+        return CswattnLayer(self.B, self.T, self.n_head, self.n_kv_head, self.head_dim,
+                            self.window, self.rope_base, self.eps, self.softmax_scale,
+                            int(bool(self.has_ve)), BF16 if self.dtype == "bf16" else F32)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_contiguous():
+        raise ValueError("tensors passed to cswattn must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int):
+    if status != OK:
+        raise CswattnError(status, lib().cswattn_last_error().decode())
+
+
+def attn_prologue(spec: LayerSpec, q, k, v, ve, gate, q_out, k_out, v_out, rstd_q, rstd_k,
+                  stream=None):
+    layer = spec.c()
+    _check(lib().attn_prologue(ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(v), _ptr(ve),
+                               _ptr(gate), _ptr(q_out), _ptr(k_out), _ptr(v_out),
+                               _ptr(rstd_q), _ptr(rstd_k), _stream(stream)))
+
+
+def attn_fwd(spec: LayerSpec, q_out, k_out, v_out, O, lse, stream=None):
+    layer = spec.c()
+    _check(lib().attn_fwd(ctypes.byref(layer), _ptr(q_out), _ptr(k_out), _ptr(v_out),
+                          _ptr(O), _ptr(lse), _stream(stream)))
+
+
+def attn_bwd_workspace_bytes(spec: LayerSpec) -> int:
+    layer = spec.c()
+    return int(lib().attn_bwd_workspace_bytes(ctypes.byref(layer)))
+
+
+def attn_bwd(spec: LayerSpec, q, k, ve, gate, q_out, k_out, v_out, rstd_q, rstd_k, O, lse,
+             dO, dQ, dK, dV, dve, dgate, workspace, workspace_bytes=None, stream=None):
+    layer = spec.c()
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().attn_bwd(ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(ve), _ptr(gate),
+                          _ptr(q_out), _ptr(k_out), _ptr(v_out), _ptr(rstd_q), _ptr(rstd_k),
+                          _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV),
+                          _ptr(dve), _ptr(dgate), _ptr(workspace), workspace_bytes,
+                          _stream(stream)))
+
+
+def cswattn_sync_status(stream=None):
+    _check(lib().cswattn_sync_status(_stream(stream)))
+
+
+def cswattn_set_wait_limit_ns(ns: int):
+    lib().cswattn_set_wait_limit_ns(int(ns))
+
+
+def cswattn_set_timing(enable: bool):
+    lib().cswattn_set_timing(1 if enable else 0)
+
+
+def cswattn_kernel_times():
+    """{kind: (total_ms, launches)} since the last read, for the kernel kinds."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int * n)()
+    _check(lib().cswattn_kernel_times(ms, cnt))
+    return {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def cswattn_version() -> int:
+    return int(lib().cswattn_version())
+
+
+# ------------------------------------------------------------------ convenience
+
+class LayerBuffers:
+    """Device buffers of one layer (torch tensors), allocated once and reused."""
+
+    def __init__(self, spec: LayerSpec, device="cuda"):
+        import torch
+        dt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+        B, T, H, Hk, D = spec.B, spec.T, spec.n_head, spec.n_kv_head, spec.head_dim
+        e = dict(device=device, dtype=dt)
+        f = dict(device=device, dtype=torch.float32)
+        self.spec = spec
+        self.q_out = torch.empty(B, T, H, D, **e)
+        self.k_out = torch.empty(B, T, Hk, D, **e)
+        self.v_out = torch.empty(B, T, Hk, D, **e)
+        self.rstd_q = torch.empty(B, T, H, **f)
+        self.rstd_k = torch.empty(B, T, Hk, **f)
+        self.O = torch.empty(B, T, H, D, **e)
+        self.lse = torch.empty(B, H, T, **f)
+        self.dQ = torch.empty(B, T, H, D, **e)
+        self.dK = torch.empty(B, T, Hk, D, **e)
+        self.dV = torch.empty(B, T, Hk, D, **e)
+        self.dve = torch.empty(B, T, Hk, D, **e) if spec.has_ve else None
+        self.dgate = torch.empty(B, T, Hk, **e) if spec.has_ve else None
+        nbytes = attn_bwd_workspace_bytes(spec)
+        self.workspace = torch.empty(max(nbytes, 256), device=device, dtype=torch.uint8)
+
+
+def layer_forward(spec: LayerSpec, buf: LayerBuffers, q, k, v, ve=None, gate=None, stream=None):
+    attn_prologue(spec, q, k, v, ve, gate, buf.q_out, buf.k_out, buf.v_out, buf.rstd_q,
+                  buf.rstd_k, stream)
+    attn_fwd(spec, buf.q_out, buf.k_out, buf.v_out, buf.O, buf.lse, stream)
+
+
+def layer_backward(spec: LayerSpec, buf: LayerBuffers, q, k, ve, gate, dO, stream=None):
+    attn_bwd(spec, q, k, ve, gate, buf.q_out, buf.k_out, buf.v_out, buf.rstd_q, buf.rstd_k,
+             buf.O, buf.lse, dO, buf.dQ, buf.dK, buf.dV, buf.dve, buf.dgate, buf.workspace,
+             stream=stream)

@@ -1,0 +1,415 @@
+// bwd_sm100.cuh -- attention backward on tcgen05 tensor cores (bf16, D = 128).
+//
+// Gradient of the causal sliding-window attention of the page
+// "5만원으로 나만의 ChatGPT 훈련하는 방법" (section "5. 플래시 어텐션 통합",
+// with the architecture list's sliding window and GQA), written out:
+//   p_ij = exp(c q~_i.k~_j - lse_i),  dp_ij = dO_i . v_j,
+//   ds_ij = p_ij (dp_ij - Delta_i),   Delta_i = dO_i . O_i,
+//   dv_j  = sum_{h in group} sum_i p_ij dO_i,
+//   dk~_j = c sum_{h in group} sum_i ds_ij q~_i,   dq~_i = c sum_j ds_ij k~_j.
+//
+// Work unit (one CTA): one 128-key tile of one (batch, KV head). It keeps
+// K and V in shared memory and its dK/dV accumulators in TMEM while it walks
+// every query head of the GQA group and every 64-query step that sees the
+// tile, so dK and dV are summed over the group without atomics and written
+// once. Per step (transposed products, keys on the TMEM lanes):
+//   S^T  = K Q^T      (M=128 keys, N=64 queries, K=128 d)   SS MMA
+//   dP^T = V dO^T     (same shape)                         SS MMA
+//   softmax warps: P^T = exp2(c2 S^T - lse2), dS^T = P^T (dP^T - Delta),
+//                  both as bf16 into shared memory (128B-swizzled, K-major)
+//   dV  += P^T dO     (M=128 keys, N=128 d, K=64)           SS MMA
+//   dK  += dS^T Q     (same shape)                         SS MMA
+//   dQ^T = K^T dS^T   (M=128 d, N=64 queries, K=128 keys)   SS MMA, into
+//          the S^T columns of the step, drained by the dQ warps into a
+//          float32 tile that a bulk reduce-add sends to the dq accumulator.
+// TMEM (512 columns): SP0 | SP1 (S^T at +0, dP^T at +64; double buffered so
+// the next step's products overlap this step's softmax) | dV | dK.
+// Roles: warp 0 TMA, warp 1 MMA issuer + TMEM owner, warps 4-7 softmax
+// (thread = key row), warps 8-11 dQ drain (thread = head_dim row of dQ^T).
+#pragma once
+#include "common.cuh"
+
+namespace cswattn {
+namespace bwd {
+
+constexpr int kBN = 128;  // keys per tile
+constexpr int kBQ = 64;   // queries per step
+constexpr int kD = 128;
+constexpr int kThreads = 384;
+constexpr int kKVBytes = kBN * kD * 2;   // 32 KB
+constexpr int kKVPanel = kKVBytes / 2;   // 16 KB: 128 rows x 128 B
+constexpr int kQBytes = kBQ * kD * 2;    // 16 KB
+constexpr int kQPanel = kQBytes / 2;     // 8 KB: 64 rows x 128 B
+constexpr int kPBytes = kBN * kBQ * 2;   // 16 KB: 128 rows x 128 B
+constexpr int kDQBytes = kBQ * kD * 4;   // 32 KB float32 staging
+
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKVBytes;
+constexpr int kOffQ = kOffV + kKVBytes;        // [2]
+constexpr int kOffDO = kOffQ + 2 * kQBytes;    // [2]
+constexpr int kOffP = kOffDO + 2 * kQBytes;    // [2]
+constexpr int kOffDS = kOffP + 2 * kPBytes;    // [2]
+constexpr int kOffDQ = kOffDS + 2 * kPBytes;
+constexpr int kOffBar = kOffDQ + kDQBytes;
+constexpr int kOffRow = kOffBar + 256;         // lse2[2][64], delta[2][64]
+constexpr int kSmemBytes = kOffRow + 4 * kBQ * 4 + 1024;
+
+// TMEM column of the S^T / dP^T buffer st (0 or 1).
+__host__ __device__ constexpr uint32_t col_sp(int st) { return st ? 128u : 0u; }
+constexpr uint32_t kColDV = 256u;
+constexpr uint32_t kColDK = 384u;
+
+struct Params {
+  int B, T, H, Hk, W, g, nkv;
+  float scale_log2;  // c * log2(e)
+  float scale;       // c
+  const float* lse;    // (B,H,T) natural log
+  const float* delta;  // (B,H,T)
+  float* dq_acc;       // (B,H,T,D), accumulated (must start at zero)
+  float* dk_acc;       // (B,T,Hk,D)
+  float* dv_acc;       // (B,T,Hk,D)
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > ns) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;     // [2]
+  uint64_t* q_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* p_full = bars + 7;     // [2]
+  uint64_t* ps_empty = bars + 9;   // [2]
+  uint64_t* dq_full = bars + 11;   // [2]
+  uint64_t* dq_empty = bars + 13;  // [2]
+  uint64_t* acc_full = bars + 15;
+  uint64_t* mma_done = bars + 16;
+  uint64_t* row_full = bars + 17;    // [2] lse2/delta of a step staged
+  uint64_t* row_empty = bars + 19;   // [2] every softmax thread done with a slot
+  uint64_t* stage_free = bars + 21;  // dQ staging tile may be overwritten
+  uint64_t* stage_full = bars + 22;  // dQ staging tile written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 24);
+  float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [2][64]
+  float* s_delta = s_lse2 + 2 * kBQ;                                // [2][64]
+
+  const int warp = warp_id(), lane = lane_id();
+
+  // ---- work unit: KV block j (ascending = most queries first), (b, hk)
+  const int BHk = p.B * p.Hk;
+  const int j = static_cast<int>(blockIdx.x) / BHk;
+  const int bh = static_cast<int>(blockIdx.x) % BHk;
+  const int b = bh / p.Hk, hk = bh % p.Hk;
+  const int k0 = j * kBN;
+  const long long q_last_ll = min(static_cast<long long>(p.T) - 1,
+                                  static_cast<long long>(k0) + kBN - 1 + p.W - 1);
+  const int qs_lo = k0 / kBQ;
+  const int qs_hi = static_cast<int>(q_last_ll) / kBQ;
+  const int nsph = qs_hi - qs_lo + 1;  // steps per head
+  const int N = p.g * nsph;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&ps_empty[s], 1);
+      mbar_init(&dq_full[s], 1);
+      mbar_init(&dq_empty[s], 128);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&row_full[s], kBQ);
+      mbar_init(&row_empty[s], 128);
+    }
+    mbar_init(stage_free, 1);
+    mbar_init(stage_full, 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.wait_ns};
+
+  auto step_head = [&](int n) { return hk * p.g + n / nsph; };
+  auto step_q0 = [&](int n) { return (qs_lo + n % nsph) * kBQ; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int nq[2] = {0, 0};
+      mbar_expect_tx(kv_full, 2 * kKVBytes);
+      tma_load_4d(&tmK, kv_full, smem + kOffK, 0, hk, k0, b);
+      tma_load_4d(&tmK, kv_full, smem + kOffK + kKVPanel, 64, hk, k0, b);
+      tma_load_4d(&tmV, kv_full, smem + kOffV, 0, hk, k0, b);
+      tma_load_4d(&tmV, kv_full, smem + kOffV + kKVPanel, 64, hk, k0, b);
+      for (int n = 0; n < N; ++n) {
+        const int st = n & 1, use = n >> 1;
+        if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, wc)) break;
+        const int h = step_head(n), q0 = step_q0(n);
+        mbar_expect_tx(&q_full[st], 2 * kQBytes);
+        uint8_t* qd = smem + kOffQ + st * kQBytes;
+        uint8_t* od = smem + kOffDO + st * kQBytes;
+        tma_load_4d(&tmQ, &q_full[st], qd, 0, h, q0, b);
+        tma_load_4d(&tmQ, &q_full[st], qd + kQPanel, 64, h, q0, b);
+        tma_load_4d(&tmDO, &q_full[st], od, 0, h, q0, b);
+        tma_load_4d(&tmDO, &q_full[st], od + kQPanel, 64, h, q0, b);
+        ++nq[st];
+      }
+      drain_wait(kv_full, 0, p.wait_ns);
+      for (int s = 0; s < 2; ++s)
+        if (nq[s] > 0) drain_wait(&q_full[s], (nq[s] - 1) & 1, p.wait_ns);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idS = idesc_bf16(128, 64, 0, 0);    // K Q^T, V dO^T
+      constexpr uint32_t idKV = idesc_bf16(128, 128, 0, 1);  // P^T dO, dS^T Q
+      constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T
+      const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV);
+      const uint32_t sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO);
+      const uint32_t sP = smem_u32(smem + kOffP), sDS = smem_u32(smem + kOffDS);
+      bool ok = mbar_wait(kv_full, 0, wc);
+      tc_fence_after();
+
+      auto issue_SdP = [&](int n) -> bool {
+        const int st = n & 1, use = n >> 1;
+        if (!mbar_wait(&q_full[st], use & 1, wc)) return false;
+        if (use > 0 && !mbar_wait(&dq_empty[st], (use - 1) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t qa = sQ + st * kQBytes, oa = sDO + st * kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ok_ = (kk >> 2) * kKVPanel + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * kQPanel + (kk & 3) * 32;
+          mma_ss(tmem + col_sp(st), sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(qa + oq, 16, 1024),
+                 idS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ok_ = (kk >> 2) * kKVPanel + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * kQPanel + (kk & 3) * 32;
+          mma_ss(tmem + col_sp(st) + 64, sdesc_sw128(sV + ok_, 16, 1024),
+                 sdesc_sw128(oa + oq, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[st]);
+        return true;
+      };
+
+      if (ok) ok = issue_SdP(0);
+      for (int n = 0; ok && n < N; ++n) {
+        const int st = n & 1, use = n >> 1;
+        if (n + 1 < N && !issue_SdP(n + 1)) break;
+        if (!mbar_wait(&p_full[st], use & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t pa = sP + st * kPBytes, da = sDS + st * kPBytes;
+        const uint32_t qa = sQ + st * kQBytes, oa = sDO + st * kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
+          mma_ss(tmem + kColDV, sdesc_sw128(pa + kk * 32, 16, 1024),
+                 sdesc_sw128(oa + kk * 2048, kQPanel, 1024), idKV, (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
+          mma_ss(tmem + kColDK, sdesc_sw128(da + kk * 32, 16, 1024),
+                 sdesc_sw128(qa + kk * 2048, kQPanel, 1024), idKV, (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
+          mma_ss(tmem + col_sp(st), sdesc_sw128(sK + kk * 2048, kKVPanel, 1024),
+                 sdesc_sw128(da + kk * 2048, kPBytes, 1024), idDQ, kk > 0 ? 1u : 0u);
+        mma_commit(&dq_full[st]);
+        mma_commit(&ps_empty[st]);
+        mma_commit(&q_empty[st]);
+      }
+      mma_commit(acc_full);
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0, p.wait_ns);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // -------------------------------------------------- softmax / dS
+    const int r = (warp & 3) * 32 + lane;  // key row within the tile
+    const int tid = (warp - 4) * 32 + lane;
+    const int kj = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float c2 = p.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < N; ++n) {
+      const int st = n & 1, use = n >> 1;
+      const int h = step_head(n), q0 = step_q0(n);
+      // Stage lse2 / Delta of this step's 64 queries (slot st) once every
+      // thread has finished with the slot's previous contents.
+      if (tid < kBQ) {
+        bool got = use == 0 || mbar_wait(&row_empty[st], (use - 1) & 1, wc);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        const int q = q0 + tid;
+        const size_t row = (static_cast<size_t>(b) * p.H + h) * p.T + q;
+        s_lse2[st * kBQ + tid] = q < p.T ? p.lse[row] * 1.4426950408889634f : INFINITY;
+        s_delta[st * kBQ + tid] = q < p.T ? p.delta[row] : 0.f;
+        mbar_arrive(&row_full[st]);
+      }
+      bool got = mbar_wait(&row_full[st], use & 1, wc);
+      got = got && mbar_wait(&s_full[st], use & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[2][32], dv[2][32];
+      tmem_ld32(tmem + lane_off + col_sp(st), sv[0]);
+      tmem_ld32(tmem + lane_off + col_sp(st) + 32, sv[1]);
+      tmem_ld32(tmem + lane_off + col_sp(st) + 64, dv[0]);
+      tmem_ld32(tmem + lane_off + col_sp(st) + 96, dv[1]);
+      tmem_ld_wait();
+      const bool need_mask = (q0 < k0 + kBN - 1) || (q0 + kBQ - 1 - k0 >= p.W);
+      const float* L2 = s_lse2 + st * kBQ;
+      const float* DL = s_delta + st * kBQ;
+      uint32_t pp[32], dd[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = c * 32 + i + e;
+            const int q = q0 + col;
+            float pr = ex2(fmaf(__uint_as_float(sv[c][i + e]), c2, -L2[col]));
+            if (need_mask && (q < kj || q - kj >= p.W)) pr = 0.f;
+            pv[e] = pr;
+            dsv[e] = pr * (__uint_as_float(dv[c][i + e]) - DL[col]);
+          }
+          pp[c * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
+          dd[c * 16 + i / 2] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+      mbar_arrive(&row_empty[st]);
+      got = use == 0 || mbar_wait(&ps_empty[st], (use - 1) & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      // Row r of P^T / dS^T: 64 bf16 = 8 chunks of 16 B, 128B-swizzled.
+      uint8_t* prow = smem + kOffP + st * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+      uint8_t* drow = smem + kOffDS + st * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const int pos = (ch ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(prow + pos) =
+            make_uint4(pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(drow + pos) =
+            make_uint4(dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[st]);
+    }
+    // dK / dV write-out: thread r holds key row r of both accumulators.
+    const bool acc_ok = ok && mbar_wait(acc_full, 0, wc);
+    if (__all_sync(0xffffffffu, acc_ok)) {
+      tc_fence_after();
+      const bool row_ok = kj < p.T;
+      const size_t off = ((static_cast<size_t>(b) * p.T + (row_ok ? kj : 0)) * p.Hk + hk) * kD;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + kColDV + c * 32, a);
+        tmem_ld_wait();
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(p.dv_acc + off + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            dst[v4] = make_float4(__uint_as_float(a[4 * v4]), __uint_as_float(a[4 * v4 + 1]),
+                                  __uint_as_float(a[4 * v4 + 2]), __uint_as_float(a[4 * v4 + 3]));
+        }
+        tmem_ld32(tmem + lane_off + kColDK + c * 32, a);
+        tmem_ld_wait();
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(p.dk_acc + off + c * 32);
+          const float sc = p.scale;
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            dst[v4] = make_float4(__uint_as_float(a[4 * v4]) * sc, __uint_as_float(a[4 * v4 + 1]) * sc,
+                                  __uint_as_float(a[4 * v4 + 2]) * sc, __uint_as_float(a[4 * v4 + 3]) * sc);
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // -------------------------------------------------- dQ drain
+    const int d = (warp & 3) * 32 + lane;  // TMEM lane = head_dim index of dQ^T
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const bool leader = (warp == 8 && lane == 0);
+    float* sdq = reinterpret_cast<float*>(smem + kOffDQ);
+    const float sc = p.scale;
+    for (int n = 0; n < N; ++n) {
+      const int st = n & 1, use = n >> 1;
+      const int h = step_head(n), q0 = step_q0(n);
+      bool got = mbar_wait(&dq_full[st], use & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      uint32_t a[2][32];
+      tmem_ld32(tmem + lane_off + col_sp(st), a[0]);
+      tmem_ld32(tmem + lane_off + col_sp(st) + 32, a[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&dq_empty[st]);
+      if (leader) {
+        bulk_wait_read0();  // the previous reduction has read the staging tile
+        mbar_arrive(stage_free);
+      }
+      got = mbar_wait(stage_free, n & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) break;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sdq[(c * 32 + i) * kD + d] = __uint_as_float(a[c][i]) * sc;
+      fence_proxy_async_smem();
+      mbar_arrive(stage_full);
+      if (leader) {
+        if (!mbar_wait(stage_full, n & 1, wc)) break;
+        const int nrows = min(kBQ, p.T - q0);
+        float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.T + q0) * kD;
+        bulk_reduce_add_f32(dst, sdq, static_cast<uint32_t>(nrows) * kD * 4);
+        bulk_commit();
+      }
+    }
+    if (leader) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bwd
+}  // namespace cswattn

@@ -1,0 +1,621 @@
+// cswattn.cu -- C ABI of libcswattn.so: host-side validation, tensor maps,
+// launches. Single translation unit (the kernels are in the .cuh files) so
+// that every kernel shares one device status word.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <cmath>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/cswattn.h"
+#include "common.cuh"
+#include "prologue.cuh"
+#include "simt_f32.cuh"
+#include "bwd_aux.cuh"
+#include "fwd_sm100.cuh"
+#include "bwd_sm100.cuh"
+
+using namespace cswattn;
+
+namespace {
+
+thread_local std::string t_err;
+std::atomic<unsigned long long> g_wait_ns{2000000000ull};
+
+cswattn_status fail(cswattn_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return s;
+}
+
+cswattn_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(CSWATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxT = 1 << 20;
+
+struct Shape {
+  int B, T, H, Hk, D, W, g;
+  bool bf16;
+  size_t esize;
+  float scale;
+};
+
+cswattn_status check_layer(const cswattn_layer* L, Shape* s) {
+  if (!L) return fail(CSWATTN_ERR_INVALID_ARG, "layer is NULL");
+  if (L->B < 1 || L->T < 1 || L->n_head < 1 || L->n_kv_head < 1 || L->head_dim < 1)
+    return fail(CSWATTN_ERR_INVALID_ARG, "B, T, n_head, n_kv_head, head_dim must be >= 1");
+  if (L->n_head % L->n_kv_head != 0)
+    return fail(CSWATTN_ERR_INVALID_ARG, "n_head (%d) must be a multiple of n_kv_head (%d)",
+                L->n_head, L->n_kv_head);
+  if (L->window < 1) return fail(CSWATTN_ERR_INVALID_ARG, "window must be >= 1 (got %d)", L->window);
+  if (L->has_ve != 0 && L->has_ve != 1) return fail(CSWATTN_ERR_INVALID_ARG, "has_ve must be 0 or 1");
+  if (!(L->rope_base > 0.f) || !std::isfinite(L->rope_base))
+    return fail(CSWATTN_ERR_INVALID_ARG, "rope_base must be finite and > 0");
+  if (!(L->eps >= 0.f) || !std::isfinite(L->eps))
+    return fail(CSWATTN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (!(L->softmax_scale >= 0.f) || !std::isfinite(L->softmax_scale))
+    return fail(CSWATTN_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (L->dtype != CSWATTN_F32 && L->dtype != CSWATTN_BF16)
+    return fail(CSWATTN_ERR_INVALID_ARG, "dtype must be CSWATTN_F32 or CSWATTN_BF16");
+  if (L->T > kMaxT) return fail(CSWATTN_ERR_UNSUPPORTED, "T = %d exceeds %d", L->T, kMaxT);
+  const long long rows = static_cast<long long>(L->B) * L->T * L->n_head;
+  if (rows * L->head_dim >= (1ll << 40) || static_cast<long long>(L->B) * L->n_kv_head * 2048 >= (1ll << 31))
+    return fail(CSWATTN_ERR_UNSUPPORTED, "layer too large");
+  if (L->dtype == CSWATTN_BF16) {
+    if (L->head_dim != 128)
+      return fail(CSWATTN_ERR_UNSUPPORTED, "bf16 supports head_dim 128 only (got %d)", L->head_dim);
+  } else {
+    const int d = L->head_dim;
+    if (d != 4 && d != 8 && d != 16 && d != 32 && d != 64 && d != 128)
+      return fail(CSWATTN_ERR_UNSUPPORTED, "f32 supports head_dim 4, 8, 16, 32, 64, 128 (got %d)", d);
+  }
+  s->B = L->B;
+  s->T = L->T;
+  s->H = L->n_head;
+  s->Hk = L->n_kv_head;
+  s->D = L->head_dim;
+  s->W = L->window < L->T ? L->window : L->T;  // W >= T is plain causal
+  s->g = L->n_head / L->n_kv_head;
+  s->bf16 = L->dtype == CSWATTN_BF16;
+  s->esize = s->bf16 ? 2 : 4;
+  s->scale = L->softmax_scale > 0.f ? L->softmax_scale : 1.0f / std::sqrt(static_cast<float>(L->head_dim));
+  return CSWATTN_OK;
+}
+
+cswattn_status check_ptr(const void* p, const char* name, size_t align) {
+  if (!p) return fail(CSWATTN_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(CSWATTN_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return CSWATTN_OK;
+}
+
+#define CHECK_PTR(p, a)                                          \
+  do {                                                           \
+    cswattn_status st_ = check_ptr((p), #p, (a));                \
+    if (st_ != CSWATTN_OK) return st_;                           \
+  } while (0)
+
+void fill_omega(float* omega, int D, float base) {
+  for (int i = 0; i < D / 2; ++i)
+    omega[i] = static_cast<float>(std::pow(static_cast<double>(base), -2.0 * i / D));
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+cswattn_status get_encoder(EncodeTiledFn* fn) {
+  static std::once_flag once;
+  static EncodeTiledFn cached = nullptr;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  if (!cached) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s", cudaGetErrorString(err));
+  *fn = cached;
+  return CSWATTN_OK;
+}
+
+// (B, T, heads, 128) bf16 tensor; box = 64 head_dim elements x `rows` tokens
+// of one head, 128-byte swizzle; out-of-range rows read as zero.
+cswattn_status make_map(CUtensorMap* map, const void* base, int B, int T, int heads, int rows) {
+  EncodeTiledFn enc;
+  cswattn_status s = get_encoder(&enc);
+  if (s != CSWATTN_OK) return s;
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(heads) * 256,
+                                 static_cast<cuuint64_t>(T) * heads * 256};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CSWATTN_OK;
+}
+
+template <typename Kernel>
+cswattn_status set_smem(Kernel k, int bytes, std::once_flag& flag, cudaError_t& err) {
+  std::call_once(flag, [&] {
+    err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+  if (err != cudaSuccess) return cuda_fail(err, "cudaFuncSetAttribute");
+  return CSWATTN_OK;
+}
+
+cswattn_status launched(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return CSWATTN_OK;
+}
+
+template <typename T>
+void launch_prologue(const Shape& s, const PrologueParams& pp, cudaStream_t st) {
+  const long long ntok = static_cast<long long>(s.B) * s.T;
+  const unsigned grid = static_cast<unsigned>((ntok + kPrologueTok - 1) / kPrologueTok);
+  switch (s.D) {
+    case 4: if constexpr (sizeof(T) == 4) prologue_kernel<T, 4><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 8: if constexpr (sizeof(T) == 4) prologue_kernel<T, 8><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 16: if constexpr (sizeof(T) == 4) prologue_kernel<T, 16><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 32: if constexpr (sizeof(T) == 4) prologue_kernel<T, 32><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 64: if constexpr (sizeof(T) == 4) prologue_kernel<T, 64><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    default: prologue_kernel<T, 128><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+  }
+}
+
+template <typename T>
+void launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t st) {
+  const long long ntok = static_cast<long long>(s.B) * s.T;
+  const unsigned grid = static_cast<unsigned>((ntok + kPrologueTok - 1) / kPrologueTok);
+  switch (s.D) {
+    case 4: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 4><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+    case 8: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 8><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+    case 16: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 16><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+    case 32: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 32><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+    case 64: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 64><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+    default: epilogue_kernel<T, 128><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+  }
+}
+
+template <typename T>
+void launch_preprocess(const Shape& s, const PreParams& pp, cudaStream_t st) {
+  const int lpr = s.D / Vec16<T>::N;
+  const long long rows_per_block = 256 / lpr;
+  long long blocks = (pp.rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  const unsigned grid = static_cast<unsigned>(blocks);
+  switch (s.D) {
+    case 4: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 4><<<grid, 256, 0, st>>>(pp); break;
+    case 8: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 8><<<grid, 256, 0, st>>>(pp); break;
+    case 16: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 16><<<grid, 256, 0, st>>>(pp); break;
+    case 32: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 32><<<grid, 256, 0, st>>>(pp); break;
+    case 64: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 64><<<grid, 256, 0, st>>>(pp); break;
+    default: preprocess_kernel<T, 128><<<grid, 256, 0, st>>>(pp); break;
+  }
+}
+
+void launch_simt_fwd(const Shape& s, const SimtParams& sp, cudaStream_t st) {
+  const long long rows = static_cast<long long>(s.B) * s.H * s.T;
+  const unsigned grid = static_cast<unsigned>((rows + 127) / 128);
+  switch (s.D) {
+    case 4: simt_fwd_kernel<4><<<grid, 128, 0, st>>>(sp); break;
+    case 8: simt_fwd_kernel<8><<<grid, 128, 0, st>>>(sp); break;
+    case 16: simt_fwd_kernel<16><<<grid, 128, 0, st>>>(sp); break;
+    case 32: simt_fwd_kernel<32><<<grid, 128, 0, st>>>(sp); break;
+    case 64: simt_fwd_kernel<64><<<grid, 128, 0, st>>>(sp); break;
+    default: simt_fwd_kernel<128><<<grid, 128, 0, st>>>(sp); break;
+  }
+}
+
+void launch_simt_bwd(const Shape& s, const SimtParams& sp, cudaStream_t st) {
+  const long long qrows = static_cast<long long>(s.B) * s.H * s.T;
+  const long long krows = static_cast<long long>(s.B) * s.Hk * s.T;
+  const unsigned gq = static_cast<unsigned>((qrows + 127) / 128);
+  const unsigned gk = static_cast<unsigned>((krows + 127) / 128);
+  switch (s.D) {
+#define CSW_CASE(DD)                                        \
+  case DD:                                                  \
+    simt_bwd_dq_kernel<DD><<<gq, 128, 0, st>>>(sp);         \
+    simt_bwd_dkv_kernel<DD><<<gk, 128, 0, st>>>(sp);        \
+    break;
+    CSW_CASE(4)
+    CSW_CASE(8)
+    CSW_CASE(16)
+    CSW_CASE(32)
+    CSW_CASE(64)
+    default:
+      simt_bwd_dq_kernel<128><<<gq, 128, 0, st>>>(sp);
+      simt_bwd_dkv_kernel<128><<<gk, 128, 0, st>>>(sp);
+      break;
+#undef CSW_CASE
+  }
+}
+
+// ---------------------------------------------------------------- timing
+
+std::atomic<int> g_timing{0};
+std::mutex g_timing_mu;
+struct EventPair {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int kind = 0;
+};
+std::vector<EventPair> g_pool;   // created once, reused
+size_t g_used = 0;
+
+// Records a start event for `kind` when timing is on; returns the pair index
+// (or -1). Call timing_end(idx) after the launch.
+long timing_begin(int kind, cudaStream_t st) {
+  if (!g_timing.load()) return -1;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  if (g_used == g_pool.size()) {
+    EventPair e;
+    if (cudaEventCreate(&e.a) != cudaSuccess || cudaEventCreate(&e.b) != cudaSuccess) return -1;
+    g_pool.push_back(e);
+  }
+  EventPair& e = g_pool[g_used];
+  e.kind = kind;
+  if (cudaEventRecord(e.a, st) != cudaSuccess) return -1;
+  return static_cast<long>(g_used++);
+}
+
+void timing_end(long idx, cudaStream_t st) {
+  if (idx < 0) return;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  cudaEventRecord(g_pool[static_cast<size_t>(idx)].b, st);
+}
+
+struct ScopedTiming {
+  long idx;
+  cudaStream_t st;
+  ScopedTiming(int kind, cudaStream_t s) : idx(timing_begin(kind, s)), st(s) {}
+  ~ScopedTiming() { timing_end(idx, st); }
+};
+
+size_t pad256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Workspace {
+  float *dq_acc, *dk_acc, *dv_acc, *delta;
+  size_t bytes;
+};
+
+Workspace carve(const Shape& s, void* base) {
+  const size_t nq = static_cast<size_t>(s.B) * s.H * s.T * s.D;
+  const size_t nk = static_cast<size_t>(s.B) * s.T * s.Hk * s.D;
+  const size_t nr = static_cast<size_t>(s.B) * s.H * s.T;
+  Workspace w;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  w.dq_acc = reinterpret_cast<float*>(p + off);
+  off += pad256(nq * 4);
+  w.dk_acc = reinterpret_cast<float*>(p + off);
+  off += pad256(nk * 4);
+  w.dv_acc = reinterpret_cast<float*>(p + off);
+  off += pad256(nk * 4);
+  w.delta = reinterpret_cast<float*>(p + off);
+  off += pad256(nr * 4);
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int cswattn_version(void) { return (1 << 16) | 0; }
+
+const char* cswattn_last_error(void) { return t_err.c_str(); }
+
+void cswattn_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns < 1000 ? 1000 : ns); }
+
+void cswattn_set_timing(int enable) { g_timing.store(enable ? 1 : 0); }
+
+cswattn_status cswattn_kernel_times(double* ms, int* launches) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  double acc[CSWATTN_NUM_KERNELS] = {0};
+  int cnt[CSWATTN_NUM_KERNELS] = {0};
+  cswattn_status st = CSWATTN_OK;
+  for (size_t i = 0; i < g_used; ++i) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(g_pool[i].b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, g_pool[i].a, g_pool[i].b);
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "cudaEventElapsedTime");
+      continue;
+    }
+    acc[g_pool[i].kind] += t;
+    cnt[g_pool[i].kind] += 1;
+  }
+  g_used = 0;
+  for (int k = 0; k < CSWATTN_NUM_KERNELS; ++k) {
+    if (ms) ms[k] = acc[k];
+    if (launches) launches[k] = cnt[k];
+  }
+  return st;
+}
+
+cswattn_status cswattn_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+  if (v != 0) {
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    if (v & kStatusTimeout) return fail(CSWATTN_ERR_TIMEOUT, "a device-side wait ran out (status 0x%x)", v);
+  }
+  return CSWATTN_OK;
+}
+
+cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const void* k,
+                             const void* v, const void* ve, const void* gate, void* q_out,
+                             void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                             void* stream) {
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(k, 16);
+  CHECK_PTR(v, 16);
+  CHECK_PTR(q_out, 16);
+  CHECK_PTR(k_out, 16);
+  CHECK_PTR(v_out, 16);
+  CHECK_PTR(rstd_q, 4);
+  CHECK_PTR(rstd_k, 4);
+  if (layer->has_ve) {
+    CHECK_PTR(ve, 16);
+    CHECK_PTR(gate, s.esize);
+  }
+  if (q_out == q || k_out == k || v_out == v || q_out == k_out || k_out == v_out || q_out == v_out)
+    return fail(CSWATTN_ERR_INVALID_ARG, "prologue outputs must not alias its inputs or each other");
+  PrologueParams pp;
+  pp.B = s.B;
+  pp.T = s.T;
+  pp.H = s.H;
+  pp.Hk = s.Hk;
+  pp.has_ve = layer->has_ve;
+  pp.eps = layer->eps;
+  fill_omega(pp.omega, s.D, layer->rope_base);
+  pp.q = q;
+  pp.k = k;
+  pp.v = v;
+  pp.ve = ve;
+  pp.gate = gate;
+  pp.q_out = q_out;
+  pp.k_out = k_out;
+  pp.v_out = v_out;
+  pp.rstd_q = rstd_q;
+  pp.rstd_k = rstd_k;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  {
+    ScopedTiming tm(CSWATTN_K_PROLOGUE, cs);
+    if (s.bf16)
+      launch_prologue<__nv_bfloat16>(s, pp, cs);
+    else
+      launch_prologue<float>(s, pp, cs);
+  }
+  return launched("prologue launch");
+}
+
+cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const void* k_out,
+                        const void* v_out, void* O, float* lse, void* stream) {
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  CHECK_PTR(q_out, 16);
+  CHECK_PTR(k_out, 16);
+  CHECK_PTR(v_out, 16);
+  CHECK_PTR(O, 16);
+  CHECK_PTR(lse, 4);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (!s.bf16) {
+    SimtParams sp{};
+    sp.B = s.B;
+    sp.T = s.T;
+    sp.H = s.H;
+    sp.Hk = s.Hk;
+    sp.W = s.W;
+    sp.scale = s.scale;
+    sp.q = static_cast<const float*>(q_out);
+    sp.k = static_cast<const float*>(k_out);
+    sp.v = static_cast<const float*>(v_out);
+    sp.out_O = static_cast<float*>(O);
+    sp.out_lse = lse;
+    {
+      ScopedTiming tm(CSWATTN_K_FWD, cs);
+      launch_simt_fwd(s, sp, cs);
+    }
+    return launched("fp32 forward launch");
+  }
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q_out, s.B, s.T, s.H, fwd::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, fwd::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, fwd::kBM)) != CSWATTN_OK) return st;
+  static std::once_flag flag;
+  static cudaError_t ferr;
+  if ((st = set_smem(fwd::fwd_kernel, fwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
+  fwd::Params fp;
+  fp.B = s.B;
+  fp.T = s.T;
+  fp.H = s.H;
+  fp.Hk = s.Hk;
+  fp.W = s.W;
+  fp.g = s.g;
+  fp.nq = (s.T + fwd::kBM - 1) / fwd::kBM;
+  fp.npairs = (fp.nq * s.g + 1) / 2;
+  fp.scale_log2 = s.scale * 1.4426950408889634f;
+  fp.O = static_cast<__nv_bfloat16*>(O);
+  fp.lse = lse;
+  fp.wait_ns = g_wait_ns.load();
+  const unsigned grid = static_cast<unsigned>(fp.npairs) * s.B * s.Hk;
+  {
+    ScopedTiming tm(CSWATTN_K_FWD, cs);
+    fwd::fwd_kernel<<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, fp);
+  }
+  return launched("forward launch");
+}
+
+size_t attn_bwd_workspace_bytes(const cswattn_layer* layer) {
+  Shape s;
+  if (check_layer(layer, &s) != CSWATTN_OK) return 0;
+  return carve(s, nullptr).bytes;
+}
+
+cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k,
+                        const void* ve, const void* gate, const void* q_out,
+                        const void* k_out, const void* v_out, const float* rstd_q,
+                        const float* rstd_k, const void* O, const float* lse, const void* dO,
+                        void* dQ, void* dK, void* dV, void* dve, void* dgate, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(k, 16);
+  CHECK_PTR(q_out, 16);
+  CHECK_PTR(k_out, 16);
+  CHECK_PTR(v_out, 16);
+  CHECK_PTR(rstd_q, 4);
+  CHECK_PTR(rstd_k, 4);
+  CHECK_PTR(O, 16);
+  CHECK_PTR(lse, 4);
+  CHECK_PTR(dO, 16);
+  CHECK_PTR(dQ, 16);
+  CHECK_PTR(dK, 16);
+  CHECK_PTR(dV, 16);
+  CHECK_PTR(workspace, 256);
+  if (layer->has_ve) {
+    CHECK_PTR(ve, 16);
+    CHECK_PTR(gate, s.esize);
+    CHECK_PTR(dve, 16);
+    CHECK_PTR(dgate, s.esize);
+  }
+  const Workspace w = carve(s, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CSWATTN_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+  // Delta = rowsum(dO * O)
+  PreParams pre;
+  pre.rows = static_cast<long long>(s.B) * s.T * s.H;
+  pre.T = s.T;
+  pre.H = s.H;
+  pre.O = O;
+  pre.dO = dO;
+  pre.delta = w.delta;
+  {
+    ScopedTiming tm(CSWATTN_K_BWD_PRE, cs);
+    if (s.bf16)
+      launch_preprocess<__nv_bfloat16>(s, pre, cs);
+    else
+      launch_preprocess<float>(s, pre, cs);
+  }
+  if ((st = launched("preprocess launch")) != CSWATTN_OK) return st;
+
+  if (!s.bf16) {
+    SimtParams sp{};
+    sp.B = s.B;
+    sp.T = s.T;
+    sp.H = s.H;
+    sp.Hk = s.Hk;
+    sp.W = s.W;
+    sp.scale = s.scale;
+    sp.q = static_cast<const float*>(q_out);
+    sp.k = static_cast<const float*>(k_out);
+    sp.v = static_cast<const float*>(v_out);
+    sp.O = static_cast<const float*>(O);
+    sp.dO = static_cast<const float*>(dO);
+    sp.lse = lse;
+    sp.delta = w.delta;
+    sp.dq_acc = w.dq_acc;
+    sp.dk_acc = w.dk_acc;
+    sp.dv_acc = w.dv_acc;
+    {
+      ScopedTiming tm(CSWATTN_K_BWD, cs);
+      launch_simt_bwd(s, sp, cs);
+    }
+    if ((st = launched("fp32 backward launch")) != CSWATTN_OK) return st;
+  } else {
+    const size_t dq_bytes = static_cast<size_t>(s.B) * s.H * s.T * s.D * 4;
+    cudaError_t e = cudaMemsetAsync(w.dq_acc, 0, dq_bytes, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    CUtensorMap mq, mdo, mk, mv;
+    if ((st = make_map(&mq, q_out, s.B, s.T, s.H, bwd::kBQ)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdo, dO, s.B, s.T, s.H, bwd::kBQ)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, bwd::kBN)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, bwd::kBN)) != CSWATTN_OK) return st;
+    static std::once_flag flag;
+    static cudaError_t ferr;
+    if ((st = set_smem(bwd::bwd_kernel, bwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
+    bwd::Params bp;
+    bp.B = s.B;
+    bp.T = s.T;
+    bp.H = s.H;
+    bp.Hk = s.Hk;
+    bp.W = s.W;
+    bp.g = s.g;
+    bp.nkv = (s.T + bwd::kBN - 1) / bwd::kBN;
+    bp.scale_log2 = s.scale * 1.4426950408889634f;
+    bp.scale = s.scale;
+    bp.lse = lse;
+    bp.delta = w.delta;
+    bp.dq_acc = w.dq_acc;
+    bp.dk_acc = w.dk_acc;
+    bp.dv_acc = w.dv_acc;
+    bp.wait_ns = g_wait_ns.load();
+    const unsigned grid = static_cast<unsigned>(bp.nkv) * s.B * s.Hk;
+    {
+      ScopedTiming tm(CSWATTN_K_BWD, cs);
+      bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, bp);
+    }
+    if ((st = launched("backward launch")) != CSWATTN_OK) return st;
+  }
+
+  EpiParams ep;
+  ep.B = s.B;
+  ep.T = s.T;
+  ep.H = s.H;
+  ep.Hk = s.Hk;
+  ep.has_ve = layer->has_ve;
+  fill_omega(ep.omega, s.D, layer->rope_base);
+  ep.q = q;
+  ep.k = k;
+  ep.ve = ve;
+  ep.gate = gate;
+  ep.rstd_q = rstd_q;
+  ep.rstd_k = rstd_k;
+  ep.dq_acc = w.dq_acc;
+  ep.dk_acc = w.dk_acc;
+  ep.dv_acc = w.dv_acc;
+  ep.dq = dQ;
+  ep.dk = dK;
+  ep.dv = dV;
+  ep.dve = dve;
+  ep.dgate = dgate;
+  {
+    ScopedTiming tm(CSWATTN_K_BWD_EPI, cs);
+    if (s.bf16)
+      launch_epilogue<__nv_bfloat16>(s, ep, cs);
+    else
+      launch_epilogue<float>(s, ep, cs);
+  }
+  return launched("epilogue launch");
+}
+
+}  // extern "C"

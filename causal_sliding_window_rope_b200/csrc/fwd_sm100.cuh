@@ -1,0 +1,361 @@
+// fwd_sm100.cuh -- attention forward on tcgen05 tensor cores (bf16, D = 128).
+//
+// Computes O_i = sum_j softmax_j(c q~_i . k~_j) v_eff_j over the causal
+// sliding window (i - W < j <= i) and the row log-sum-exp, the attention
+// call of the page "5만원으로 나만의 ChatGPT 훈련하는 방법", section
+// "5. 플래시 어텐션 통합 (nanochat/flash_attention.py)", with the window of
+// the architecture list's "sliding window attention" and its GQA.
+//
+// Work unit (one CTA): two 128-row query tiles of the same (batch, KV head)
+// that share every K/V tile staged in shared memory. Tiles of a (b, KV head)
+// are ordered (query block, head within the group) and paired in that order,
+// so for group size >= 2 a unit holds two heads of the group at the same
+// query block (identical KV range) and for group size 1 two consecutive
+// query blocks (the union of their ranges; each tile skips the KV tiles
+// outside its own range). Only KV tiles inside [first window key, diagonal]
+// are loaded and multiplied; masks are applied on the diagonal and
+// window-edge tiles only.
+//
+// Roles (12 warps):
+//   warp 0      TMA producer: Q tiles once, then K_j, V_j through 2-stage rings
+//   warp 1      TMEM owner + single-thread MMA issuer
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r
+//               owns TMEM lane r = query row r, so the row max and sum are
+//               in-thread; P goes back to TMEM as bf16 over the S columns
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
+// Per KV tile: S_X = Q_X K_j^T (SS MMA, K-major both), softmax -> P_X,
+// O_X += P_X V_j (TS MMA: P from TMEM, V MN-major from shared memory).
+// The MMA order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) lets one tile's softmax
+// overlap the other tile's matrix products. O is rescaled lazily: only when
+// a row's max grows by more than 2^8 (in exp2 units).
+#pragma once
+#include "common.cuh"
+
+namespace cswattn {
+namespace fwd {
+
+constexpr int kBM = 128;
+constexpr int kD = 128;
+constexpr int kThreads = 384;
+constexpr int kTileBytes = kBM * kD * 2;     // 32 KB: 128 rows x 128 bf16
+constexpr int kPanelBytes = kTileBytes / 2;  // 16 KB: 128 rows x 64 bf16 (one swizzle panel)
+constexpr int kOffQ = 0;                     // 2 tiles
+constexpr int kOffK = 2 * kTileBytes;        // 2 stages
+constexpr int kOffV = 4 * kTileBytes;        // 2 stages
+constexpr int kOffBar = 6 * kTileBytes;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+struct Params {
+  int B, T, H, Hk, W, g, nq, npairs;
+  float scale_log2;  // softmax scale * log2(e)
+  __nv_bfloat16* O;
+  float* lse;
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Waits for a phase without looking at the abort flag (used to drain
+// in-flight copies and MMAs before the CTA exits). Bounded by `ns`.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > ns) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] per tile
+  uint64_t* p_full = bars + 11;   // [2] per tile
+  uint64_t* o_full = bars + 13;   // [2] per tile
+  uint64_t* mma_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+
+  const int warp = warp_id(), lane = lane_id();
+
+  // ---- work unit: heavy (late query blocks) first
+  const int BHk = p.B * p.Hk;
+  const int pr = p.npairs - 1 - static_cast<int>(blockIdx.x) / BHk;
+  const int bh = static_cast<int>(blockIdx.x) % BHk;
+  const int b = bh / p.Hk, hk = bh % p.Hk;
+  const int ntiles = p.nq * p.g;
+  int qblk[2], head[2], lo_t[2], hi_t[2];
+  bool valid[2];
+#pragma unroll
+  for (int X = 0; X < 2; ++X) {
+    int t = 2 * pr + X;
+    valid[X] = t < ntiles;
+    if (!valid[X]) t = 2 * pr;
+    qblk[X] = t / p.g;
+    head[X] = hk * p.g + t % p.g;
+    const int q0 = qblk[X] * kBM;
+    lo_t[X] = max(0, q0 - p.W + 1) / kBM;
+    hi_t[X] = qblk[X];
+  }
+  const int lo = valid[1] ? min(lo_t[0], lo_t[1]) : lo_t[0];
+  const int hi = valid[1] ? max(hi_t[0], hi_t[1]) : hi_t[0];
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&o_full[s], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.wait_ns};
+
+  const uint32_t colS[2] = {0u, 128u};
+  const uint32_t colO[2] = {256u, 384u};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int nk[2] = {0, 0}, nv[2] = {0, 0};
+      mbar_expect_tx(q_full, (valid[1] ? 2 : 1) * kTileBytes);
+      for (int X = 0; X < 2; ++X) {
+        if (!valid[X]) continue;
+        uint8_t* dst = smem + kOffQ + X * kTileBytes;
+        tma_load_4d(&tmQ, q_full, dst, 0, head[X], qblk[X] * kBM, b);
+        tma_load_4d(&tmQ, q_full, dst + kPanelBytes, 64, head[X], qblk[X] * kBM, b);
+      }
+      for (int j = lo; j <= hi; ++j) {
+        const int it = j - lo, s = it & 1, use = it >> 1;
+        if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, wc)) break;
+        mbar_expect_tx(&k_full[s], kTileBytes);
+        uint8_t* kd = smem + kOffK + s * kTileBytes;
+        tma_load_4d(&tmK, &k_full[s], kd, 0, hk, j * kBM, b);
+        tma_load_4d(&tmK, &k_full[s], kd + kPanelBytes, 64, hk, j * kBM, b);
+        ++nk[s];
+        if (use > 0 && !mbar_wait(&v_empty[s], (use - 1) & 1, wc)) break;
+        mbar_expect_tx(&v_full[s], kTileBytes);
+        uint8_t* vd = smem + kOffV + s * kTileBytes;
+        tma_load_4d(&tmV, &v_full[s], vd, 0, hk, j * kBM, b);
+        tma_load_4d(&tmV, &v_full[s], vd + kPanelBytes, 64, hk, j * kBM, b);
+        ++nv[s];
+      }
+      // Drain: every issued copy has landed before the CTA may exit.
+      drain_wait(q_full, 0, p.wait_ns);
+      for (int s = 0; s < 2; ++s) {
+        if (nk[s] > 0) drain_wait(&k_full[s], (nk[s] - 1) & 1, p.wait_ns);
+        if (nv[s] > 0) drain_wait(&v_full[s], (nv[s] - 1) & 1, p.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
+      constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // P V: V MN-major
+      const uint32_t sQa = smem_u32(smem + kOffQ);
+      const uint32_t sKa = smem_u32(smem + kOffK);
+      const uint32_t sVa = smem_u32(smem + kOffV);
+      bool ok = mbar_wait(q_full, 0, wc);
+      tc_fence_after();
+
+      auto issue_S = [&](int X, int j) -> bool {
+        const int it = j - lo, s = it & 1, use = it >> 1;
+        if (!mbar_wait(&k_full[s], use & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t qa = sQa + X * kTileBytes, ka = sKa + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
+          mma_ss(tmem + colS[X], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                 idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[X]);
+        return true;
+      };
+      auto issue_PV = [&](int X, int j) -> bool {
+        const int it = j - lo, s = it & 1, use = it >> 1;
+        const int n = j - lo_t[X];
+        if (!mbar_wait(&v_full[s], use & 1, wc)) return false;
+        if (!mbar_wait(&p_full[X], n & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t va = sVa + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_ts(tmem + colO[X], tmem + colS[X] + kk * 8,
+                 sdesc_sw128(va + kk * 2048, kPanelBytes, 1024), idPV,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        return true;
+      };
+
+      if (ok) {
+        for (int X = 0; X < 2 && ok; ++X)
+          if (valid[X] && lo_t[X] == lo) ok = issue_S(X, lo);
+        if (ok) mma_commit(&k_empty[0]);
+      }
+      for (int j = lo; ok && j <= hi; ++j) {
+        const int it = j - lo;
+        for (int X = 0; X < 2 && ok; ++X) {
+          if (!valid[X]) continue;
+          if (j >= lo_t[X] && j <= hi_t[X]) {
+            ok = issue_PV(X, j);
+            if (ok && j == hi_t[X]) mma_commit(&o_full[X]);
+          }
+          if (ok && j + 1 >= lo_t[X] && j + 1 <= hi_t[X]) ok = issue_S(X, j + 1);
+        }
+        if (!ok) break;
+        mma_commit(&v_empty[it & 1]);
+        if (j + 1 <= hi) mma_commit(&k_empty[(it + 1) & 1]);
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      mma_commit(mma_done);
+      drain_wait(mma_done, 0, p.wait_ns);
+    }
+  } else if (warp >= 4) {
+    // -------------------------------------------------- softmax + epilogue
+    const int X = (warp - 4) >> 2;
+    if (valid[X]) {
+      const int r = (warp & 3) * 32 + lane;  // TMEM lane = query row in the tile
+      const int q0 = qblk[X] * kBM;
+      const int qi = q0 + r;
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t tS = tmem + lane_off + colS[X];
+      const uint32_t tO = tmem + lane_off + colO[X];
+      const float c2 = p.scale_log2;
+      float m2 = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = lo_t[X]; j <= hi_t[X]; ++j) {
+        const int n = j - lo_t[X];
+        const bool got = mbar_wait(&s_full[X], n & 1, wc);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv[c]);
+        tmem_ld_wait();
+        const int k0 = j * kBM;
+        if (k0 + kBM - 1 > q0 || q0 + kBM - 1 - k0 >= p.W) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int kj = k0 + c * 32 + i;
+              if (kj > qi || qi - kj >= p.W) sv[c][i] = __float_as_uint(-INFINITY);
+            }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+        mx *= c2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (n == 0) {
+          m2 = mx;
+        } else if (mx > m2 + kRescaleThreshold) {
+          alpha = ex2(m2 - mx);
+          m2 = mx;
+          rescale = true;
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + c * 32, o);
+          }
+          tmem_st_wait();
+        }
+        l *= alpha;
+        const float mu = (m2 == -INFINITY) ? 0.f : m2;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -mu));
+            const float p1 = ex2(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -mu));
+            l += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[X]);
+      }
+      const bool o_ok = ok && mbar_wait(&o_full[X], 0, wc);
+      if (__all_sync(0xffffffffu, o_ok)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool row_ok = qi < p.T;
+        __nv_bfloat16* orow =
+            p.O + ((static_cast<size_t>(b) * p.T + (row_ok ? qi : 0)) * p.H + head[X]) * kD;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait();
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+              dst[v4] = w;
+            }
+          }
+        }
+        if (row_ok)
+          p.lse[(static_cast<size_t>(b) * p.H + head[X]) * p.T + qi] =
+              (m2 + log2f(l)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+}  // namespace cswattn

@@ -1,0 +1,163 @@
+/*
+ * cswattn.h -- C ABI of the causal sliding-window RoPE attention library
+ * (libcswattn.so), built for NVIDIA B200 (sm_100a).
+ *
+ * The library computes one attention layer of a nanochat-style GPT block,
+ * forward and backward, as described on the page
+ * "5만원으로 나만의 ChatGPT 훈련하는 방법" (apidog.com):
+ *   - section "1. GPT 모델 (nanochat/gpt.py)", architecture list: rotary
+ *     position embeddings (RoPE), QK normalisation, grouped-query attention
+ *     (fewer KV heads than query heads) and sliding-window attention with a
+ *     per-layer pattern such as "SSSL";
+ *   - same section, "값 임베딩 (Value Embeddings, ResFormer)": the value
+ *     embedding is viewed per KV head and mixed in as v + 3*sigmoid(gate)*ve;
+ *   - section "5. 플래시 어텐션 통합 (nanochat/flash_attention.py)": the
+ *     attention is a causal call with a window size on (B, T, H, D) tensors.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout: all tensors are dense row-major, head_dim contiguous:
+ *   q, q_out, O, dO, dQ          (B, T, n_head, head_dim)
+ *   k, v, ve, k_out, v_out,
+ *   dK, dV, dve                  (B, T, n_kv_head, head_dim)
+ *   gate, dgate                  (B, T, n_kv_head)
+ *   rstd_q                       (B, T, n_head)       float32
+ *   rstd_k                       (B, T, n_kv_head)    float32
+ *   lse                          (B, n_head, T)       float32, natural log
+ * Element type: layer->dtype for every tensor except rstd and lse (float32).
+ * Query head h reads KV head h / (n_head / n_kv_head).
+ * Window: a query at position i sees keys j with i - window < j <= i, itself
+ * included; window >= T is plain causal attention, window = 1 sees itself.
+ * RoPE: pairs (i, i + head_dim/2) rotated by angle t * rope_base^(-2i/head_dim),
+ * positions t = 0 .. T-1. RMSNorm: x * (mean(x^2) + eps)^(-1/2), no weight.
+ *
+ * Ownership: every pointer is caller-owned device memory (except where a
+ * function says host). The library allocates no device memory; the backward's
+ * scratch is the caller's `workspace`. Pointers to element tensors must be
+ * 16-byte aligned; rstd/lse/gate pointers 4-byte (2-byte for bf16 gate).
+ * Streams: every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and returns once the work is enqueued.
+ * Errors: arguments are validated on the host before anything is enqueued;
+ * a rejected call returns CSWATTN_ERR_INVALID_ARG or CSWATTN_ERR_UNSUPPORTED
+ * and enqueues nothing. A failed launch returns CSWATTN_ERR_CUDA. Device-side
+ * waits are bounded: a kernel whose wait runs out records CSWATTN_ERR_TIMEOUT
+ * in a device status word and returns; cswattn_sync_status() reports it.
+ * cswattn_last_error() gives a message for the last failure on this thread.
+ */
+#ifndef CSWATTN_H
+#define CSWATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSWATTN_OK = 0,
+  CSWATTN_ERR_INVALID_ARG = 1,
+  CSWATTN_ERR_UNSUPPORTED = 2,
+  CSWATTN_ERR_CUDA = 3,
+  CSWATTN_ERR_TIMEOUT = 4
+} cswattn_status;
+
+typedef enum { CSWATTN_F32 = 0, CSWATTN_BF16 = 1 } cswattn_dtype;
+
+/* Shape of one attention layer. Supported: bf16 with head_dim 128 (tensor
+ * cores), f32 with head_dim in {4, 8, 16, 32, 64, 128} (CUDA cores, fp32
+ * throughout). n_head % n_kv_head == 0, window >= 1, T <= 2^20. */
+typedef struct {
+  int B, T, n_head, n_kv_head, head_dim;
+  int window;          /* keys visible to a query, itself included */
+  float rope_base;     /* > 0; 10000 in the d12/d24 workloads */
+  float eps;           /* >= 0; RMSNorm epsilon inside the square root */
+  float softmax_scale; /* > 0, or 0 for 1/sqrt(head_dim) */
+  int has_ve;          /* 1: the value embedding and its gate are present */
+  cswattn_dtype dtype;
+} cswattn_layer;
+
+/* Prologue: q_out = RoPE(RMSNorm(q)), k_out = RoPE(RMSNorm(k)),
+ * v_out = v + 3*sigmoid(gate)*ve (v_out = v when has_ve == 0), and the
+ * RMSNorm factors rstd_q = (mean(q^2)+eps)^(-1/2), rstd_k likewise.
+ * Page sections "1. GPT 모델" (architecture list; value-embedding code).
+ * ve and gate are read only when has_ve and may be NULL otherwise.
+ * Outputs must not alias inputs. */
+cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const void* k,
+                             const void* v, const void* ve, const void* gate,
+                             void* q_out, void* k_out, void* v_out, float* rstd_q,
+                             float* rstd_k, void* stream);
+
+/* Forward: O_i = sum_j softmax_j(scale * q_out_i . k_out_j) v_out_j over the
+ * causal window, and lse_i = log sum_j exp(scale * q_out_i . k_out_j).
+ * Page section "5. 플래시 어텐션 통합" (causal call with window_size).
+ * Inputs are the prologue's outputs. */
+cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const void* k_out,
+                        const void* v_out, void* O, float* lse, void* stream);
+
+/* Bytes of device scratch attn_bwd needs for this layer: float32
+ * accumulators of dq_out (B, n_head, T, head_dim), dk_out and dv_out
+ * (B, T, n_kv_head, head_dim) and the row terms dO.O (B, n_head, T),
+ * each padded to 256 bytes. Returns 0 for an invalid layer. */
+size_t attn_bwd_workspace_bytes(const cswattn_layer* layer);
+
+/* Backward of prologue + forward for the loss L with dL/dO = dO:
+ * dQ, dK (through RoPE^-1 and RMSNorm), dV = dL/dv_out, and when has_ve
+ * dve = 3*sigmoid(gate)*dV and dgate = 3*sigmoid(gate)*(1-sigmoid(gate)) *
+ * sum_d dV*ve. q, k, ve, gate are the prologue's inputs; q_out, k_out, v_out,
+ * rstd_q, rstd_k its outputs; O and lse the forward's outputs.
+ * workspace: caller-owned device scratch of at least
+ * attn_bwd_workspace_bytes(layer) bytes, 256-byte aligned, whose contents on
+ * entry do not matter; it must not be used by another call in flight.
+ * dve and dgate are written only when has_ve (may be NULL otherwise). */
+cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k,
+                        const void* ve, const void* gate, const void* q_out,
+                        const void* k_out, const void* v_out, const float* rstd_q,
+                        const float* rstd_k, const void* O, const float* lse,
+                        const void* dO, void* dQ, void* dK, void* dV, void* dve,
+                        void* dgate, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Waits for `stream`, then returns and clears the device status word of the
+ * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
+ * since the last check, CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
+cswattn_status cswattn_sync_status(void* stream);
+
+/* Upper bound, in nanoseconds, of every device-side wait of later launches
+ * (default 2e9). Values below 1000 are raised to 1000. Process-wide. */
+void cswattn_set_wait_limit_ns(uint64_t ns);
+
+/* Kernel kinds reported by cswattn_kernel_times(). */
+enum {
+  CSWATTN_K_PROLOGUE = 0, /* fused RMSNorm + RoPE + value residual */
+  CSWATTN_K_FWD = 1,      /* attention forward (tensor cores, or fp32 CUDA cores) */
+  CSWATTN_K_BWD_PRE = 2,  /* backward row terms Delta = rowsum(dO * O) */
+  CSWATTN_K_BWD = 3,      /* attention backward main kernel(s) */
+  CSWATTN_K_BWD_EPI = 4,  /* backward epilogue: RoPE^-1, RMSNorm', dv/dve/dgate */
+  CSWATTN_NUM_KERNELS = 5
+};
+
+/* Per-kernel device timing for measurement tools. With enable != 0, every
+ * later call records a CUDA event pair around each kernel it launches, on the
+ * caller's stream (events are created once and reused; no device memory is
+ * allocated). Process-wide; off by default. */
+void cswattn_set_timing(int enable);
+
+/* Waits for the recorded event pairs, writes the summed milliseconds and the
+ * launch count of each kernel kind into ms[CSWATTN_NUM_KERNELS] and
+ * launches[CSWATTN_NUM_KERNELS] (host arrays, either may be NULL), and clears
+ * the record. Returns CSWATTN_ERR_CUDA if an event query fails. */
+cswattn_status cswattn_kernel_times(double* ms, int* launches);
+
+/* Message for the last failed call on this thread ("" if none). The string
+ * is owned by the library and valid until the next call on this thread. */
+const char* cswattn_last_error(void);
+
+/* Library ABI version, (major << 16) | minor. */
+int cswattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSWATTN_H */

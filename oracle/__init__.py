@@ -125,6 +125,8 @@ def prologue(L: Layer, q, k, v, ve=None, gate=None):
     lib = _get()
     sq, skv = (L.B, L.T, L.H, L.D), (L.B, L.T, L.Hk, L.D)
     q, k, v = _f64(q, sq), _f64(k, skv), _f64(v, skv)
+    if L.has_ve and (ve is None or gate is None):
+        raise ValueError("has_ve layer needs ve and gate")
     ve = _f64(ve, skv) if L.has_ve else None
     gate = _f64(gate, (L.B, L.T, L.Hk)) if L.has_ve else None
     qt, kt, veff = np.empty(sq), np.empty(skv), np.empty(skv)
@@ -188,6 +190,8 @@ def prologue_bwd(L: Layer, q, k, ve, gate, dqt, dkt, dveff):
     """dQ, dK, dV, dve, dgate (dve/dgate are None without a value embedding)."""
     lib = _get()
     q, k, dqt, dkt, dveff = (_f64(a) for a in (q, k, dqt, dkt, dveff))
+    if L.has_ve and (ve is None or gate is None):
+        raise ValueError("has_ve layer needs ve and gate")
     ve = _f64(ve) if L.has_ve else None
     gate = _f64(gate) if L.has_ve else None
     dq, dk, dv = np.empty(q.shape), np.empty(k.shape), np.empty(k.shape)

@@ -1,0 +1,108 @@
+"""C ABI checks that need no GPU: the library loads, exports what the header
+declares, and rejects bad arguments on the host with the documented codes
+before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import causal_sliding_window_rope_b200 as cs
+from causal_sliding_window_rope_b200 import build as cs_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "cswattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    cs_build.build()
+    return cs.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:cswattn_status|size_t|void|const char\s*\*|int)\s+(\w+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(cs.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version(lib):
+    assert cs.cswattn_version() >> 16 == 1
+
+
+def call_fwd(spec, ptrs=(16, 32, 48, 64, 80)):
+    layer = spec.c() if spec is not None else None
+    ref = ctypes.byref(layer) if layer is not None else None
+    return cs.lib().attn_fwd(ref, *ptrs, None)
+
+
+@pytest.mark.parametrize("change,code", [
+    (dict(B=0), cs.ERR_INVALID_ARG),
+    (dict(T=0), cs.ERR_INVALID_ARG),
+    (dict(window=0), cs.ERR_INVALID_ARG),
+    (dict(n_kv_head=3), cs.ERR_INVALID_ARG),
+    (dict(has_ve=2), cs.ERR_INVALID_ARG),
+    (dict(rope_base=0.0), cs.ERR_INVALID_ARG),
+    (dict(rope_base=float("inf")), cs.ERR_INVALID_ARG),
+    (dict(eps=-1.0), cs.ERR_INVALID_ARG),
+    (dict(softmax_scale=-0.5), cs.ERR_INVALID_ARG),
+    (dict(head_dim=64), cs.ERR_UNSUPPORTED),
+    (dict(head_dim=6, dtype="f32"), cs.ERR_UNSUPPORTED),
+    (dict(T=(1 << 20) + 1), cs.ERR_UNSUPPORTED),
+])
+def test_layer_validation(lib, change, code):
+    base = dict(B=2, T=64, n_head=4, n_kv_head=2, head_dim=128, window=32)
+    spec = cs.LayerSpec(**{**base, **change})
+    layer = spec.c()
+    if "has_ve" in change:
+        layer.has_ve = change["has_ve"]
+    assert lib.attn_fwd(ctypes.byref(layer), 16, 32, 48, 64, 80, None) == code
+    assert lib.cswattn_last_error().decode() != ""
+    assert lib.attn_bwd_workspace_bytes(ctypes.byref(layer)) == 0
+
+
+def test_bad_dtype_and_null_layer(lib):
+    spec = cs.LayerSpec(2, 64, 4, 2, 128, 32)
+    layer = spec.c()
+    layer.dtype = 7
+    assert lib.attn_fwd(ctypes.byref(layer), 16, 32, 48, 64, 80, None) == cs.ERR_INVALID_ARG
+    assert lib.attn_fwd(None, 16, 32, 48, 64, 80, None) == cs.ERR_INVALID_ARG
+
+
+def test_pointer_validation(lib):
+    spec = cs.LayerSpec(2, 64, 4, 2, 128, 32)
+    layer = ctypes.byref(spec.c())
+    assert lib.attn_fwd(layer, None, 32, 48, 64, 80, None) == cs.ERR_INVALID_ARG
+    assert b"q_out" in lib.cswattn_last_error()
+    assert lib.attn_fwd(layer, 16 + 8, 32, 48, 64, 80, None) == cs.ERR_INVALID_ARG
+    assert b"aligned" in lib.cswattn_last_error()
+    assert lib.attn_fwd(layer, 16, 32, 48, 64, 82, None) == cs.ERR_INVALID_ARG  # lse 4-byte
+    # prologue: outputs may not alias inputs; ve/gate required with has_ve
+    args = [16, 32, 48, 64, 80, 16, 112, 128, 144, 160, None]
+    assert lib.attn_prologue(layer, *args) == cs.ERR_INVALID_ARG
+    assert b"alias" in lib.cswattn_last_error()
+    args = [16, 32, 48, None, 80, 96, 112, 128, 144, 160, None]
+    assert lib.attn_prologue(layer, *args) == cs.ERR_INVALID_ARG
+    assert b"ve" in lib.cswattn_last_error()
+
+
+def test_workspace_size_and_check(lib):
+    spec = cs.LayerSpec(2, 100, 6, 2, 128, 32)
+    n = cs.attn_bwd_workspace_bytes(spec)
+    pad = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    B, T, H, Hk, D = 2, 100, 6, 2, 128
+    assert n == pad(4 * B * H * T * D) + 2 * pad(4 * B * T * Hk * D) + pad(4 * B * H * T)
+    layer = ctypes.byref(spec.c())
+    ptrs = [256 * (i + 1) for i in range(17)]
+    st = lib.attn_bwd(layer, *ptrs[:12], *ptrs[12:17], 256 * 40, n - 1, None)
+    assert st == cs.ERR_INVALID_ARG
+    assert b"workspace" in lib.cswattn_last_error()
