@@ -136,6 +136,11 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     w = cs.WORKLOADS[CONFIG_ID]
+    if args.single_layer is not None:
+        # Profiling case: one layer of the workload, same shapes and launches.
+        i = args.single_layer
+        w = cs.Workload(w.config, w.name + f" (layer {i} only)", w.B, w.T, w.H, w.Hk, w.D,
+                        [w.windows[i]], [w.ve[i]], w.dtype, w.rope_base, w.eps, w.dO_std)
     specs = [cs.LayerSpec(w.B, w.T, w.H, w.Hk, w.D, W, has_ve=ve, dtype=w.dtype,
                           rope_base=w.rope_base, eps=w.eps)
              for W, ve in zip(w.windows, w.ve)]
@@ -211,11 +216,14 @@ def run_ours(args):
     cs.cswattn_sync_status()
 
     # e2e: host buffers in, results out, copies inside the timed region
-    for _ in range(2):
-        step_e2e()
-    torch.cuda.synchronize(dev)
-    e2e_ms = timed(step_e2e, max(1, min(args.steps, 5)), flush=False)
     e2e_steps = max(1, min(args.steps, 5))
+    if args.single_layer is None:
+        for _ in range(2):
+            step_e2e()
+        torch.cuda.synchronize(dev)
+        e2e_ms = timed(step_e2e, e2e_steps, flush=False)
+    else:
+        e2e_ms = float("nan")
     cs.cswattn_sync_status()
 
     t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
@@ -271,7 +279,7 @@ def run_ours(args):
                     "ms_per_step": round(e2e_ms / e2e_steps, 3)},
             "clocks": clk,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.single_layer is None:
             line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -396,6 +404,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--single-layer", type=int, default=None,
+                    help="profiling case: time only this layer of the stack (no e2e, no CPU leg)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
