@@ -25,31 +25,41 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const PreParams p) {
   using V = Vec16<T>;
   constexpr int VEC = V::N;
   constexpr int LPR = D / VEC;
-  constexpr int RPB = 256 / LPR;  // rows per block pass
+  constexpr int RPW = 32 / LPR;           // rows per warp per slot
+  constexpr int U = kRowsInFlight;        // slots per pass
   const int sub = threadIdx.x % LPR;
-  const long long stride = static_cast<long long>(gridDim.x) * RPB;
-  const long long first = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / LPR;
-  // Uniform trip count across the warp.
-  const long long warp_first = first - (threadIdx.x % 32) / LPR;
-  for (long long base = warp_first; base < p.rows; base += stride) {
-    const long long row = base + (threadIdx.x % 32) / LPR;
-    const bool valid = row < p.rows;
-    float acc = 0.f;
-    if (valid) {
-      float o[VEC], g[VEC];
-      V::load(static_cast<const T*>(p.O) + row * D + sub * VEC, o);
-      V::load(static_cast<const T*>(p.dO) + row * D + sub * VEC, g);
+  const int lrow = (threadIdx.x % 32) / LPR;
+  const long long warp_global = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / 32;
+  const long long n_warps = static_cast<long long>(gridDim.x) * 8;
+  // Uniform trip count across the warp; U rows' loads in flight per lane.
+  for (long long base = warp_global * RPW * U; base < p.rows; base += n_warps * RPW * U) {
+    float o[U][VEC], g[U][VEC];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) acc = fmaf(o[i], g[i], acc);
+    for (int u = 0; u < U; ++u) {
+      const long long row = base + u * RPW + lrow;
+      if (row < p.rows) {
+        V::load(static_cast<const T*>(p.O) + row * D + sub * VEC, o[u]);
+        V::load(static_cast<const T*>(p.dO) + row * D + sub * VEC, g[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) o[u][i] = g[u][i] = 0.f;
+      }
     }
 #pragma unroll
-    for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, LPR);
-    if (valid && sub == 0) {
-      // row = (b*T + t)*H + h  ->  delta[(b*H + h)*T + t]
-      const long long h = row % p.H;
-      const long long bt = row / p.H;
-      const long long t = bt % p.T, b = bt / p.T;
-      p.delta[(b * p.H + h) * p.T + t] = acc;
+    for (int u = 0; u < U; ++u) {
+      const long long row = base + u * RPW + lrow;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc = fmaf(o[u][i], g[u][i], acc);
+#pragma unroll
+      for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, LPR);
+      if (row < p.rows && sub == 0) {
+        // row = (b*T + t)*H + h  ->  delta[(b*H + h)*T + t]
+        const long long h = row % p.H;
+        const long long bt = row / p.H;
+        const long long t = bt % p.T, b = bt / p.T;
+        p.delta[(b * p.H + h) * p.T + t] = acc;
+      }
     }
   }
 }
@@ -106,116 +116,122 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
   const int sub = threadIdx.x % LPR;
   const int grp = threadIdx.x / LPR;
 
-  for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
-    const int r = base + grp;
-    const bool in_range = r < total_rows;
-    const int rr = in_range ? r : 0;
-    const int tt = rr / rows_per_tok;
-    const int kind_row = rr % rows_per_tok;
-    const long long tok = tok0 + tt;
-    const bool valid = in_range && tok < n_tok;
-    const long long tk = valid ? tok : 0;
-    const int t = static_cast<int>(tk % p.T);
-    const long long b = tk / p.T;
-    int kind, head, nheads;
-    if (kind_row < p.H) {
-      kind = 0; head = kind_row; nheads = p.H;
-    } else if (kind_row < p.H + p.Hk) {
-      kind = 1; head = kind_row - p.H; nheads = p.Hk;
-    } else {
-      kind = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
-    }
-    const size_t row = static_cast<size_t>(tk) * nheads + head;  // (b,t,head)
-    const size_t off = row * D + static_cast<size_t>(sub) * VEC;
-
-    // Gradient w.r.t. the rotated, normalised row (or dv_eff for kind 2).
-    float dy[VEC];
-    if (valid) {
-      const float* src;
-      if (kind == 0)
-        src = p.dq_acc + ((static_cast<size_t>(b) * p.H + head) * p.T + t) * D + sub * VEC;
-      else
-        src = (kind == 1 ? p.dk_acc : p.dv_acc) + off;
-      load_f32<VEC>(src, dy);
-    } else {
+  // Like the prologue: U rows per lane per pass, loads first.
+  constexpr int U = kRowsInFlight;
+  for (int base = 0; base < total_rows; base += ROWS_PER_PASS * U) {
+    float dy[U][VEC], x[U][VEC];
+    float rs[U], gl[U];
+    int kind[U], tt[U];
+    bool valid[U];
+    size_t row[U], off[U];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) dy[i] = 0.f;
-    }
-
-    // RoPE^-1 (the transpose rotation).
-    float dn[VEC];
-    if constexpr (LPR >= 2) {
-      float partner[VEC];
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, dy[i], LPR / 2, LPR);
-      const bool lower = sub < LPR / 2;
-      const int pair0 = (lower ? sub : sub - LPR / 2) * VEC;
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        const float c = s_cos[tt][pair0 + i], s = s_sin[tt][pair0 + i];
-        // lower: dy_i c + dy_{i+D/2} s ; upper: -dy_{i-D/2} s + dy_i c
-        dn[i] = lower ? fmaf(dy[i], c, partner[i] * s) : fmaf(-partner[i], s, dy[i] * c);
+    for (int u = 0; u < U; ++u) {
+      const int r = base + u * ROWS_PER_PASS + grp;
+      const bool in_range = r < total_rows;
+      const int rr = in_range ? r : 0;
+      tt[u] = rr / rows_per_tok;
+      const int kind_row = rr % rows_per_tok;
+      const long long tok = tok0 + tt[u];
+      valid[u] = in_range && tok < n_tok;
+      const long long tk = valid[u] ? tok : 0;
+      const int t = static_cast<int>(tk % p.T);
+      const long long b = tk / p.T;
+      int head, nheads;
+      if (kind_row < p.H) {
+        kind[u] = 0; head = kind_row; nheads = p.H;
+      } else if (kind_row < p.H + p.Hk) {
+        kind[u] = 1; head = kind_row - p.H; nheads = p.Hk;
+      } else {
+        kind[u] = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
       }
-    } else {
+      row[u] = static_cast<size_t>(tk) * nheads + head;  // (b,t,head)
+      off[u] = row[u] * D + static_cast<size_t>(sub) * VEC;
+      rs[u] = 0.f;
+      gl[u] = 0.f;
+      if (valid[u]) {
+        // Gradient w.r.t. the rotated, normalised row (or dv_eff for kind 2).
+        const float* src;
+        if (kind[u] == 0)
+          src = p.dq_acc + ((static_cast<size_t>(b) * p.H + head) * p.T + t) * D + sub * VEC;
+        else
+          src = (kind[u] == 1 ? p.dk_acc : p.dv_acc) + off[u];
+        load_f32<VEC>(src, dy[u]);
+        if (kind[u] != 2) {
+          V::load(static_cast<const T*>(kind[u] == 0 ? p.q : p.k) + off[u], x[u]);
+          rs[u] = (kind[u] == 0 ? p.rstd_q : p.rstd_k)[row[u]];
+        } else if (p.has_ve) {
+          V::load(static_cast<const T*>(p.ve) + off[u], x[u]);  // ve for the value rows
+          gl[u] = V::scalar(p.gate, row[u]);
+        } else {
 #pragma unroll
-      for (int i = 0; i < HALF; ++i) {
-        const float c = s_cos[tt][i], s = s_sin[tt][i];
-        dn[i] = fmaf(dy[i], c, dy[i + HALF] * s);
-        dn[i + HALF] = fmaf(-dy[i], s, dy[i + HALF] * c);
+          for (int i = 0; i < VEC; ++i) x[u][i] = 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) dy[u][i] = x[u][i] = 0.f;
       }
     }
 
-    // RMSNorm backward: dx = r (dn - n mean(dn * n)), n = r x.
-    float x[VEC];
-    float rs = 0.f;
-    if (valid && kind != 2) {
-      V::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off, x);
-      rs = (kind == 0 ? p.rstd_q : p.rstd_k)[row];
-    } else {
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) x[i] = 0.f;
-    }
-    float dot = 0.f;
+    for (int u = 0; u < U; ++u) {
+      // RoPE^-1 (the transpose rotation).
+      float dn[VEC];
+      if constexpr (LPR >= 2) {
+        float partner[VEC];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) dot = fmaf(dn[i], x[i] * rs, dot);
+        for (int i = 0; i < VEC; ++i)
+          partner[i] = __shfl_xor_sync(0xffffffffu, dy[u][i], LPR / 2, LPR);
+        const bool lower = sub < LPR / 2;
+        const int pair0 = (lower ? sub : sub - LPR / 2) * VEC;
 #pragma unroll
-    for (int o = LPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o, LPR);
-    dot /= static_cast<float>(D);
-
-    // Value side: dgate reduction (all lanes take part).
-    float ve[VEC];
-    float coef = 0.f, dg = 0.f;
-    if (valid && kind == 2 && p.has_ve) {
-      V::load(static_cast<const T*>(p.ve) + off, ve);
-      const float s = 1.0f / (1.0f + expf(-V::scalar(p.gate, row)));
-      coef = 3.0f * s;
+        for (int i = 0; i < VEC; ++i) {
+          const float c = s_cos[tt[u]][pair0 + i], s = s_sin[tt[u]][pair0 + i];
+          // lower: dy_i c + dy_{i+D/2} s ; upper: -dy_{i-D/2} s + dy_i c
+          dn[i] = lower ? fmaf(dy[u][i], c, partner[i] * s) : fmaf(-partner[i], s, dy[u][i] * c);
+        }
+      } else {
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) dg = fmaf(dy[i], ve[i], dg);
-      dg *= coef * (1.0f - s);
-    }
-#pragma unroll
-    for (int o = LPR / 2; o >= 1; o >>= 1) dg += __shfl_xor_sync(0xffffffffu, dg, o, LPR);
-
-    if (!valid) continue;
-    if (kind == 2) {
-      V::store(static_cast<T*>(p.dv) + off, dy);
-      if (p.has_ve) {
-        float o[VEC];
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) o[i] = coef * dy[i];
-        V::store(static_cast<T*>(p.dve) + off, o);
-        if (sub == 0) {
-          if constexpr (sizeof(T) == 2)
-            static_cast<__nv_bfloat16*>(p.dgate)[row] = __float2bfloat16_rn(dg);
-          else
-            static_cast<float*>(p.dgate)[row] = dg;
+        for (int i = 0; i < HALF; ++i) {
+          const float c = s_cos[tt[u]][i], s = s_sin[tt[u]][i];
+          dn[i] = fmaf(dy[u][i], c, dy[u][i + HALF] * s);
+          dn[i + HALF] = fmaf(-dy[u][i], s, dy[u][i + HALF] * c);
         }
       }
-    } else {
-      float o[VEC];
+      // One shuffle reduction serves both row kinds: for q/k rows the
+      // RMSNorm term sum_d dn*n (n = r x); for value rows sum_d dv_eff*ve.
+      const bool vrow = kind[u] == 2;
+      float dot = 0.f;
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) o[i] = rs * (dn[i] - x[i] * rs * dot);
-      V::store(static_cast<T*>(kind == 0 ? p.dq : p.dk) + off, o);
+      for (int i = 0; i < VEC; ++i)
+        dot = vrow ? fmaf(dy[u][i], x[u][i], dot) : fmaf(dn[i], x[u][i] * rs[u], dot);
+#pragma unroll
+      for (int o = LPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o, LPR);
+      if (!valid[u]) continue;
+      if (vrow) {
+        V::store(static_cast<T*>(p.dv) + off[u], dy[u]);
+        if (p.has_ve) {
+          const float sg = 1.0f / (1.0f + expf(-gl[u]));
+          const float coef = 3.0f * sg;
+          float o[VEC];
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) o[i] = coef * dy[u][i];
+          V::store(static_cast<T*>(p.dve) + off[u], o);
+          if (sub == 0) {
+            const float dg = dot * coef * (1.0f - sg);
+            if constexpr (sizeof(T) == 2)
+              static_cast<__nv_bfloat16*>(p.dgate)[row[u]] = __float2bfloat16_rn(dg);
+            else
+              static_cast<float*>(p.dgate)[row[u]] = dg;
+          }
+        }
+      } else {
+        // RMSNorm backward: dx = r (dn - n mean(dn * n)), n = r x.
+        const float mean = dot / static_cast<float>(D);
+        float o[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) o[i] = rs[u] * (dn[i] - x[u][i] * rs[u] * mean);
+        V::store(static_cast<T*>(kind[u] == 0 ? p.dq : p.dk) + off[u], o);
+      }
     }
   }
 }

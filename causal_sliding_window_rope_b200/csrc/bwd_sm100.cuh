@@ -22,8 +22,10 @@
 //   dQ^T = K^T dS^T   (M=128 d, N=64 queries, K=128 keys)   SS MMA, into
 //          the S^T columns of the step, drained by the dQ warps into a
 //          float32 tile that a bulk reduce-add sends to the dq accumulator.
-// TMEM (512 columns): SP0 | SP1 (S^T at +0, dP^T at +64; double buffered so
-// the next step's products overlap this step's softmax) | dV | dK.
+// TMEM (512 columns): SP (S^T at +0, dP^T at +64) | dQ^T x2 (64 columns
+// each) | dV | dK. The softmax warps release SP as soon as they have loaded
+// it into registers, so the next step's S^T/dP^T run while they compute; the
+// dQ^T double buffer lets the drain of one step overlap the next step.
 // Roles: warp 0 TMA, warp 1 MMA issuer + TMEM owner, warps 4-7 softmax
 // (thread = key row), warps 8-11 dQ drain (thread = head_dim row of dQ^T).
 #pragma once
@@ -54,8 +56,15 @@ constexpr int kOffBar = kOffDQ + kDQBytes;
 constexpr int kOffRow = kOffBar + 256;         // lse2[2][64], delta[2][64]
 constexpr int kSmemBytes = kOffRow + 4 * kBQ * 4 + 1024;
 
-// TMEM column of the S^T / dP^T buffer st (0 or 1).
-__host__ __device__ constexpr uint32_t col_sp(int st) { return st ? 128u : 0u; }
+// Register budgets after setmaxnreg (launch: 384 threads x 168 registers).
+constexpr int kRegLo = 80;   // producer / MMA warpgroup
+constexpr int kRegSm = 240;  // softmax warpgroup (S^T, dP^T rows + packed P, dS)
+constexpr int kRegDq = 184;  // dQ drain warpgroup
+static_assert(128 * (kRegLo + kRegSm + kRegDq) <= kThreads * 168, "register budget");
+
+constexpr uint32_t kColSP = 0u;  // S^T at +0, dP^T at +64
+// TMEM column of dQ^T buffer st (0 or 1).
+__host__ __device__ constexpr uint32_t col_dq(int st) { return st ? 192u : 128u; }
 constexpr uint32_t kColDV = 256u;
 constexpr uint32_t kColDK = 384u;
 
@@ -95,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;     // [2]
   uint64_t* q_empty = bars + 3;    // [2]
-  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_full = bars + 5;     // [0]: S^T/dP^T ready; [1]: SP loaded by softmax (free)
   uint64_t* p_full = bars + 7;     // [2]
   uint64_t* ps_empty = bars + 9;   // [2]
   uint64_t* dq_full = bars + 11;   // [2]
@@ -131,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
-      mbar_init(&s_full[s], 1);
+      mbar_init(&s_full[s], s == 0 ? 1 : 128);
       mbar_init(&p_full[s], 128);
       mbar_init(&ps_empty[s], 1);
       mbar_init(&dq_full[s], 1);
@@ -157,10 +166,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.wait_ns};
+  uint64_t* sp_full = &s_full[0];
+  uint64_t* sp_free = &s_full[1];
+
 
   auto step_head = [&](int n) { return hk * p.g + n / nsph; };
   auto step_q0 = [&](int n) { return (qs_lo + n % nsph) * kBQ; };
 
+  if (warp < 4) {
+    regs_dec<kRegLo>();
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
@@ -199,59 +213,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(kv_full, 0, wc);
       tc_fence_after();
 
+      // Descriptors: a base per buffer plus a compile-time offset per k-step
+      // (the start-address field holds address >> 4).
+      const uint64_t dK_k = sdesc_sw128(sK, 16, 1024);         // K, K-major
+      const uint64_t dV_k = sdesc_sw128(sV, 16, 1024);         // V, K-major
+      const uint64_t dQ_k = sdesc_sw128(sQ, 16, 1024);         // Q, K-major
+      const uint64_t dO_k = sdesc_sw128(sDO, 16, 1024);        // dO, K-major
+      const uint64_t dQ_m = sdesc_sw128(sQ, kQPanel, 1024);    // Q, MN-major
+      const uint64_t dO_m = sdesc_sw128(sDO, kQPanel, 1024);   // dO, MN-major
+      const uint64_t dP_k = sdesc_sw128(sP, 16, 1024);         // P^T, K-major
+      const uint64_t dS_k = sdesc_sw128(sDS, 16, 1024);        // dS^T, K-major
+      const uint64_t dS_m = sdesc_sw128(sDS, kPBytes, 1024);   // dS^T, MN-major
+      const uint64_t dK_m = sdesc_sw128(sK, kKVPanel, 1024);   // K^T, MN-major
+      auto ofs = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
+
       auto issue_SdP = [&](int n) -> bool {
         const int st = n & 1, use = n >> 1;
         if (!mbar_wait(&q_full[st], use & 1, wc)) return false;
-        if (use > 0 && !mbar_wait(&dq_empty[st], (use - 1) & 1, wc)) return false;
+        if (n > 0 && !mbar_wait(sp_free, (n - 1) & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t qa = sQ + st * kQBytes, oa = sDO + st * kQBytes;
+        const uint64_t qb = ofs(st * kQBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ok_ = (kk >> 2) * kKVPanel + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * kQPanel + (kk & 3) * 32;
-          mma_ss(tmem + col_sp(st), sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(qa + oq, 16, 1024),
-                 idS, kk > 0 ? 1u : 0u);
+          const uint64_t okv = ofs((kk >> 2) * kKVPanel + (kk & 3) * 32);
+          const uint64_t oq = ofs((kk >> 2) * kQPanel + (kk & 3) * 32);
+          mma_ss(tmem + kColSP, dK_k + okv, dQ_k + qb + oq, idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ok_ = (kk >> 2) * kKVPanel + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * kQPanel + (kk & 3) * 32;
-          mma_ss(tmem + col_sp(st) + 64, sdesc_sw128(sV + ok_, 16, 1024),
-                 sdesc_sw128(oa + oq, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          const uint64_t okv = ofs((kk >> 2) * kKVPanel + (kk & 3) * 32);
+          const uint64_t oq = ofs((kk >> 2) * kQPanel + (kk & 3) * 32);
+          mma_ss(tmem + kColSP + 64, dV_k + okv, dO_k + qb + oq, idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[st]);
+        mma_commit(sp_full);
         return true;
       };
 
       if (ok) ok = issue_SdP(0);
       for (int n = 0; ok && n < N; ++n) {
         const int st = n & 1, use = n >> 1;
+        // The next step's S^T/dP^T as soon as the softmax has loaded this one.
         if (n + 1 < N && !issue_SdP(n + 1)) break;
         if (!mbar_wait(&p_full[st], use & 1, wc)) break;
         tc_fence_after();
-        const uint32_t pa = sP + st * kPBytes, da = sDS + st * kPBytes;
-        const uint32_t qa = sQ + st * kQBytes, oa = sDO + st * kQBytes;
+        const uint64_t pb = ofs(st * kPBytes), qb = ofs(st * kQBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
-          mma_ss(tmem + kColDV, sdesc_sw128(pa + kk * 32, 16, 1024),
-                 sdesc_sw128(oa + kk * 2048, kQPanel, 1024), idKV, (n > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tmem + kColDV, dP_k + pb + ofs(kk * 32), dO_m + qb + ofs(kk * 2048), idKV,
+                 (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-          mma_ss(tmem + kColDK, sdesc_sw128(da + kk * 32, 16, 1024),
-                 sdesc_sw128(qa + kk * 2048, kQPanel, 1024), idKV, (n > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tmem + kColDK, dS_k + pb + ofs(kk * 32), dQ_m + qb + ofs(kk * 2048), idKV,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&q_empty[st]);
+        if (use > 0 && !mbar_wait(&dq_empty[st], (use - 1) & 1, wc)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
-          mma_ss(tmem + col_sp(st), sdesc_sw128(sK + kk * 2048, kKVPanel, 1024),
-                 sdesc_sw128(da + kk * 2048, kPBytes, 1024), idDQ, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + col_dq(st), dK_m + ofs(kk * 2048), dS_m + pb + ofs(kk * 2048), idDQ,
+                 kk > 0 ? 1u : 0u);
         mma_commit(&dq_full[st]);
         mma_commit(&ps_empty[st]);
-        mma_commit(&q_empty[st]);
       }
       mma_commit(acc_full);
       mma_commit(mma_done);
       drain_wait(mma_done, 0, p.wait_ns);
     }
-  } else if (warp >= 4 && warp < 8) {
+  }
+  } else if (warp < 8) {
+    regs_inc<kRegSm>();
     // -------------------------------------------------- softmax / dS
     const int r = (warp & 3) * 32 + lane;  // key row within the tile
     const int tid = (warp - 4) * 32 + lane;
@@ -277,38 +307,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&row_full[st]);
       }
       bool got = mbar_wait(&row_full[st], use & 1, wc);
-      got = got && mbar_wait(&s_full[st], use & 1, wc);
+      got = got && mbar_wait(sp_full, n & 1, wc);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sv[2][32], dv[2][32];
-      tmem_ld32(tmem + lane_off + col_sp(st), sv[0]);
-      tmem_ld32(tmem + lane_off + col_sp(st) + 32, sv[1]);
-      tmem_ld32(tmem + lane_off + col_sp(st) + 64, dv[0]);
-      tmem_ld32(tmem + lane_off + col_sp(st) + 96, dv[1]);
+      tmem_ld32(tmem + lane_off + kColSP, sv[0]);
+      tmem_ld32(tmem + lane_off + kColSP + 32, sv[1]);
+      tmem_ld32(tmem + lane_off + kColSP + 64, dv[0]);
+      tmem_ld32(tmem + lane_off + kColSP + 96, dv[1]);
       tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(sp_free);  // the MMA warp may overwrite SP now
       const bool need_mask = (q0 < k0 + kBN - 1) || (q0 + kBQ - 1 - k0 >= p.W);
-      const float* L2 = s_lse2 + st * kBQ;
-      const float* DL = s_delta + st * kBQ;
+      const float4* L2 = reinterpret_cast<const float4*>(s_lse2 + st * kBQ);
+      const float4* DL = reinterpret_cast<const float4*>(s_delta + st * kBQ);
       uint32_t pp[32], dd[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float pv[2], dsv[2];
+        for (int i = 0; i < 32; i += 4) {
+          const float4 l4 = L2[(c * 32 + i) >> 2];
+          const float4 d4 = DL[(c * 32 + i) >> 2];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
+          for (int e = 0; e < 4; ++e) {
             const int col = c * 32 + i + e;
             const int q = q0 + col;
-            float pr = ex2(fmaf(__uint_as_float(sv[c][i + e]), c2, -L2[col]));
+            float pr = ex2(fmaf(__uint_as_float(sv[c][i + e]), c2, -lv[e]));
             if (need_mask && (q < kj || q - kj >= p.W)) pr = 0.f;
             pv[e] = pr;
-            dsv[e] = pr * (__uint_as_float(dv[c][i + e]) - DL[col]);
+            dsv[e] = pr * (__uint_as_float(dv[c][i + e]) - dl[e]);
           }
           pp[c * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
+          pp[c * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
           dd[c * 16 + i / 2] = pack_bf16x2(dsv[0], dsv[1]);
+          dd[c * 16 + i / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
       mbar_arrive(&row_empty[st]);
       got = use == 0 || mbar_wait(&ps_empty[st], (use - 1) & 1, wc);
@@ -361,7 +399,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= 8) {
+  } else {
+    if constexpr (kRegDq > 168)
+      regs_inc<kRegDq>();
+    else
+      regs_dec<kRegDq>();
     // -------------------------------------------------- dQ drain
     const int d = (warp & 3) * 32 + lane;  // TMEM lane = head_dim index of dQ^T
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -375,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       uint32_t a[2][32];
-      tmem_ld32(tmem + lane_off + col_sp(st), a[0]);
-      tmem_ld32(tmem + lane_off + col_sp(st) + 32, a[1]);
+      tmem_ld32(tmem + lane_off + col_dq(st), a[0]);
+      tmem_ld32(tmem + lane_off + col_dq(st) + 32, a[1]);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&dq_empty[st]);

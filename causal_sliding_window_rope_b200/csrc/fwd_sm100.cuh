@@ -45,6 +45,11 @@ constexpr int kOffV = 4 * kTileBytes;        // 2 stages
 constexpr int kOffBar = 6 * kTileBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
+// Register budgets after setmaxnreg; the sum may not exceed the launch
+// allocation (384 threads x 168 registers).
+constexpr int kRegLo = 80;   // producer / MMA warpgroup
+constexpr int kRegHi = 208;  // each softmax warpgroup
+static_assert(128 * kRegLo + 256 * kRegHi <= kThreads * 168, "register budget");
 
 struct Params {
   int B, T, H, Hk, W, g, nq, npairs;
@@ -140,6 +145,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t colS[2] = {0u, 128u};
   const uint32_t colO[2] = {256u, 384u};
 
+  // Registers move from the producer/MMA warpgroup to the softmax
+  // warpgroups, which hold a full 128-column S row per thread. Each role's
+  // code sits inside its warpgroup's branch so ptxas compiles it under that
+  // warpgroup's budget.
+  if (warp < 4) {
+    regs_dec<kRegLo>();
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
@@ -184,16 +195,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(q_full, 0, wc);
       tc_fence_after();
 
+      // Descriptors: a base per buffer plus a compile-time offset per k-step
+      // (the start-address field holds address >> 4).
+      const uint64_t dQ0 = sdesc_sw128(sQa, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sKa, 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(sVa, kPanelBytes, 1024);
+
       auto issue_S = [&](int X, int j) -> bool {
         const int it = j - lo, s = it & 1, use = it >> 1;
         if (!mbar_wait(&k_full[s], use & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t qa = sQa + X * kTileBytes, ka = sKa + s * kTileBytes;
+        const uint64_t qd = dQ0 + static_cast<uint64_t>((X * kTileBytes) >> 4);
+        const uint64_t kd = dK0 + static_cast<uint64_t>((s * kTileBytes) >> 4);
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(X) * 128u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          mma_ss(tmem + colS[X], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                 idS, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d_tmem, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[X]);
         return true;
@@ -204,13 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&v_full[s], use & 1, wc)) return false;
         if (!mbar_wait(&p_full[X], n & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t va = sVa + s * kTileBytes;
+        const uint64_t vd = dV0 + static_cast<uint64_t>((s * kTileBytes) >> 4);
+        const uint32_t o_tmem = tmem + 256u + static_cast<uint32_t>(X) * 128u;
+        const uint32_t p_tmem = tmem + static_cast<uint32_t>(X) * 128u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(tmem + colO[X], tmem + colS[X] + kk * 8,
-                 sdesc_sw128(va + kk * 2048, kPanelBytes, 1024), idPV,
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
                  (n > 0 || kk > 0) ? 1u : 0u);
-        }
         return true;
       };
 
@@ -237,7 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(mma_done);
       drain_wait(mma_done, 0, p.wait_ns);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<kRegHi>();
     // -------------------------------------------------- softmax + epilogue
     const int X = (warp - 4) >> 2;
     if (valid[X]) {
@@ -272,12 +292,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (kj > qi || qi - kj >= p.W) sv[c][i] = __float_as_uint(-INFINITY);
             }
         }
-        float mx = -INFINITY;
+        // Row max as a tree (8 independent chains, then combine).
+        float mp[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) mp[t] = __uint_as_float(sv[t >> 1][(t & 1) * 16]);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
-        mx *= c2;
+          for (int i = 0; i < 32; ++i)
+            if (i != 0 && i != 16)
+              mp[c * 2 + (i >> 4)] = fmaxf(mp[c * 2 + (i >> 4)], __uint_as_float(sv[c][i]));
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mp[t] = fmaxf(mp[t], mp[t + 4]);
+        float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * c2;
         float alpha = 1.f;
         bool rescale = false;
         if (n == 0) {
@@ -299,8 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st_wait();
         }
-        l *= alpha;
         const float mu = (m2 == -INFINITY) ? 0.f : m2;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
@@ -308,11 +335,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) {
             const float p0 = ex2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -mu));
             const float p1 = ex2(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -mu));
-            l += p0 + p1;
+            ls[i & 3] += p0 + p1;
             pk[i] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tS + c * 16, pk);
         }
+        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[X]);

@@ -20,6 +20,7 @@ namespace cswattn {
 constexpr int kPrologueThreads = 256;
 constexpr int kPrologueTok = 8;
 constexpr int kMaxHalfD = 64;
+constexpr int kRowsInFlight = 4;
 
 struct PrologueParams {
   int B, T, H, Hk;
@@ -108,85 +109,104 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int sub = threadIdx.x % LPR;        // lane within the row group
   const int grp = threadIdx.x / LPR;        // row group within the CTA
 
-  // Uniform trip count: every lane takes part in every shuffle.
-  for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
-    const int r = base + grp;
-    const bool in_range = r < total_rows;
-    const int rr = in_range ? r : 0;
-    const int tt = rr / rows_per_tok;
-    const int kind_row = rr % rows_per_tok;
-    const long long tok = tok0 + tt;
-    const bool valid = in_range && tok < n_tok;
-    // Row kinds: [0, H) query heads, [H, H+Hk) key heads, then value heads.
-    int kind, head, nheads;
-    if (kind_row < p.H) {
-      kind = 0; head = kind_row; nheads = p.H;
-    } else if (kind_row < p.H + p.Hk) {
-      kind = 1; head = kind_row - p.H; nheads = p.Hk;
-    } else {
-      kind = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
-    }
-    const size_t row = static_cast<size_t>(valid ? tok : 0) * nheads + head;
-    const size_t off = row * D + static_cast<size_t>(sub) * VEC;
-    const void* src = kind == 0 ? p.q : (kind == 1 ? p.k : p.v);
-    float x[VEC];
-    if (valid) {
-      V::load(static_cast<const T*>(src) + off, x);
-    } else {
+  // kRowsInFlight rows per lane per pass: all loads of a pass are issued
+  // before any arithmetic, so each lane keeps several 16-byte loads in
+  // flight. Uniform trip count: every lane takes part in every shuffle.
+  constexpr int U = kRowsInFlight;
+  for (int base = 0; base < total_rows; base += ROWS_PER_PASS * U) {
+    float x[U][VEC], e[U][VEC];
+    float gl[U];
+    int kind[U];
+    bool valid[U];
+    size_t row[U], off[U];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) x[i] = 0.f;
-    }
-
-    // RMSNorm: mean of squares over the row's LPR lanes (shuffle reduction).
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) ss = fmaf(x[i], x[i], ss);
-#pragma unroll
-    for (int o = LPR / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPR);
-    const float rstd = rsqrtf(ss / static_cast<float>(D) + p.eps);
-    float n[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) n[i] = x[i] * rstd;
-
-    // RoPE on half-split pairs (i, i + D/2).
-    float y[VEC];
-    if constexpr (LPR >= 2) {
-      float partner[VEC];
-#pragma unroll
-      for (int i = 0; i < VEC; ++i)
-        partner[i] = __shfl_xor_sync(0xffffffffu, n[i], LPR / 2, LPR);
-      const bool lower = sub < LPR / 2;
-      const int pair0 = (lower ? sub : sub - LPR / 2) * VEC;
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) {
-        const float c = s_cos[tt][pair0 + i], s = s_sin[tt][pair0 + i];
-        // lower half: x_i c - x_{i+D/2} s ; upper half: x_{i-D/2} s + x_i c
-        y[i] = lower ? fmaf(n[i], c, -partner[i] * s) : fmaf(partner[i], s, n[i] * c);
+    for (int u = 0; u < U; ++u) {
+      const int r = base + u * ROWS_PER_PASS + grp;
+      const bool in_range = r < total_rows;
+      const int rr = in_range ? r : 0;
+      const int tt = rr / rows_per_tok;
+      const int kind_row = rr % rows_per_tok;
+      const long long tok = tok0 + tt;
+      valid[u] = in_range && tok < n_tok;
+      // Row kinds: [0, H) query heads, [H, H+Hk) key heads, then value heads.
+      int head, nheads;
+      if (kind_row < p.H) {
+        kind[u] = 0; head = kind_row; nheads = p.H;
+      } else if (kind_row < p.H + p.Hk) {
+        kind[u] = 1; head = kind_row - p.H; nheads = p.Hk;
+      } else {
+        kind[u] = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
       }
-    } else {
+      row[u] = static_cast<size_t>(valid[u] ? tok : 0) * nheads + head;
+      off[u] = row[u] * D + static_cast<size_t>(sub) * VEC;
+      const void* src = kind[u] == 0 ? p.q : (kind[u] == 1 ? p.k : p.v);
+      if (valid[u]) {
+        V::load(static_cast<const T*>(src) + off[u], x[u]);
+      } else {
 #pragma unroll
-      for (int i = 0; i < HALF; ++i) {
-        const float c = s_cos[tt][i], s = s_sin[tt][i];
-        y[i] = fmaf(n[i], c, -n[i + HALF] * s);
-        y[i + HALF] = fmaf(n[i], s, n[i + HALF] * c);
+        for (int i = 0; i < VEC; ++i) x[u][i] = 0.f;
+      }
+      gl[u] = 0.f;
+      if (valid[u] && kind[u] == 2 && p.has_ve) {
+        V::load(static_cast<const T*>(p.ve) + off[u], e[u]);
+        gl[u] = V::scalar(p.gate, row[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) e[u][i] = 0.f;
       }
     }
-    if (!valid) continue;
 
-    if (kind == 2) {
-      // Value residual: v + 3 sigmoid(gate) ve.
-      if (p.has_ve) {
-        float e[VEC];
-        V::load(static_cast<const T*>(p.ve) + off, e);
-        const float gl = V::scalar(p.gate, row);
-        const float coef = 3.0f / (1.0f + expf(-gl));
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) x[i] = fmaf(coef, e[i], x[i]);
+    for (int u = 0; u < U; ++u) {
+      const int r = base + u * ROWS_PER_PASS + grp;
+      const int tt = (r < total_rows ? r : 0) / rows_per_tok;
+      // RMSNorm: mean of squares over the row's LPR lanes (shuffle reduction).
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) ss = fmaf(x[u][i], x[u][i], ss);
+#pragma unroll
+      for (int o = LPR / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPR);
+      const float rstd = rsqrtf(ss / static_cast<float>(D) + p.eps);
+      float n[VEC];
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) n[i] = x[u][i] * rstd;
+
+      // RoPE on half-split pairs (i, i + D/2).
+      float y[VEC];
+      if constexpr (LPR >= 2) {
+        float partner[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i)
+          partner[i] = __shfl_xor_sync(0xffffffffu, n[i], LPR / 2, LPR);
+        const bool lower = sub < LPR / 2;
+        const int pair0 = (lower ? sub : sub - LPR / 2) * VEC;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+          const float c = s_cos[tt][pair0 + i], s = s_sin[tt][pair0 + i];
+          // lower half: x_i c - x_{i+D/2} s ; upper half: x_{i-D/2} s + x_i c
+          y[i] = lower ? fmaf(n[i], c, -partner[i] * s) : fmaf(partner[i], s, n[i] * c);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          const float c = s_cos[tt][i], s = s_sin[tt][i];
+          y[i] = fmaf(n[i], c, -n[i + HALF] * s);
+          y[i + HALF] = fmaf(n[i], s, n[i + HALF] * c);
+        }
       }
-      V::store(static_cast<T*>(p.v_out) + off, x);
-    } else {
-      V::store(static_cast<T*>(kind == 0 ? p.q_out : p.k_out) + off, y);
-      if (sub == 0) (kind == 0 ? p.rstd_q : p.rstd_k)[row] = rstd;
+      if (!valid[u]) continue;
+
+      if (kind[u] == 2) {
+        // Value residual: v + 3 sigmoid(gate) ve (e = 0 without ve).
+        const float coef = p.has_ve ? 3.0f / (1.0f + expf(-gl[u])) : 0.f;
+        float vv[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) vv[i] = fmaf(coef, e[u][i], x[u][i]);
+        V::store(static_cast<T*>(p.v_out) + off[u], vv);
+      } else {
+        V::store(static_cast<T*>(kind[u] == 0 ? p.q_out : p.k_out) + off[u], y);
+        if (sub == 0) (kind[u] == 0 ? p.rstd_q : p.rstd_k)[row[u]] = rstd;
+      }
     }
   }
 }
