@@ -13,11 +13,16 @@
 
 namespace cswattn {
 
+// Row terms of the backward, in the padded layout (B, H, Tpad) with Tpad a
+// multiple of 64: delta = dO.O and lse2 = lse * log2(e); past T, delta = 0
+// and lse2 = +inf (so exp2(s - lse2) = 0 for padding queries).
 struct PreParams {
   long long rows;  // B * T * H
-  int T, H;
+  int T, H, Tpad;
   const void *O, *dO;
-  float* delta;    // (B, H, T)
+  const float* lse;  // (B, H, T)
+  float* delta;      // (B, H, Tpad)
+  float* lse2;       // (B, H, Tpad)
 };
 
 template <typename T, int D>
@@ -54,11 +59,19 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const PreParams p) {
 #pragma unroll
       for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, LPR);
       if (row < p.rows && sub == 0) {
-        // row = (b*T + t)*H + h  ->  delta[(b*H + h)*T + t]
+        // row = (b*T + t)*H + h  ->  (b*H + h)*Tpad + t
         const long long h = row % p.H;
         const long long bt = row / p.H;
         const long long t = bt % p.T, b = bt / p.T;
-        p.delta[(b * p.H + h) * p.T + t] = acc;
+        const long long o = (b * p.H + h) * p.Tpad;
+        p.delta[o + t] = acc;
+        p.lse2[o + t] = p.lse[(b * p.H + h) * p.T + t] * 1.4426950408889634f;
+        if (t == p.T - 1) {
+          for (long long tp = p.T; tp < p.Tpad; ++tp) {
+            p.delta[o + tp] = 0.f;
+            p.lse2[o + tp] = INFINITY;
+          }
+        }
       }
     }
   }

@@ -45,21 +45,23 @@ constexpr int kQPanel = kQBytes / 2;     // 8 KB: 64 rows x 128 B
 constexpr int kPBytes = kBN * kBQ * 2;   // 16 KB: 128 rows x 128 B
 constexpr int kDQBytes = kBQ * kD * 4;   // 32 KB float32 staging
 
+constexpr int kQStages = 3;             // Q/dO ring depth
+constexpr int kStageBytes = 2 * kQBytes;  // Q then dO
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKVBytes;
-constexpr int kOffQ = kOffV + kKVBytes;        // [2]
-constexpr int kOffDO = kOffQ + 2 * kQBytes;    // [2]
-constexpr int kOffP = kOffDO + 2 * kQBytes;    // [2]
-constexpr int kOffDS = kOffP + 2 * kPBytes;    // [2]
-constexpr int kOffDQ = kOffDS + 2 * kPBytes;
+constexpr int kOffQD = kOffV + kKVBytes;                 // [kQStages] x (Q | dO)
+constexpr int kOffP = kOffQD + kQStages * kStageBytes;   // P^T (single buffer)
+constexpr int kOffDS = kOffP + kPBytes;                  // dS^T (single buffer)
+constexpr int kOffDQ = kOffDS + kPBytes;
 constexpr int kOffBar = kOffDQ + kDQBytes;
-constexpr int kOffRow = kOffBar + 256;         // lse2[2][64], delta[2][64]
-constexpr int kSmemBytes = kOffRow + 4 * kBQ * 4 + 1024;
+constexpr int kOffRow = kOffBar + 256;         // per Q stage: lse2[64], delta[64]
+constexpr int kSmemBytes = kOffRow + kQStages * 2 * kBQ * 4 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 // Register budgets after setmaxnreg (launch: 384 threads x 168 registers).
-constexpr int kRegLo = 80;   // producer / MMA warpgroup
-constexpr int kRegSm = 240;  // softmax warpgroup (S^T, dP^T rows + packed P, dS)
-constexpr int kRegDq = 184;  // dQ drain warpgroup
+constexpr int kRegLo = 96;   // producer / MMA warpgroup
+constexpr int kRegSm = 248;  // softmax warpgroup (S^T, dP^T rows + packed P, dS)
+constexpr int kRegDq = 160;  // dQ drain warpgroup
 static_assert(128 * (kRegLo + kRegSm + kRegDq) <= kThreads * 168, "register budget");
 
 constexpr uint32_t kColSP = 0u;  // S^T at +0, dP^T at +64
@@ -69,11 +71,11 @@ constexpr uint32_t kColDV = 256u;
 constexpr uint32_t kColDK = 384u;
 
 struct Params {
-  int B, T, H, Hk, W, g, nkv;
+  int B, T, H, Hk, W, g, nkv, Tpad;
   float scale_log2;  // c * log2(e)
   float scale;       // c
-  const float* lse;    // (B,H,T) natural log
-  const float* delta;  // (B,H,T)
+  const float* lse2;   // (B,H,Tpad) lse * log2(e), +inf past T
+  const float* delta;  // (B,H,Tpad) dO.O, 0 past T
   float* dq_acc;       // (B,H,T,D), accumulated (must start at zero)
   float* dk_acc;       // (B,T,Hk,D)
   float* dv_acc;       // (B,T,Hk,D)
@@ -102,23 +104,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;     // [2]
-  uint64_t* q_empty = bars + 3;    // [2]
-  uint64_t* s_full = bars + 5;     // [0]: S^T/dP^T ready; [1]: SP loaded by softmax (free)
-  uint64_t* p_full = bars + 7;     // [2]
-  uint64_t* ps_empty = bars + 9;   // [2]
-  uint64_t* dq_full = bars + 11;   // [2]
-  uint64_t* dq_empty = bars + 13;  // [2]
+  uint64_t* q_full = bars + 1;      // [kQStages]
+  uint64_t* q_empty = bars + 4;     // [kQStages]
+  uint64_t* sp_full = bars + 7;     // S^T/dP^T in TMEM
+  uint64_t* sp_free = bars + 8;     // softmax has loaded S^T/dP^T
+  uint64_t* p_full = bars + 9;      // P^T/dS^T written to shared memory
+  uint64_t* ps_empty = bars + 10;   // MMAs done reading P^T/dS^T
+  uint64_t* dq_full = bars + 11;    // [2]
+  uint64_t* dq_empty = bars + 13;   // [2]
   uint64_t* acc_full = bars + 15;
   uint64_t* mma_done = bars + 16;
-  uint64_t* row_full = bars + 17;    // [2] lse2/delta of a step staged
-  uint64_t* row_empty = bars + 19;   // [2] every softmax thread done with a slot
-  uint64_t* stage_free = bars + 21;  // dQ staging tile may be overwritten
-  uint64_t* stage_full = bars + 22;  // dQ staging tile written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 24);
-  float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [2][64]
-  float* s_delta = s_lse2 + 2 * kBQ;                                // [2][64]
+  uint64_t* stage_free = bars + 17;  // dQ staging tile may be overwritten
+  uint64_t* stage_full = bars + 18;  // dQ staging tile written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
+  float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [kQStages][64]
+  float* s_delta = s_lse2 + kQStages * kBQ;                         // [kQStages][64]
 
   const int warp = warp_id(), lane = lane_id();
 
@@ -137,21 +138,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kQStages; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
-      mbar_init(&s_full[s], s == 0 ? 1 : 128);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&ps_empty[s], 1);
+    }
+    mbar_init(sp_full, 1);
+    mbar_init(sp_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(ps_empty, 1);
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_empty[s], 128);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&row_full[s], kBQ);
-      mbar_init(&row_empty[s], 128);
-    }
     mbar_init(stage_free, 1);
     mbar_init(stage_full, 128);
     *abort_flag = 0;
@@ -166,39 +166,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.wait_ns};
-  uint64_t* sp_full = &s_full[0];
-  uint64_t* sp_free = &s_full[1];
 
 
-  auto step_head = [&](int n) { return hk * p.g + n / nsph; };
-  auto step_q0 = [&](int n) { return (qs_lo + n % nsph) * kBQ; };
+  // Step n = (head within the group, 64-query block), walked without
+  // divisions: every role keeps its own cursor and advances it per step.
+  struct Cursor {
+    int h, qs, h_end, qs_lo, qs_hi;
+    __device__ void next() {
+      if (++qs > qs_hi) {
+        qs = qs_lo;
+        ++h;
+      }
+    }
+    __device__ int q0() const { return qs * kBQ; }
+  };
+  const Cursor cur0{hk * p.g, qs_lo, hk * p.g + p.g, qs_lo, qs_hi};
 
   if (warp < 4) {
     regs_dec<kRegLo>();
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      int nq[2] = {0, 0};
+      int nq[kQStages] = {0, 0, 0};
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmDO);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      Cursor c = cur0;
+      int st = 0, use = 0;
       mbar_expect_tx(kv_full, 2 * kKVBytes);
       tma_load_4d(&tmK, kv_full, smem + kOffK, 0, hk, k0, b);
       tma_load_4d(&tmK, kv_full, smem + kOffK + kKVPanel, 64, hk, k0, b);
       tma_load_4d(&tmV, kv_full, smem + kOffV, 0, hk, k0, b);
       tma_load_4d(&tmV, kv_full, smem + kOffV + kKVPanel, 64, hk, k0, b);
-      for (int n = 0; n < N; ++n) {
-        const int st = n & 1, use = n >> 1;
+      for (int n = 0; n < N; ++n, c.next()) {
         if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, wc)) break;
-        const int h = step_head(n), q0 = step_q0(n);
-        mbar_expect_tx(&q_full[st], 2 * kQBytes);
-        uint8_t* qd = smem + kOffQ + st * kQBytes;
-        uint8_t* od = smem + kOffDO + st * kQBytes;
+        const int h = c.h, q0 = c.q0();
+        mbar_expect_tx(&q_full[st], 2 * kQBytes + 2 * kBQ * 4);
+        uint8_t* qd = smem + kOffQD + st * kStageBytes;
+        uint8_t* od = qd + kQBytes;
         tma_load_4d(&tmQ, &q_full[st], qd, 0, h, q0, b);
         tma_load_4d(&tmQ, &q_full[st], qd + kQPanel, 64, h, q0, b);
         tma_load_4d(&tmDO, &q_full[st], od, 0, h, q0, b);
         tma_load_4d(&tmDO, &q_full[st], od + kQPanel, 64, h, q0, b);
+        // Row terms of the step's 64 queries (padded layout: always in range).
+        const size_t ro = (static_cast<size_t>(b) * p.H + h) * p.Tpad + q0;
+        bulk_load(s_lse2 + st * kBQ, p.lse2 + ro, kBQ * 4, &q_full[st]);
+        bulk_load(s_delta + st * kBQ, p.delta + ro, kBQ * 4, &q_full[st]);
         ++nq[st];
+        if (++st == kQStages) {
+          st = 0;
+          ++use;
+        }
       }
       drain_wait(kv_full, 0, p.wait_ns);
-      for (int s = 0; s < 2; ++s)
+      for (int s = 0; s < kQStages; ++s)
         if (nq[s] > 0) drain_wait(&q_full[s], (nq[s] - 1) & 1, p.wait_ns);
     }
   } else if (warp == 1) {
@@ -208,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idKV = idesc_bf16(128, 128, 0, 1);  // P^T dO, dS^T Q
       constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T
       const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV);
-      const uint32_t sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO);
+      const uint32_t sQ = smem_u32(smem + kOffQD), sDO = sQ + kQBytes;
       const uint32_t sP = smem_u32(smem + kOffP), sDS = smem_u32(smem + kOffDS);
       bool ok = mbar_wait(kv_full, 0, wc);
       tc_fence_after();
@@ -228,11 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto ofs = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
 
       auto issue_SdP = [&](int n) -> bool {
-        const int st = n & 1, use = n >> 1;
+        const int st = n % kQStages, use = n / kQStages;
         if (!mbar_wait(&q_full[st], use & 1, wc)) return false;
         if (n > 0 && !mbar_wait(sp_free, (n - 1) & 1, wc)) return false;
         tc_fence_after();
-        const uint64_t qb = ofs(st * kQBytes);
+        const uint64_t qb = ofs(st * kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t okv = ofs((kk >> 2) * kKVPanel + (kk & 3) * 32);
@@ -251,29 +273,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (ok) ok = issue_SdP(0);
       for (int n = 0; ok && n < N; ++n) {
-        const int st = n & 1, use = n >> 1;
+        const int st = n % kQStages;
+        const int db = n & 1, duse = n >> 1;  // dQ^T TMEM buffer
         // The next step's S^T/dP^T as soon as the softmax has loaded this one.
         if (n + 1 < N && !issue_SdP(n + 1)) break;
-        if (!mbar_wait(&p_full[st], use & 1, wc)) break;
+        if (!mbar_wait(p_full, n & 1, wc)) break;
         tc_fence_after();
-        const uint64_t pb = ofs(st * kPBytes), qb = ofs(st * kQBytes);
+        const uint64_t qb = ofs(st * kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
-          mma_ss(tmem + kColDV, dP_k + pb + ofs(kk * 32), dO_m + qb + ofs(kk * 2048), idKV,
+          mma_ss(tmem + kColDV, dP_k + ofs(kk * 32), dO_m + qb + ofs(kk * 2048), idKV,
                  (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-          mma_ss(tmem + kColDK, dS_k + pb + ofs(kk * 32), dQ_m + qb + ofs(kk * 2048), idKV,
+          mma_ss(tmem + kColDK, dS_k + ofs(kk * 32), dQ_m + qb + ofs(kk * 2048), idKV,
                  (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
-        if (use > 0 && !mbar_wait(&dq_empty[st], (use - 1) & 1, wc)) break;
+        if (duse > 0 && !mbar_wait(&dq_empty[db], (duse - 1) & 1, wc)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
-          mma_ss(tmem + col_dq(st), dK_m + ofs(kk * 2048), dS_m + pb + ofs(kk * 2048), idDQ,
+          mma_ss(tmem + col_dq(db), dK_m + ofs(kk * 2048), dS_m + ofs(kk * 2048), idDQ,
                  kk > 0 ? 1u : 0u);
-        mma_commit(&dq_full[st]);
-        mma_commit(&ps_empty[st]);
+        mma_commit(&dq_full[db]);
+        mma_commit(ps_empty);
       }
       mma_commit(acc_full);
       mma_commit(mma_done);
@@ -284,30 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_inc<kRegSm>();
     // -------------------------------------------------- softmax / dS
     const int r = (warp & 3) * 32 + lane;  // key row within the tile
-    const int tid = (warp - 4) * 32 + lane;
     const int kj = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c2 = p.scale_log2;
     bool ok = true;
-    for (int n = 0; n < N; ++n) {
-      const int st = n & 1, use = n >> 1;
-      const int h = step_head(n), q0 = step_q0(n);
-      // Stage lse2 / Delta of this step's 64 queries (slot st) once every
-      // thread has finished with the slot's previous contents.
-      if (tid < kBQ) {
-        bool got = use == 0 || mbar_wait(&row_empty[st], (use - 1) & 1, wc);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        const int q = q0 + tid;
-        const size_t row = (static_cast<size_t>(b) * p.H + h) * p.T + q;
-        s_lse2[st * kBQ + tid] = q < p.T ? p.lse[row] * 1.4426950408889634f : INFINITY;
-        s_delta[st * kBQ + tid] = q < p.T ? p.delta[row] : 0.f;
-        mbar_arrive(&row_full[st]);
-      }
-      bool got = mbar_wait(&row_full[st], use & 1, wc);
-      got = got && mbar_wait(sp_full, n & 1, wc);
+    Cursor c = cur0;
+    for (int n = 0; n < N; ++n, c.next()) {
+      const int st = n % kQStages, use = n / kQStages;
+      const int q0 = c.q0();
+      // S^T/dP^T of this step, and (same stage barrier as Q/dO) its lse2/Delta.
+      bool got = mbar_wait(sp_full, n & 1, wc);
+      got = got && mbar_wait(&q_full[st], use & 1, wc);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -348,15 +358,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd[c * 16 + i / 2] = pack_bf16x2(dsv[0], dsv[1]);
           dd[c * 16 + i / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-      mbar_arrive(&row_empty[st]);
-      got = use == 0 || mbar_wait(&ps_empty[st], (use - 1) & 1, wc);
+      got = n == 0 || mbar_wait(ps_empty, (n - 1) & 1, wc);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       // Row r of P^T / dS^T: 64 bf16 = 8 chunks of 16 B, 128B-swizzled.
-      uint8_t* prow = smem + kOffP + st * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
-      uint8_t* drow = smem + kOffDS + st * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+      uint8_t* prow = smem + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
+      uint8_t* drow = smem + kOffDS + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         const int pos = (ch ^ (r & 7)) << 4;
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[st]);
+      mbar_arrive(p_full);
     }
     // dK / dV write-out: thread r holds key row r of both accumulators.
     const bool acc_ok = ok && mbar_wait(acc_full, 0, wc);
@@ -410,9 +419,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = (warp == 8 && lane == 0);
     float* sdq = reinterpret_cast<float*>(smem + kOffDQ);
     const float sc = p.scale;
-    for (int n = 0; n < N; ++n) {
+    Cursor c = cur0;
+    for (int n = 0; n < N; ++n, c.next()) {
       const int st = n & 1, use = n >> 1;
-      const int h = step_head(n), q0 = step_q0(n);
+      const int h = c.h, q0 = c.q0();
       bool got = mbar_wait(&dq_full[st], use & 1, wc);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();

@@ -290,14 +290,17 @@ struct ScopedTiming {
 size_t pad256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Workspace {
-  float *dq_acc, *dk_acc, *dv_acc, *delta;
+  float *dq_acc, *dk_acc, *dv_acc, *delta, *lse2;
+  int Tpad;
   size_t bytes;
 };
+
+int padded_T(int T) { return (T + 63) / 64 * 64; }
 
 Workspace carve(const Shape& s, void* base) {
   const size_t nq = static_cast<size_t>(s.B) * s.H * s.T * s.D;
   const size_t nk = static_cast<size_t>(s.B) * s.T * s.Hk * s.D;
-  const size_t nr = static_cast<size_t>(s.B) * s.H * s.T;
+  const size_t nr = static_cast<size_t>(s.B) * s.H * padded_T(s.T);
   Workspace w;
   uint8_t* p = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -309,6 +312,9 @@ Workspace carve(const Shape& s, void* base) {
   off += pad256(nk * 4);
   w.delta = reinterpret_cast<float*>(p + off);
   off += pad256(nr * 4);
+  w.lse2 = reinterpret_cast<float*>(p + off);
+  off += pad256(nr * 4);
+  w.Tpad = padded_T(s.T);
   w.bytes = off;
   return w;
 }
@@ -516,9 +522,12 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   pre.rows = static_cast<long long>(s.B) * s.T * s.H;
   pre.T = s.T;
   pre.H = s.H;
+  pre.Tpad = w.Tpad;
   pre.O = O;
   pre.dO = dO;
+  pre.lse = lse;
   pre.delta = w.delta;
+  pre.lse2 = w.lse2;
   {
     ScopedTiming tm(CSWATTN_K_BWD_PRE, cs);
     if (s.bf16)
@@ -543,6 +552,7 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     sp.dO = static_cast<const float*>(dO);
     sp.lse = lse;
     sp.delta = w.delta;
+    sp.Tpad = w.Tpad;
     sp.dq_acc = w.dq_acc;
     sp.dk_acc = w.dk_acc;
     sp.dv_acc = w.dv_acc;
@@ -573,7 +583,8 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     bp.nkv = (s.T + bwd::kBN - 1) / bwd::kBN;
     bp.scale_log2 = s.scale * 1.4426950408889634f;
     bp.scale = s.scale;
-    bp.lse = lse;
+    bp.Tpad = w.Tpad;
+    bp.lse2 = w.lse2;
     bp.delta = w.delta;
     bp.dq_acc = w.dq_acc;
     bp.dk_acc = w.dk_acc;

@@ -17,7 +17,7 @@
 // window-edge tiles only.
 //
 // Roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, then K_j, V_j through 2-stage rings
+//   warp 0      TMA producer: Q tiles once, then K_j, V_j through one 5-slot ring
 //   warp 1      TMEM owner + single-thread MMA issuer
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r
 //               owns TMEM lane r = query row r, so the row max and sum are
@@ -39,11 +39,12 @@ constexpr int kD = 128;
 constexpr int kThreads = 384;
 constexpr int kTileBytes = kBM * kD * 2;     // 32 KB: 128 rows x 128 bf16
 constexpr int kPanelBytes = kTileBytes / 2;  // 16 KB: 128 rows x 64 bf16 (one swizzle panel)
+constexpr int kSlots = 5;                    // K/V ring: K_j, V_j, K_j+1, ... (2.5 KV steps)
 constexpr int kOffQ = 0;                     // 2 tiles
-constexpr int kOffK = 2 * kTileBytes;        // 2 stages
-constexpr int kOffV = 4 * kTileBytes;        // 2 stages
-constexpr int kOffBar = 6 * kTileBytes;
+constexpr int kOffKV = 2 * kTileBytes;       // kSlots tiles
+constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 // Register budgets after setmaxnreg; the sum may not exceed the launch
 // allocation (384 threads x 168 registers).
@@ -82,16 +83,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2] per tile
-  uint64_t* p_full = bars + 11;   // [2] per tile
-  uint64_t* o_full = bars + 13;   // [2] per tile
-  uint64_t* mma_done = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+  uint64_t* kv_full = bars + 1;   // [kSlots]
+  uint64_t* kv_empty = bars + 6;  // [kSlots]
+  uint64_t* s_full = bars + 11;   // [2] per tile
+  uint64_t* p_full = bars + 13;   // [2] per tile
+  uint64_t* o_full = bars + 15;   // [2] per tile
+  uint64_t* mma_done = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
 
   const int warp = warp_id(), lane = lane_id();
 
@@ -119,11 +118,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
       mbar_init(&o_full[s], 1);
@@ -154,7 +153,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
-      int nk[2] = {0, 0}, nv[2] = {0, 0};
+      // Ring slot of tile i (K_j at i = 2(j-lo), V_j at i+1): i % kSlots,
+      // use i / kSlots; slots are consumed in the order they are filled.
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      int filled[kSlots] = {0, 0, 0, 0, 0};
       mbar_expect_tx(q_full, (valid[1] ? 2 : 1) * kTileBytes);
       for (int X = 0; X < 2; ++X) {
         if (!valid[X]) continue;
@@ -162,27 +166,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(&tmQ, q_full, dst, 0, head[X], qblk[X] * kBM, b);
         tma_load_4d(&tmQ, q_full, dst + kPanelBytes, 64, head[X], qblk[X] * kBM, b);
       }
-      for (int j = lo; j <= hi; ++j) {
-        const int it = j - lo, s = it & 1, use = it >> 1;
-        if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, wc)) break;
-        mbar_expect_tx(&k_full[s], kTileBytes);
-        uint8_t* kd = smem + kOffK + s * kTileBytes;
-        tma_load_4d(&tmK, &k_full[s], kd, 0, hk, j * kBM, b);
-        tma_load_4d(&tmK, &k_full[s], kd + kPanelBytes, 64, hk, j * kBM, b);
-        ++nk[s];
-        if (use > 0 && !mbar_wait(&v_empty[s], (use - 1) & 1, wc)) break;
-        mbar_expect_tx(&v_full[s], kTileBytes);
-        uint8_t* vd = smem + kOffV + s * kTileBytes;
-        tma_load_4d(&tmV, &v_full[s], vd, 0, hk, j * kBM, b);
-        tma_load_4d(&tmV, &v_full[s], vd + kPanelBytes, 64, hk, j * kBM, b);
-        ++nv[s];
+      int slot = 0, use = 0;
+      for (int i = 0; i < 2 * (hi - lo + 1); ++i) {
+        if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, wc)) break;
+        const int j = lo + (i >> 1);
+        const CUtensorMap* tm = (i & 1) ? &tmV : &tmK;
+        mbar_expect_tx(&kv_full[slot], kTileBytes);
+        uint8_t* dst = smem + kOffKV + slot * kTileBytes;
+        tma_load_4d(tm, &kv_full[slot], dst, 0, hk, j * kBM, b);
+        tma_load_4d(tm, &kv_full[slot], dst + kPanelBytes, 64, hk, j * kBM, b);
+        ++filled[slot];
+        if (++slot == kSlots) {
+          slot = 0;
+          ++use;
+        }
       }
       // Drain: every issued copy has landed before the CTA may exit.
       drain_wait(q_full, 0, p.wait_ns);
-      for (int s = 0; s < 2; ++s) {
-        if (nk[s] > 0) drain_wait(&k_full[s], (nk[s] - 1) & 1, p.wait_ns);
-        if (nv[s] > 0) drain_wait(&v_full[s], (nv[s] - 1) & 1, p.wait_ns);
-      }
+      for (int s2 = 0; s2 < kSlots; ++s2)
+        if (filled[s2] > 0) drain_wait(&kv_full[s2], (filled[s2] - 1) & 1, p.wait_ns);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -190,20 +192,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);   // Q K^T: both K-major
       constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);  // P V: V MN-major
       const uint32_t sQa = smem_u32(smem + kOffQ);
-      const uint32_t sKa = smem_u32(smem + kOffK);
-      const uint32_t sVa = smem_u32(smem + kOffV);
+      const uint32_t sKVa = smem_u32(smem + kOffKV);
       bool ok = mbar_wait(q_full, 0, wc);
       tc_fence_after();
 
       // Descriptors: a base per buffer plus a compile-time offset per k-step
       // (the start-address field holds address >> 4).
       const uint64_t dQ0 = sdesc_sw128(sQa, 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(sKa, 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(sVa, kPanelBytes, 1024);
+      const uint64_t dK0 = sdesc_sw128(sKVa, 16, 1024);           // K: K-major
+      const uint64_t dV0 = sdesc_sw128(sKVa, kPanelBytes, 1024);  // V: MN-major
+      // Ring position of K_j (kind 0) or V_j (kind 1).
+      auto ring = [&](int j, int kind, int& slot, int& use) {
+        const int i = 2 * (j - lo) + kind;
+        slot = i % kSlots;
+        use = i / kSlots;
+      };
 
       auto issue_S = [&](int X, int j) -> bool {
-        const int it = j - lo, s = it & 1, use = it >> 1;
-        if (!mbar_wait(&k_full[s], use & 1, wc)) return false;
+        int s, use;
+        ring(j, 0, s, use);
+        if (!mbar_wait(&kv_full[s], use & 1, wc)) return false;
         tc_fence_after();
         const uint64_t qd = dQ0 + static_cast<uint64_t>((X * kTileBytes) >> 4);
         const uint64_t kd = dK0 + static_cast<uint64_t>((s * kTileBytes) >> 4);
@@ -217,9 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto issue_PV = [&](int X, int j) -> bool {
-        const int it = j - lo, s = it & 1, use = it >> 1;
+        int s, use;
+        ring(j, 1, s, use);
         const int n = j - lo_t[X];
-        if (!mbar_wait(&v_full[s], use & 1, wc)) return false;
+        if (!mbar_wait(&kv_full[s], use & 1, wc)) return false;
         if (!mbar_wait(&p_full[X], n & 1, wc)) return false;
         tc_fence_after();
         const uint64_t vd = dV0 + static_cast<uint64_t>((s * kTileBytes) >> 4);
@@ -232,13 +241,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
+      int rs, ru;
       if (ok) {
         for (int X = 0; X < 2 && ok; ++X)
           if (valid[X] && lo_t[X] == lo) ok = issue_S(X, lo);
-        if (ok) mma_commit(&k_empty[0]);
+        ring(lo, 0, rs, ru);
+        if (ok) mma_commit(&kv_empty[rs]);
       }
       for (int j = lo; ok && j <= hi; ++j) {
-        const int it = j - lo;
         for (int X = 0; X < 2 && ok; ++X) {
           if (!valid[X]) continue;
           if (j >= lo_t[X] && j <= hi_t[X]) {
@@ -248,8 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && j + 1 >= lo_t[X] && j + 1 <= hi_t[X]) ok = issue_S(X, j + 1);
         }
         if (!ok) break;
-        mma_commit(&v_empty[it & 1]);
-        if (j + 1 <= hi) mma_commit(&k_empty[(it + 1) & 1]);
+        ring(j, 1, rs, ru);
+        mma_commit(&kv_empty[rs]);  // V_j consumed
+        if (j + 1 <= hi) {
+          ring(j + 1, 0, rs, ru);
+          mma_commit(&kv_empty[rs]);  // K_j+1 consumed
+        }
       }
       // Drain: all issued MMAs complete before TMEM is released.
       mma_commit(mma_done);

@@ -20,7 +20,11 @@ namespace cswattn {
 constexpr int kPrologueThreads = 256;
 constexpr int kPrologueTok = 8;
 constexpr int kMaxHalfD = 64;
-constexpr int kRowsInFlight = 4;
+#ifndef CSW_ROWS_IN_FLIGHT
+#define CSW_ROWS_IN_FLIGHT 1
+#endif
+// Rows each lane loads before computing, in the HBM-bound row kernels.
+constexpr int kRowsInFlight = CSW_ROWS_IN_FLIGHT;
 
 struct PrologueParams {
   int B, T, H, Hk;

@@ -14,10 +14,11 @@ namespace cswattn {
 
 struct SimtParams {
   int B, T, H, Hk, W;
+  int Tpad;                    // row stride of delta (B,H,Tpad)
   float scale;
   const float *q, *k, *v;      // q_out (B,T,H,D), k_out, v_out (B,T,Hk,D)
   const float *O, *dO, *lse;   // backward inputs
-  const float* delta;          // (B,H,T) dO.O
+  const float* delta;          // (B,H,Tpad) dO.O
   float *out_O, *out_lse;      // forward outputs
   float *dq_acc;               // (B,H,T,D) dq~ (scaled)
   float *dk_acc, *dv_acc;      // (B,T,Hk,D) dk~ (scaled), dv_eff
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const SimtParams p) {
     acc[d] = 0.f;
   }
   const size_t row = (static_cast<size_t>(b) * p.H + h) * p.T + i;
-  const float li = p.lse[row], di = p.delta[row];
+  const float li = p.lse[row];
+  const float di = p.delta[(static_cast<size_t>(b) * p.H + h) * p.Tpad + i];
   const int lo = max(0, i - p.W + 1);
   for (int j = lo; j <= i; ++j) {
     const size_t kv = ((static_cast<size_t>(b) * p.T + j) * p.Hk + hk) * D;
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dkv_kernel(const SimtParams p) {
         dp = fmaf(p.dO[qo + d], vv[d], dp);
       }
       const float pij = expf(s * p.scale - p.lse[row]);
-      const float ds = pij * (dp - p.delta[row]);
+      const float ds = pij * (dp - p.delta[(static_cast<size_t>(b) * p.H + h) * p.Tpad + i]);
 #pragma unroll
       for (int d = 0; d < D; ++d) {
         dk[d] = fmaf(ds, p.q[qo + d], dk[d]);

@@ -97,8 +97,9 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
 
 /* Bytes of device scratch attn_bwd needs for this layer: float32
  * accumulators of dq_out (B, n_head, T, head_dim), dk_out and dv_out
- * (B, T, n_kv_head, head_dim) and the row terms dO.O (B, n_head, T),
- * each padded to 256 bytes. Returns 0 for an invalid layer. */
+ * (B, T, n_kv_head, head_dim), and two row terms (dO.O and lse*log2(e)),
+ * each (B, n_head, Tpad) with Tpad = T rounded up to a multiple of 64;
+ * every part padded to 256 bytes. Returns 0 for an invalid layer. */
 size_t attn_bwd_workspace_bytes(const cswattn_layer* layer);
 
 /* Backward of prologue + forward for the loss L with dL/dO = dO:
