@@ -25,7 +25,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
 
 # Every symbol the header declares; the CPU tests check the library exports them.
-EXPORTS = ("attn_prologue", "attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd",
+EXPORTS = ("attn_prologue", "attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
            "cswattn_sync_status", "cswattn_set_wait_limit_ns", "cswattn_set_timing",
            "cswattn_kernel_times", "cswattn_last_error", "cswattn_version")
 KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi")
@@ -73,7 +73,9 @@ def lib():
         L.cswattn_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double),
                                            ctypes.POINTER(ctypes.c_int)]
         L.cswattn_kernel_times.restype = ctypes.c_int
-        for name in ("attn_prologue", "attn_fwd", "attn_bwd", "cswattn_sync_status"):
+        L.attn_bwd_noalloc.argtypes = [lp] + [vp] * 7 + [fp, fp, vp, fp, vp] + [vp] * 5 + [vp]
+        for name in ("attn_prologue", "attn_fwd", "attn_bwd", "attn_bwd_noalloc",
+                     "cswattn_sync_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -153,6 +155,22 @@ def attn_bwd(spec: LayerSpec, q, k, ve, gate, q_out, k_out, v_out, rstd_q, rstd_
                           _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV),
                           _ptr(dve), _ptr(dgate), _ptr(workspace), workspace_bytes,
                           _stream(stream)))
+
+
+# Size of the fixed scratch array behind attn_bwd_noalloc (bytes).
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def attn_bwd_noalloc(spec: LayerSpec, q, k, ve, gate, q_out, k_out, v_out, rstd_q, rstd_k, O,
+                     lse, dO, dQ, dK, dV, dve, dgate, stream=None):
+    """attn_bwd for callers that cannot allocate device memory: the scratch is
+    a fixed array inside the library (see the C header for the limit and for
+    why overlapping calls must be ordered)."""
+    layer = spec.c()
+    _check(lib().attn_bwd_noalloc(ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(ve), _ptr(gate),
+                                  _ptr(q_out), _ptr(k_out), _ptr(v_out), _ptr(rstd_q),
+                                  _ptr(rstd_k), _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
+                                  _ptr(dV), _ptr(dve), _ptr(dgate), _stream(stream)))
 
 
 def cswattn_sync_status(stream=None):

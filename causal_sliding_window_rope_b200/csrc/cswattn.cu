@@ -319,6 +319,36 @@ Workspace carve(const Shape& s, void* base) {
   return w;
 }
 
+// ---------------------------------------------------------------- fixed scratch
+
+// Backward scratch of attn_bwd_noalloc, for callers that cannot allocate
+// device memory. Every GPU that loads this library holds it until exit.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CSWATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device with that device current and cached.
+cswattn_status noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(CSWATTN_ERR_UNSUPPORTED, "device ordinal %d is outside the scratch table", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CSWATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -627,6 +657,27 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
       launch_epilogue<float>(s, ep, cs);
   }
   return launched("epilogue launch");
+}
+
+cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const void* k,
+                                const void* ve, const void* gate, const void* q_out,
+                                const void* k_out, const void* v_out, const float* rstd_q,
+                                const float* rstd_k, const void* O, const float* lse,
+                                const void* dO, void* dQ, void* dK, void* dV, void* dve,
+                                void* dgate, void* stream) {
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  const size_t need = carve(s, nullptr).bytes;
+  if (need > CSWATTN_NOALLOC_SCRATCH_BYTES)
+    return fail(CSWATTN_ERR_UNSUPPORTED,
+                "attn_bwd_noalloc: this layer needs %zu bytes of scratch, the fixed array holds %u; "
+                "use attn_bwd with a caller workspace",
+                need, static_cast<unsigned>(CSWATTN_NOALLOC_SCRATCH_BYTES));
+  void* ws = nullptr;
+  if ((st = noalloc_scratch(&ws)) != CSWATTN_OK) return st;
+  return attn_bwd(layer, q, k, ve, gate, q_out, k_out, v_out, rstd_q, rstd_k, O, lse, dO, dQ, dK,
+                  dV, dve, dgate, ws, CSWATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

@@ -119,6 +119,42 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
                         void* dgate, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* Size of the fixed scratch array that attn_bwd_noalloc uses: 32 MiB. */
+#define CSWATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* attn_bwd without a caller-provided workspace, for callers that cannot
+ * allocate device memory. The web pages this library follows describe no
+ * such entry point; it exists for library users only.
+ *
+ * Who needs it: code whose device memory is owned entirely by another
+ * allocator (a framework's caching allocator or a fixed arena that must
+ * account for every byte), and code that may not call cudaMalloc in its
+ * step loop because cudaMalloc can synchronize the device and stall other
+ * work. Such callers can still pass their input and output tensors, but
+ * they cannot hand over the few tens of megabytes of float32 scratch that
+ * attn_bwd needs.
+ *
+ * Behaviour: identical arguments and results to attn_bwd, minus
+ * `workspace`/`workspace_bytes`. The scratch is a static array of
+ * CSWATTN_NOALLOC_SCRATCH_BYTES inside this library; every GPU that loads
+ * the library holds it until the process exits. Layers whose
+ * attn_bwd_workspace_bytes() exceeds that size are rejected with
+ * CSWATTN_ERR_UNSUPPORTED before anything is enqueued (use attn_bwd with
+ * your own workspace for those). No call allocates device memory.
+ * The first call on a device looks up the array's device address on that
+ * device (the device current at the call); make that first call before
+ * any stream capture. All calls on a device share the one array: two calls
+ * that may overlap on the GPU (different streams, no ordering between
+ * them) race and corrupt each other's results, so order them, for example
+ * by issuing them on one stream. The array keeps whatever the last call
+ * left in it; each call clears what must start at zero itself. */
+cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const void* k,
+                                const void* ve, const void* gate, const void* q_out,
+                                const void* k_out, const void* v_out, const float* rstd_q,
+                                const float* rstd_k, const void* O, const float* lse,
+                                const void* dO, void* dQ, void* dK, void* dV, void* dve,
+                                void* dgate, void* stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the
  * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last check, CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
