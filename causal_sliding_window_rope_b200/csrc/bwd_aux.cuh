@@ -6,8 +6,8 @@
 //   "1. GPT 모델": RoPE, QK normalisation, value-embedding code):
 //   dq = RMSNorm'(RoPE^-1(dq~)), dk likewise, dv = dv_eff,
 //   dve = 3 s dv_eff, dgate = 3 s (1 - s) sum_d dv_eff ve with s = sigmoid(gate).
-// Both use the prologue's row layout: a row of D elements is owned by
-// D / VEC lanes holding one 16-byte vector each; reductions are shuffles.
+// Both use the prologue's split-halves row layout (each lane holds matching
+// slices of both halves of a row); reductions are shuffles over a row's lanes.
 #pragma once
 #include "prologue.cuh"
 
@@ -25,52 +25,59 @@ struct PreParams {
   float* lse2;       // (B, H, Tpad)
 };
 
+// One CTA per kPrologueTok consecutive tokens; each row (token, head) is
+// owned by LPR lanes in the prologue's split-halves layout (two vector loads
+// per lane per tensor), reduced with shuffles.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) preprocess_kernel(const PreParams p) {
-  using V = Vec16<T>;
-  constexpr int VEC = V::N;
-  constexpr int LPR = D / VEC;
-  constexpr int RPW = 32 / LPR;           // rows per warp per slot
-  constexpr int U = kRowsInFlight;        // slots per pass
+__global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreParams p) {
+  using RL = RowLayout<T, D>;
+  using HVec = HalfVec<T, RL::HV>;
+  constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
+  constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
+  __shared__ int s_b[kPrologueTok], s_t[kPrologueTok];
+  __shared__ bool s_valid[kPrologueTok];
+  const long long n_tok = p.rows / p.H;
+  const long long tok0 = static_cast<long long>(blockIdx.x) * kPrologueTok;
+  if (threadIdx.x < kPrologueTok) {
+    const long long tok = tok0 + threadIdx.x;
+    s_valid[threadIdx.x] = tok < n_tok;
+    const long long tk = tok < n_tok ? tok : 0;
+    s_b[threadIdx.x] = static_cast<int>(tk / p.T);
+    s_t[threadIdx.x] = static_cast<int>(tk % p.T);
+  }
+  __syncthreads();
   const int sub = threadIdx.x % LPR;
-  const int lrow = (threadIdx.x % 32) / LPR;
-  const long long warp_global = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / 32;
-  const long long n_warps = static_cast<long long>(gridDim.x) * 8;
-  // Uniform trip count across the warp; U rows' loads in flight per lane.
-  for (long long base = warp_global * RPW * U; base < p.rows; base += n_warps * RPW * U) {
-    float o[U][VEC], g[U][VEC];
+  const int grp = threadIdx.x / LPR;
+  const int total_rows = kPrologueTok * p.H;
+  RowCursor cur{0, 0};
+  cur.advance(grp, p.H);
+  for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
+    const bool in_range = base + grp < total_rows;
+    const int tt = in_range ? cur.tt : 0, h = in_range ? cur.kind_row : 0;
+    cur.advance(ROWS_PER_PASS, p.H);
+    const bool valid = in_range && s_valid[tt];
+    const long long row = (tok0 + tt) * p.H + h;  // (b*T + t)*H + h
+    float acc = 0.f;
+    if (valid) {
+      const size_t lo = static_cast<size_t>(row) * D + sub * HV;
+      float o0[HV], o1[HV], g0[HV], g1[HV];
+      HVec::load(static_cast<const T*>(p.O) + lo, o0);
+      HVec::load(static_cast<const T*>(p.O) + lo + HALF, o1);
+      HVec::load(static_cast<const T*>(p.dO) + lo, g0);
+      HVec::load(static_cast<const T*>(p.dO) + lo + HALF, g1);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long row = base + u * RPW + lrow;
-      if (row < p.rows) {
-        V::load(static_cast<const T*>(p.O) + row * D + sub * VEC, o[u]);
-        V::load(static_cast<const T*>(p.dO) + row * D + sub * VEC, g[u]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) o[u][i] = g[u][i] = 0.f;
-      }
+      for (int i = 0; i < HV; ++i) acc = fmaf(o0[i], g0[i], fmaf(o1[i], g1[i], acc));
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const long long row = base + u * RPW + lrow;
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) acc = fmaf(o[u][i], g[u][i], acc);
-#pragma unroll
-      for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, LPR);
-      if (row < p.rows && sub == 0) {
-        // row = (b*T + t)*H + h  ->  (b*H + h)*Tpad + t
-        const long long h = row % p.H;
-        const long long bt = row / p.H;
-        const long long t = bt % p.T, b = bt / p.T;
-        const long long o = (b * p.H + h) * p.Tpad;
-        p.delta[o + t] = acc;
-        p.lse2[o + t] = p.lse[(b * p.H + h) * p.T + t] * 1.4426950408889634f;
-        if (t == p.T - 1) {
-          for (long long tp = p.T; tp < p.Tpad; ++tp) {
-            p.delta[o + tp] = 0.f;
-            p.lse2[o + tp] = INFINITY;
-          }
+    acc = row_sum<LPR>(acc);
+    if (valid && sub == 0) {
+      const long long b = s_b[tt], t = s_t[tt];
+      const long long o = (b * p.H + h) * p.Tpad;
+      p.delta[o + t] = acc;
+      p.lse2[o + t] = p.lse[(b * p.H + h) * p.T + t] * 1.4426950408889634f;
+      if (t == p.T - 1) {
+        for (long long tp = p.T; tp < p.Tpad; ++tp) {
+          p.delta[o + tp] = 0.f;
+          p.lse2[o + tp] = INFINITY;
         }
       }
     }
@@ -90,161 +97,151 @@ struct EpiParams {
 
 template <int VEC>
 __device__ __forceinline__ void load_f32(const float* src, float (&x)[VEC]) {
+  if constexpr (VEC % 4 == 0) {
 #pragma unroll
-  for (int i = 0; i < VEC; i += 4) {
-    float4 u = *reinterpret_cast<const float4*>(src + i);
-    x[i] = u.x;
-    x[i + 1] = u.y;
-    x[i + 2] = u.z;
-    x[i + 3] = u.w;
+    for (int i = 0; i < VEC; i += 4) {
+      float4 u = *reinterpret_cast<const float4*>(src + i);
+      x[i] = u.x;
+      x[i + 1] = u.y;
+      x[i + 2] = u.z;
+      x[i + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VEC; i += 2) {
+      float2 u = *reinterpret_cast<const float2*>(src + i);
+      x[i] = u.x;
+      x[i + 1] = u.y;
+    }
   }
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiParams p) {
-  using V = Vec16<T>;
-  constexpr int VEC = V::N;
-  constexpr int LPR = D / VEC;
-  constexpr int HALF = D / 2;
+  using RL = RowLayout<T, D>;
+  using HVec = HalfVec<T, RL::HV>;
+  constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
 
-  __shared__ float s_cos[kPrologueTok][HALF];
-  __shared__ float s_sin[kPrologueTok][HALF];
+  __shared__ __align__(16) TokenTable<HALF> tab;
 
   const long long n_tok = static_cast<long long>(p.B) * p.T;
   const long long tok0 = static_cast<long long>(blockIdx.x) * kPrologueTok;
-  for (int e = threadIdx.x; e < kPrologueTok * HALF; e += kPrologueThreads) {
-    const int tt = e / HALF, i = e % HALF;
-    const long long tok = tok0 + tt;
-    const int t = tok < n_tok ? static_cast<int>(tok % p.T) : 0;
-    float s, c;
-    sincosf(static_cast<float>(t) * p.omega[i], &s, &c);
-    s_cos[tt][i] = c;
-    s_sin[tt][i] = s;
-  }
+  tab.fill(tok0, n_tok, p.T, p.omega);
   __syncthreads();
 
   const int rows_per_tok = p.H + 2 * p.Hk;
   const int total_rows = kPrologueTok * rows_per_tok;
   const int sub = threadIdx.x % LPR;
   const int grp = threadIdx.x / LPR;
+  RowCursor cur{0, 0};
+  cur.advance(grp, rows_per_tok);
 
-  // Like the prologue: U rows per lane per pass, loads first.
-  constexpr int U = kRowsInFlight;
-  for (int base = 0; base < total_rows; base += ROWS_PER_PASS * U) {
-    float dy[U][VEC], x[U][VEC];
-    float rs[U], gl[U];
-    int kind[U], tt[U];
-    bool valid[U];
-    size_t row[U], off[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int r = base + u * ROWS_PER_PASS + grp;
-      const bool in_range = r < total_rows;
-      const int rr = in_range ? r : 0;
-      tt[u] = rr / rows_per_tok;
-      const int kind_row = rr % rows_per_tok;
-      const long long tok = tok0 + tt[u];
-      valid[u] = in_range && tok < n_tok;
-      const long long tk = valid[u] ? tok : 0;
-      const int t = static_cast<int>(tk % p.T);
-      const long long b = tk / p.T;
-      int head, nheads;
-      if (kind_row < p.H) {
-        kind[u] = 0; head = kind_row; nheads = p.H;
-      } else if (kind_row < p.H + p.Hk) {
-        kind[u] = 1; head = kind_row - p.H; nheads = p.Hk;
+  for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
+    const bool in_range = base + grp < total_rows;
+    const int tt = in_range ? cur.tt : 0;
+    const int kind_row = in_range ? cur.kind_row : 0;
+    cur.advance(ROWS_PER_PASS, rows_per_tok);
+    const bool valid = in_range && tab.valid[tt];
+    const int t = tab.t[tt];
+    const long long b = tab.b[tt];
+    int kind, head, nheads;
+    if (kind_row < p.H) {
+      kind = 0; head = kind_row; nheads = p.H;
+    } else if (kind_row < p.H + p.Hk) {
+      kind = 1; head = kind_row - p.H; nheads = p.Hk;
+    } else {
+      kind = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
+    }
+    const size_t row = static_cast<size_t>(valid ? tok0 + tt : 0) * nheads + head;  // (b,t,head)
+    const size_t off_lo = row * D + static_cast<size_t>(sub) * HV;
+    const size_t off_hi = off_lo + HALF;
+
+    // Gradient w.r.t. the rotated, normalised row (or dv_eff for value rows),
+    // and the row's input (q or k) or ve.
+    float dl[HV], dh[HV], xl[HV], xh[HV];
+    float rs = 0.f, gl = 0.f;
+    if (valid) {
+      const float* src;
+      size_t so;
+      if (kind == 0) {
+        src = p.dq_acc;
+        so = ((static_cast<size_t>(b) * p.H + head) * p.T + t) * D + sub * HV;
       } else {
-        kind[u] = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
+        src = kind == 1 ? p.dk_acc : p.dv_acc;
+        so = off_lo;
       }
-      row[u] = static_cast<size_t>(tk) * nheads + head;  // (b,t,head)
-      off[u] = row[u] * D + static_cast<size_t>(sub) * VEC;
-      rs[u] = 0.f;
-      gl[u] = 0.f;
-      if (valid[u]) {
-        // Gradient w.r.t. the rotated, normalised row (or dv_eff for kind 2).
-        const float* src;
-        if (kind[u] == 0)
-          src = p.dq_acc + ((static_cast<size_t>(b) * p.H + head) * p.T + t) * D + sub * VEC;
-        else
-          src = (kind[u] == 1 ? p.dk_acc : p.dv_acc) + off[u];
-        load_f32<VEC>(src, dy[u]);
-        if (kind[u] != 2) {
-          V::load(static_cast<const T*>(kind[u] == 0 ? p.q : p.k) + off[u], x[u]);
-          rs[u] = (kind[u] == 0 ? p.rstd_q : p.rstd_k)[row[u]];
-        } else if (p.has_ve) {
-          V::load(static_cast<const T*>(p.ve) + off[u], x[u]);  // ve for the value rows
-          gl[u] = V::scalar(p.gate, row[u]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < VEC; ++i) x[u][i] = 0.f;
-        }
+      load_f32<HV>(src + so, dl);
+      load_f32<HV>(src + so + HALF, dh);
+      if (kind != 2) {
+        HVec::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off_lo, xl);
+        HVec::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off_hi, xh);
+        rs = (kind == 0 ? p.rstd_q : p.rstd_k)[row];
+      } else if (p.has_ve) {
+        HVec::load(static_cast<const T*>(p.ve) + off_lo, xl);
+        HVec::load(static_cast<const T*>(p.ve) + off_hi, xh);
+        gl = Vec16<T>::scalar(p.gate, row);
       } else {
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) dy[u][i] = x[u][i] = 0.f;
+        for (int i = 0; i < HV; ++i) xl[i] = xh[i] = 0.f;
       }
+    } else {
+#pragma unroll
+      for (int i = 0; i < HV; ++i) dl[i] = dh[i] = xl[i] = xh[i] = 0.f;
     }
 
+    // RoPE^-1 on this lane's pairs (kind 2 rows skip it below).
+    float cv[HV], sv[HV], nl[HV], nh[HV];
+    tab.template load<HV>(tt, sub * HV, cv, sv);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      // RoPE^-1 (the transpose rotation).
-      float dn[VEC];
-      if constexpr (LPR >= 2) {
-        float partner[VEC];
+    for (int i = 0; i < HV; ++i) {
+      nl[i] = fmaf(dl[i], cv[i], dh[i] * sv[i]);
+      nh[i] = fmaf(-dl[i], sv[i], dh[i] * cv[i]);
+    }
+    // One reduction serves both row kinds: for q/k rows sum_d dn*n with
+    // n = r x (the RMSNorm term); for value rows sum_d dv_eff*ve.
+    const bool vrow = kind == 2;
+    float dot = 0.f;
 #pragma unroll
-        for (int i = 0; i < VEC; ++i)
-          partner[i] = __shfl_xor_sync(0xffffffffu, dy[u][i], LPR / 2, LPR);
-        const bool lower = sub < LPR / 2;
-        const int pair0 = (lower ? sub : sub - LPR / 2) * VEC;
+    for (int i = 0; i < HV; ++i)
+      dot = vrow ? fmaf(dl[i], xl[i], fmaf(dh[i], xh[i], dot))
+                 : fmaf(nl[i], xl[i] * rs, fmaf(nh[i], xh[i] * rs, dot));
+    dot = row_sum<LPR>(dot);
+    if (!valid) continue;
+    if (vrow) {
+      HVec::store(static_cast<T*>(p.dv) + off_lo, dl);
+      HVec::store(static_cast<T*>(p.dv) + off_hi, dh);
+      if (p.has_ve) {
+        const float sg = 1.0f / (1.0f + expf(-gl));
+        const float coef = 3.0f * sg;
+        float ol[HV], oh[HV];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-          const float c = s_cos[tt[u]][pair0 + i], s = s_sin[tt[u]][pair0 + i];
-          // lower: dy_i c + dy_{i+D/2} s ; upper: -dy_{i-D/2} s + dy_i c
-          dn[i] = lower ? fmaf(dy[u][i], c, partner[i] * s) : fmaf(-partner[i], s, dy[u][i] * c);
+        for (int i = 0; i < HV; ++i) {
+          ol[i] = coef * dl[i];
+          oh[i] = coef * dh[i];
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const float c = s_cos[tt[u]][i], s = s_sin[tt[u]][i];
-          dn[i] = fmaf(dy[u][i], c, dy[u][i + HALF] * s);
-          dn[i + HALF] = fmaf(-dy[u][i], s, dy[u][i + HALF] * c);
+        HVec::store(static_cast<T*>(p.dve) + off_lo, ol);
+        HVec::store(static_cast<T*>(p.dve) + off_hi, oh);
+        if (sub == 0) {
+          const float dg = dot * coef * (1.0f - sg);
+          if constexpr (sizeof(T) == 2)
+            static_cast<__nv_bfloat16*>(p.dgate)[row] = __float2bfloat16_rn(dg);
+          else
+            static_cast<float*>(p.dgate)[row] = dg;
         }
       }
-      // One shuffle reduction serves both row kinds: for q/k rows the
-      // RMSNorm term sum_d dn*n (n = r x); for value rows sum_d dv_eff*ve.
-      const bool vrow = kind[u] == 2;
-      float dot = 0.f;
+    } else {
+      // RMSNorm backward: dx = r (dn - n mean(dn * n)), n = r x.
+      const float mean = dot / static_cast<float>(D);
+      float ol[HV], oh[HV];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i)
-        dot = vrow ? fmaf(dy[u][i], x[u][i], dot) : fmaf(dn[i], x[u][i] * rs[u], dot);
-#pragma unroll
-      for (int o = LPR / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o, LPR);
-      if (!valid[u]) continue;
-      if (vrow) {
-        V::store(static_cast<T*>(p.dv) + off[u], dy[u]);
-        if (p.has_ve) {
-          const float sg = 1.0f / (1.0f + expf(-gl[u]));
-          const float coef = 3.0f * sg;
-          float o[VEC];
-#pragma unroll
-          for (int i = 0; i < VEC; ++i) o[i] = coef * dy[u][i];
-          V::store(static_cast<T*>(p.dve) + off[u], o);
-          if (sub == 0) {
-            const float dg = dot * coef * (1.0f - sg);
-            if constexpr (sizeof(T) == 2)
-              static_cast<__nv_bfloat16*>(p.dgate)[row[u]] = __float2bfloat16_rn(dg);
-            else
-              static_cast<float*>(p.dgate)[row[u]] = dg;
-          }
-        }
-      } else {
-        // RMSNorm backward: dx = r (dn - n mean(dn * n)), n = r x.
-        const float mean = dot / static_cast<float>(D);
-        float o[VEC];
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) o[i] = rs[u] * (dn[i] - x[u][i] * rs[u] * mean);
-        V::store(static_cast<T*>(kind[u] == 0 ? p.dq : p.dk) + off[u], o);
+      for (int i = 0; i < HV; ++i) {
+        ol[i] = rs * (nl[i] - xl[i] * rs * mean);
+        oh[i] = rs * (nh[i] - xh[i] * rs * mean);
       }
+      T* dst = static_cast<T*>(kind == 0 ? p.dq : p.dk);
+      HVec::store(dst + off_lo, ol);
+      HVec::store(dst + off_hi, oh);
     }
   }
 }

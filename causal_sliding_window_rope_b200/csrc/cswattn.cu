@@ -195,18 +195,15 @@ void launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t st) {
 
 template <typename T>
 void launch_preprocess(const Shape& s, const PreParams& pp, cudaStream_t st) {
-  const int lpr = s.D / Vec16<T>::N;
-  const long long rows_per_block = 256 / lpr;
-  long long blocks = (pp.rows + rows_per_block - 1) / rows_per_block;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  const unsigned grid = static_cast<unsigned>(blocks);
+  const long long ntok = static_cast<long long>(s.B) * s.T;
+  const unsigned grid = static_cast<unsigned>((ntok + kPrologueTok - 1) / kPrologueTok);
   switch (s.D) {
-    case 4: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 4><<<grid, 256, 0, st>>>(pp); break;
-    case 8: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 8><<<grid, 256, 0, st>>>(pp); break;
-    case 16: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 16><<<grid, 256, 0, st>>>(pp); break;
-    case 32: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 32><<<grid, 256, 0, st>>>(pp); break;
-    case 64: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 64><<<grid, 256, 0, st>>>(pp); break;
-    default: preprocess_kernel<T, 128><<<grid, 256, 0, st>>>(pp); break;
+    case 4: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 4><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 8: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 8><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 16: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 16><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 32: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 32><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 64: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 64><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    default: preprocess_kernel<T, 128><<<grid, kPrologueThreads, 0, st>>>(pp); break;
   }
 }
 

@@ -8,10 +8,11 @@
 // One CTA handles kTok consecutive tokens (b, t). It first computes
 // cos/sin(t * omega_i) for its tokens into shared memory, then walks the
 // H query rows, Hk key rows and Hk value rows of each token. A row of D
-// elements is owned by LPR = D / VEC lanes, each holding one 16-byte vector,
-// so every load and store is a coalesced 16-byte access. The RMS is a
-// shuffle reduction over the row's lanes; the RoPE partner of element i
-// (i +- D/2) sits in lane (lane ^ LPR/2) at the same vector slot.
+// elements is owned by LPR = D / (2 HV) lanes; lane l holds the HV-element
+// slices [l HV, (l+1) HV) of both halves of the row (elements i and
+// i + D/2), so every RoPE pair is inside one lane and each lane keeps two
+// vector loads in flight per row. Loads and stores are coalesced vector
+// accesses; the RMS is a shuffle reduction over the row's LPR lanes.
 #pragma once
 #include "common.cuh"
 
@@ -20,11 +21,6 @@ namespace cswattn {
 constexpr int kPrologueThreads = 256;
 constexpr int kPrologueTok = 8;
 constexpr int kMaxHalfD = 64;
-#ifndef CSW_ROWS_IN_FLIGHT
-#define CSW_ROWS_IN_FLIGHT 1
-#endif
-// Rows each lane loads before computing, in the HBM-bound row kernels.
-constexpr int kRowsInFlight = CSW_ROWS_IN_FLIGHT;
 
 struct PrologueParams {
   int B, T, H, Hk;
@@ -80,138 +76,204 @@ struct Vec16<float> {
   }
 };
 
+// HV consecutive elements of type T <-> float[HV], as one vector access
+// (16, 8 or 4 bytes).
+template <typename T, int HV>
+struct HalfVec;
+template <>
+struct HalfVec<__nv_bfloat16, 8> {
+  __device__ static void load(const __nv_bfloat16* p, float (&x)[8]) { Vec16<__nv_bfloat16>::load(p, x); }
+  __device__ static void store(__nv_bfloat16* p, const float (&x)[8]) { Vec16<__nv_bfloat16>::store(p, x); }
+};
+template <>
+struct HalfVec<float, 4> {
+  __device__ static void load(const float* p, float (&x)[4]) { Vec16<float>::load(p, x); }
+  __device__ static void store(float* p, const float (&x)[4]) { Vec16<float>::store(p, x); }
+};
+template <>
+struct HalfVec<float, 2> {
+  __device__ static void load(const float* p, float (&x)[2]) {
+    const float2 u = *reinterpret_cast<const float2*>(p);
+    x[0] = u.x;
+    x[1] = u.y;
+  }
+  __device__ static void store(float* p, const float (&x)[2]) {
+    *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+  }
+};
+
+// Row geometry of the split-halves layout for element type T and width D.
+template <typename T, int D>
+struct RowLayout {
+  static constexpr int HALF = D / 2;
+  static constexpr int HV = (16 / static_cast<int>(sizeof(T))) < HALF ? 16 / static_cast<int>(sizeof(T)) : HALF;
+  static constexpr int LPR = HALF / HV;  // lanes per row
+  static_assert(HALF % HV == 0 && LPR >= 1 && LPR <= 32 && (LPR & (LPR - 1)) == 0, "row layout");
+};
+
+// Sum over the LPR lanes of a row (xor shuffles within the row's lane group).
+template <int LPR>
+__device__ __forceinline__ float row_sum(float v) {
+#pragma unroll
+  for (int o = LPR / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, LPR);
+  return v;
+}
+
+// Per-CTA token table of the row kernels: the CTA's kPrologueTok consecutive
+// tokens (b, t), and cos/sin(t * omega_i) for each of them.
+template <int HALF>
+struct TokenTable {
+  float cos_[kPrologueTok][HALF];
+  float sin_[kPrologueTok][HALF];
+  int b[kPrologueTok], t[kPrologueTok];
+  bool valid[kPrologueTok];
+
+  __device__ void fill(long long tok0, long long n_tok, int T, const float* omega) {
+    if (threadIdx.x < kPrologueTok) {
+      const long long tok = tok0 + threadIdx.x;
+      valid[threadIdx.x] = tok < n_tok;
+      const long long tk = tok < n_tok ? tok : 0;
+      b[threadIdx.x] = static_cast<int>(tk / T);
+      t[threadIdx.x] = static_cast<int>(tk % T);
+    }
+    for (int e = threadIdx.x; e < kPrologueTok * HALF; e += blockDim.x) {
+      const int tt = e / HALF, i = e % HALF;
+      const long long tok = tok0 + tt;
+      const int t_ = tok < n_tok ? static_cast<int>(tok % T) : 0;
+      float sn, cs;
+      sincosf(static_cast<float>(t_) * omega[i], &sn, &cs);
+      cos_[tt][i] = cs;
+      sin_[tt][i] = sn;
+    }
+  }
+  // cos and sin of the VEC consecutive pairs starting at pair0 (16-byte loads).
+  template <int VEC>
+  __device__ void load(int tt, int pair0, float (&c)[VEC], float (&s)[VEC]) const {
+    if constexpr (VEC % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < VEC; i += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(&cos_[tt][pair0 + i]);
+        const float4 s4 = *reinterpret_cast<const float4*>(&sin_[tt][pair0 + i]);
+        c[i] = c4.x; c[i + 1] = c4.y; c[i + 2] = c4.z; c[i + 3] = c4.w;
+        s[i] = s4.x; s[i + 1] = s4.y; s[i + 2] = s4.z; s[i + 3] = s4.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        c[i] = cos_[tt][pair0 + i];
+        s[i] = sin_[tt][pair0 + i];
+      }
+    }
+  }
+};
+
+// Division-free walk over the rows (token tt, row kind_row) of a CTA: each
+// lane group advances by a fixed stride per pass.
+struct RowCursor {
+  int tt, kind_row;
+  __device__ void advance(int by, int rows_per_tok) {
+    kind_row += by;
+    while (kind_row >= rows_per_tok) {
+      kind_row -= rows_per_tok;
+      ++tt;
+    }
+  }
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_kernel(const PrologueParams p) {
-  using V = Vec16<T>;
-  constexpr int VEC = V::N;
-  static_assert(D % VEC == 0, "head_dim must be a multiple of the vector width");
-  constexpr int LPR = D / VEC;          // lanes per row
-  static_assert(LPR >= 1 && LPR <= 32 && (LPR & (LPR - 1)) == 0, "lanes per row");
-  constexpr int HALF = D / 2;
+  using RL = RowLayout<T, D>;
+  using HVec = HalfVec<T, RL::HV>;
+  constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
 
-  __shared__ float s_cos[kPrologueTok][HALF];
-  __shared__ float s_sin[kPrologueTok][HALF];
+  __shared__ __align__(16) TokenTable<HALF> tab;
 
   const long long n_tok = static_cast<long long>(p.B) * p.T;
   const long long tok0 = static_cast<long long>(blockIdx.x) * kPrologueTok;
-
-  for (int e = threadIdx.x; e < kPrologueTok * HALF; e += kPrologueThreads) {
-    const int tt = e / HALF, i = e % HALF;
-    const long long tok = tok0 + tt;
-    const int t = tok < n_tok ? static_cast<int>(tok % p.T) : 0;
-    float s, c;
-    sincosf(static_cast<float>(t) * p.omega[i], &s, &c);
-    s_cos[tt][i] = c;
-    s_sin[tt][i] = s;
-  }
+  tab.fill(tok0, n_tok, p.T, p.omega);
   __syncthreads();
 
   const int rows_per_tok = p.H + 2 * p.Hk;
   const int total_rows = kPrologueTok * rows_per_tok;
-  const int sub = threadIdx.x % LPR;        // lane within the row group
-  const int grp = threadIdx.x / LPR;        // row group within the CTA
+  const int sub = threadIdx.x % LPR;  // lane within the row group
+  const int grp = threadIdx.x / LPR;  // row group within the CTA
+  RowCursor cur{0, 0};
+  cur.advance(grp, rows_per_tok);
 
-  // kRowsInFlight rows per lane per pass: all loads of a pass are issued
-  // before any arithmetic, so each lane keeps several 16-byte loads in
-  // flight. Uniform trip count: every lane takes part in every shuffle.
-  constexpr int U = kRowsInFlight;
-  for (int base = 0; base < total_rows; base += ROWS_PER_PASS * U) {
-    float x[U][VEC], e[U][VEC];
-    float gl[U];
-    int kind[U];
-    bool valid[U];
-    size_t row[U], off[U];
+  // Uniform trip count: every lane takes part in every shuffle.
+  for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
+    const bool in_range = base + grp < total_rows;
+    const int tt = in_range ? cur.tt : 0;
+    const int kind_row = in_range ? cur.kind_row : 0;
+    cur.advance(ROWS_PER_PASS, rows_per_tok);
+    const bool valid = in_range && tab.valid[tt];
+    // Row kinds: [0, H) query heads, [H, H+Hk) key heads, then value heads.
+    int kind, head, nheads;
+    if (kind_row < p.H) {
+      kind = 0; head = kind_row; nheads = p.H;
+    } else if (kind_row < p.H + p.Hk) {
+      kind = 1; head = kind_row - p.H; nheads = p.Hk;
+    } else {
+      kind = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
+    }
+    const size_t row = static_cast<size_t>(valid ? tok0 + tt : 0) * nheads + head;
+    const size_t off_lo = row * D + static_cast<size_t>(sub) * HV;
+    const size_t off_hi = off_lo + HALF;
+    const T* src = static_cast<const T*>(kind == 0 ? p.q : (kind == 1 ? p.k : p.v));
+    float xl[HV], xh[HV], el[HV], eh[HV];
+    float gl = 0.f;
+    if (valid) {
+      HVec::load(src + off_lo, xl);
+      HVec::load(src + off_hi, xh);
+    } else {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int r = base + u * ROWS_PER_PASS + grp;
-      const bool in_range = r < total_rows;
-      const int rr = in_range ? r : 0;
-      const int tt = rr / rows_per_tok;
-      const int kind_row = rr % rows_per_tok;
-      const long long tok = tok0 + tt;
-      valid[u] = in_range && tok < n_tok;
-      // Row kinds: [0, H) query heads, [H, H+Hk) key heads, then value heads.
-      int head, nheads;
-      if (kind_row < p.H) {
-        kind[u] = 0; head = kind_row; nheads = p.H;
-      } else if (kind_row < p.H + p.Hk) {
-        kind[u] = 1; head = kind_row - p.H; nheads = p.Hk;
-      } else {
-        kind[u] = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
-      }
-      row[u] = static_cast<size_t>(valid[u] ? tok : 0) * nheads + head;
-      off[u] = row[u] * D + static_cast<size_t>(sub) * VEC;
-      const void* src = kind[u] == 0 ? p.q : (kind[u] == 1 ? p.k : p.v);
-      if (valid[u]) {
-        V::load(static_cast<const T*>(src) + off[u], x[u]);
-      } else {
+      for (int i = 0; i < HV; ++i) xl[i] = xh[i] = 0.f;
+    }
+    const bool has_e = valid && kind == 2 && p.has_ve;
+    if (has_e) {
+      HVec::load(static_cast<const T*>(p.ve) + off_lo, el);
+      HVec::load(static_cast<const T*>(p.ve) + off_hi, eh);
+      gl = Vec16<T>::scalar(p.gate, row);
+    } else {
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) x[u][i] = 0.f;
-      }
-      gl[u] = 0.f;
-      if (valid[u] && kind[u] == 2 && p.has_ve) {
-        V::load(static_cast<const T*>(p.ve) + off[u], e[u]);
-        gl[u] = V::scalar(p.gate, row[u]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) e[u][i] = 0.f;
-      }
+      for (int i = 0; i < HV; ++i) el[i] = eh[i] = 0.f;
     }
 
+    // RMSNorm: mean of squares over the row (shuffle reduction over its lanes).
+    float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int r = base + u * ROWS_PER_PASS + grp;
-      const int tt = (r < total_rows ? r : 0) / rows_per_tok;
-      // RMSNorm: mean of squares over the row's LPR lanes (shuffle reduction).
-      float ss = 0.f;
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) ss = fmaf(x[u][i], x[u][i], ss);
-#pragma unroll
-      for (int o = LPR / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o, LPR);
-      const float rstd = rsqrtf(ss / static_cast<float>(D) + p.eps);
-      float n[VEC];
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) n[i] = x[u][i] * rstd;
+    for (int i = 0; i < HV; ++i) ss = fmaf(xl[i], xl[i], fmaf(xh[i], xh[i], ss));
+    ss = row_sum<LPR>(ss);
+    const float rstd = rsqrtf(ss / static_cast<float>(D) + p.eps);
+    if (!valid) continue;
 
-      // RoPE on half-split pairs (i, i + D/2).
-      float y[VEC];
-      if constexpr (LPR >= 2) {
-        float partner[VEC];
+    if (kind == 2) {
+      // Value residual: v + 3 sigmoid(gate) ve.
+      const float coef = has_e ? 3.0f / (1.0f + expf(-gl)) : 0.f;
 #pragma unroll
-        for (int i = 0; i < VEC; ++i)
-          partner[i] = __shfl_xor_sync(0xffffffffu, n[i], LPR / 2, LPR);
-        const bool lower = sub < LPR / 2;
-        const int pair0 = (lower ? sub : sub - LPR / 2) * VEC;
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-          const float c = s_cos[tt][pair0 + i], s = s_sin[tt][pair0 + i];
-          // lower half: x_i c - x_{i+D/2} s ; upper half: x_{i-D/2} s + x_i c
-          y[i] = lower ? fmaf(n[i], c, -partner[i] * s) : fmaf(partner[i], s, n[i] * c);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const float c = s_cos[tt][i], s = s_sin[tt][i];
-          y[i] = fmaf(n[i], c, -n[i + HALF] * s);
-          y[i + HALF] = fmaf(n[i], s, n[i + HALF] * c);
-        }
+      for (int i = 0; i < HV; ++i) {
+        xl[i] = fmaf(coef, el[i], xl[i]);
+        xh[i] = fmaf(coef, eh[i], xh[i]);
       }
-      if (!valid[u]) continue;
-
-      if (kind[u] == 2) {
-        // Value residual: v + 3 sigmoid(gate) ve (e = 0 without ve).
-        const float coef = p.has_ve ? 3.0f / (1.0f + expf(-gl[u])) : 0.f;
-        float vv[VEC];
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) vv[i] = fmaf(coef, e[u][i], x[u][i]);
-        V::store(static_cast<T*>(p.v_out) + off[u], vv);
-      } else {
-        V::store(static_cast<T*>(kind[u] == 0 ? p.q_out : p.k_out) + off[u], y);
-        if (sub == 0) (kind[u] == 0 ? p.rstd_q : p.rstd_k)[row[u]] = rstd;
-      }
+      HVec::store(static_cast<T*>(p.v_out) + off_lo, xl);
+      HVec::store(static_cast<T*>(p.v_out) + off_hi, xh);
+      continue;
     }
+    // RoPE on the pairs (i, i + D/2) held by this lane.
+    float cv[HV], sv[HV], yl[HV], yh[HV];
+    tab.template load<HV>(tt, sub * HV, cv, sv);
+#pragma unroll
+    for (int i = 0; i < HV; ++i) {
+      const float nl = xl[i] * rstd, nh = xh[i] * rstd;
+      yl[i] = fmaf(nl, cv[i], -nh * sv[i]);
+      yh[i] = fmaf(nl, sv[i], nh * cv[i]);
+    }
+    T* dst = static_cast<T*>(kind == 0 ? p.q_out : p.k_out);
+    HVec::store(dst + off_lo, yl);
+    HVec::store(dst + off_hi, yh);
+    if (sub == 0) (kind == 0 ? p.rstd_q : p.rstd_k)[row] = rstd;
   }
 }
 
