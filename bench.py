@@ -101,6 +101,20 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def rank_config_id(rank: int) -> int:
+    """Seed component of a rank's batch: every rank draws its own inputs."""
+    return CONFIG_ID + 1000 * rank
+
+
+def reduce_max(values, dist, device):
+    """Max over ranks of a list of floats (identity on one process)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
 def visible_gpu_indices(n_local):
     cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
     if cvd:
@@ -146,7 +160,7 @@ def run_ours(args):
              for W, ve in zip(w.windows, w.ve)]
     # Per-rank shard: its own batch, seeded by rank (config id offset).
     host = [synth.layer_inputs(w.B, w.T, w.H, w.Hk, w.D, ve, torch.bfloat16,
-                               config=CONFIG_ID + 1000 * rank, layer=i, dO_std=w.dO_std)
+                               config=rank_config_id(rank), layer=i, dO_std=w.dO_std)
             for i, ve in enumerate(w.ve)]
     names = ("q", "k", "v", "ve", "gate", "dO")
     pinned = [{k: (v.pin_memory() if v is not None else None) for k, v in h.items()} for h in host]
@@ -226,10 +240,7 @@ def run_ours(args):
         e2e_ms = float("nan")
     cs.cswattn_sync_status()
 
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
     e2e_value = flops_step * world / (e2e_ms / e2e_steps * 1e-3) / 1e12

@@ -27,7 +27,8 @@ F32, BF16 = 0, 1
 # Every symbol the header declares; the CPU tests check the library exports them.
 EXPORTS = ("attn_prologue", "attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
            "cswattn_sync_status", "cswattn_set_wait_limit_ns", "cswattn_set_timing",
-           "cswattn_kernel_times", "cswattn_last_error", "cswattn_version")
+           "cswattn_kernel_times", "cswattn_selftest_wait_timeout", "cswattn_last_error",
+           "cswattn_version")
 KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi")
 
 
@@ -73,6 +74,8 @@ def lib():
         L.cswattn_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_double),
                                            ctypes.POINTER(ctypes.c_int)]
         L.cswattn_kernel_times.restype = ctypes.c_int
+        L.cswattn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        L.cswattn_selftest_wait_timeout.restype = ctypes.c_int
         L.attn_bwd_noalloc.argtypes = [lp] + [vp] * 7 + [fp, fp, vp, fp, vp] + [vp] * 5 + [vp]
         for name in ("attn_prologue", "attn_fwd", "attn_bwd", "attn_bwd_noalloc",
                      "cswattn_sync_status"):
@@ -192,6 +195,11 @@ def cswattn_kernel_times():
     cnt = (ctypes.c_int * n)()
     _check(lib().cswattn_kernel_times(ms, cnt))
     return {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def cswattn_selftest_wait_timeout(limit_ns: int, stream=None):
+    """Launch the bounded-wait self-test kernel (its wait always runs out)."""
+    _check(lib().cswattn_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def cswattn_version() -> int:

@@ -91,7 +91,9 @@ struct EpiParams {
   const void *q, *k, *ve, *gate;        // prologue inputs (layer dtype)
   const float *rstd_q, *rstd_k;
   const float* dq_acc;                  // (B,H,T,D) dq~ (scaled)
-  const float *dk_acc, *dv_acc;         // (B,T,Hk,D) dk~ (scaled), dv_eff
+  const float *dk_acc, *dv_acc;         // [parts] x (B,T,Hk,D) partial dk~ (scaled), dv_eff
+  int parts;                            // number of partial slots to sum
+  long long kv_stride;                  // elements between partial slots
   void *dq, *dk, *dv, *dve, *dgate;     // outputs (layer dtype)
 };
 
@@ -173,6 +175,19 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
       }
       load_f32<HV>(src + so, dl);
       load_f32<HV>(src + so + HALF, dh);
+      if (kind != 0) {
+        // dK / dV arrive as partial sums from the backward's parts.
+        for (int pi = 1; pi < p.parts; ++pi) {
+          float el[HV], eh[HV];
+          load_f32<HV>(src + pi * p.kv_stride + so, el);
+          load_f32<HV>(src + pi * p.kv_stride + so + HALF, eh);
+#pragma unroll
+          for (int i = 0; i < HV; ++i) {
+            dl[i] += el[i];
+            dh[i] += eh[i];
+          }
+        }
+      }
       if (kind != 2) {
         HVec::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off_lo, xl);
         HVec::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off_hi, xh);

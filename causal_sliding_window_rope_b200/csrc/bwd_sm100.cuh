@@ -16,16 +16,21 @@
 //   S^T  = K Q^T      (M=128 keys, N=64 queries, K=128 d)   SS MMA
 //   dP^T = V dO^T     (same shape)                         SS MMA
 //   softmax warps: P^T = exp2(c2 S^T - lse2), dS^T = P^T (dP^T - Delta),
-//                  both as bf16 into shared memory (128B-swizzled, K-major)
-//   dV  += P^T dO     (M=128 keys, N=128 d, K=64)           SS MMA
-//   dK  += dS^T Q     (same shape)                         SS MMA
-//   dQ^T = K^T dS^T   (M=128 d, N=64 queries, K=128 keys)   SS MMA, into
-//          the S^T columns of the step, drained by the dQ warps into a
-//          float32 tile that a bulk reduce-add sends to the dq accumulator.
+//                  both as bf16 into TMEM (the step's dQ^T columns), and
+//                  dS^T also into shared memory (128B-swizzled)
+//   dV  += P^T dO     (M=128 keys, N=128 d, K=64)           TS MMA (P^T in TMEM)
+//   dK  += dS^T Q     (same shape)                         TS MMA (dS^T in TMEM)
+//   dQ^T = K^T dS^T   (M=128 d, N=64 queries, K=128 keys)   SS MMA, over the
+//          P^T/dS^T columns (issued after the two TS MMAs that read them),
+//          drained by the dQ warps straight from TMEM with float32
+//          reductions into the dq accumulator (one 128-byte request per warp
+//          and query).
+// Shared memory holds only the MMA operands (K, V, the Q/dO ring, dS^T), so
+// the SS products, which are bound by shared-memory bandwidth, get most of it.
 // TMEM (512 columns): SP (S^T at +0, dP^T at +64) | dQ^T x2 (64 columns
-// each) | dV | dK. The softmax warps release SP as soon as they have loaded
-// it into registers, so the next step's S^T/dP^T run while they compute; the
-// dQ^T double buffer lets the drain of one step overlap the next step.
+// each; also P^T at +0 and dS^T at +32 before the dQ^T product) | dV | dK.
+// The softmax warps release SP as soon as they have loaded it into
+// registers, so the next step's S^T/dP^T run while they compute.
 // Roles: warp 0 TMA, warp 1 MMA issuer + TMEM owner, warps 4-7 softmax
 // (thread = key row), warps 8-11 dQ drain (thread = head_dim row of dQ^T).
 #pragma once
@@ -43,17 +48,14 @@ constexpr int kKVPanel = kKVBytes / 2;   // 16 KB: 128 rows x 128 B
 constexpr int kQBytes = kBQ * kD * 2;    // 16 KB
 constexpr int kQPanel = kQBytes / 2;     // 8 KB: 64 rows x 128 B
 constexpr int kPBytes = kBN * kBQ * 2;   // 16 KB: 128 rows x 128 B
-constexpr int kDQBytes = kBQ * kD * 4;   // 32 KB float32 staging
 
 constexpr int kQStages = 3;             // Q/dO ring depth
 constexpr int kStageBytes = 2 * kQBytes;  // Q then dO
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKVBytes;
 constexpr int kOffQD = kOffV + kKVBytes;                 // [kQStages] x (Q | dO)
-constexpr int kOffP = kOffQD + kQStages * kStageBytes;   // P^T (single buffer)
-constexpr int kOffDS = kOffP + kPBytes;                  // dS^T (single buffer)
-constexpr int kOffDQ = kOffDS + kPBytes;
-constexpr int kOffBar = kOffDQ + kDQBytes;
+constexpr int kOffDS = kOffQD + kQStages * kStageBytes;  // dS^T [2]
+constexpr int kOffBar = kOffDS + 2 * kPBytes;
 constexpr int kOffRow = kOffBar + 256;         // per Q stage: lse2[64], delta[64]
 constexpr int kSmemBytes = kOffRow + kQStages * 2 * kBQ * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -72,13 +74,15 @@ constexpr uint32_t kColDK = 384u;
 
 struct Params {
   int B, T, H, Hk, W, g, nkv, Tpad;
+  int parts;               // CTAs per KV tile (each takes a share of its steps)
+  long long kv_stride;     // elements between the parts' dK/dV partial slots
   float scale_log2;  // c * log2(e)
   float scale;       // c
   const float* lse2;   // (B,H,Tpad) lse * log2(e), +inf past T
   const float* delta;  // (B,H,Tpad) dO.O, 0 past T
   float* dq_acc;       // (B,H,T,D), accumulated (must start at zero)
-  float* dk_acc;       // (B,T,Hk,D)
-  float* dv_acc;       // (B,T,Hk,D)
+  float* dk_acc;       // [parts] x (B,T,Hk,D) partial sums
+  float* dv_acc;       // [parts] x (B,T,Hk,D) partial sums
   unsigned long long wait_ns;
 };
 
@@ -108,24 +112,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_empty = bars + 4;     // [kQStages]
   uint64_t* sp_full = bars + 7;     // S^T/dP^T in TMEM
   uint64_t* sp_free = bars + 8;     // softmax has loaded S^T/dP^T
-  uint64_t* p_full = bars + 9;      // P^T/dS^T written to shared memory
-  uint64_t* ps_empty = bars + 10;   // MMAs done reading P^T/dS^T
-  uint64_t* dq_full = bars + 11;    // [2]
-  uint64_t* dq_empty = bars + 13;   // [2]
-  uint64_t* acc_full = bars + 15;
-  uint64_t* mma_done = bars + 16;
-  uint64_t* stage_free = bars + 17;  // dQ staging tile may be overwritten
-  uint64_t* stage_full = bars + 18;  // dQ staging tile written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
+  uint64_t* p_full = bars + 9;      // P^T/dS^T written (TMEM and shared memory)
+  uint64_t* ps_empty = bars + 10;   // [2] dQ^T product done reading dS^T buffer
+  uint64_t* dq_full = bars + 12;    // [2]
+  uint64_t* dq_empty = bars + 14;   // [2]
+  uint64_t* acc_full = bars + 16;
+  uint64_t* mma_done = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
   float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [kQStages][64]
   float* s_delta = s_lse2 + kQStages * kBQ;                         // [kQStages][64]
 
   const int warp = warp_id(), lane = lane_id();
 
-  // ---- work unit: KV block j (ascending = most queries first), (b, hk)
+  // ---- work unit: KV block j (ascending = most queries first), part of
+  // its steps, (b, hk). Heavy KV tiles are split into `parts` CTAs so that
+  // the grid balances across SMs; each part writes its own dK/dV partials.
   const int BHk = p.B * p.Hk;
-  const int j = static_cast<int>(blockIdx.x) / BHk;
+  const int unit = static_cast<int>(blockIdx.x) / BHk;
+  const int j = unit / p.parts, part = unit % p.parts;
   const int bh = static_cast<int>(blockIdx.x) % BHk;
   const int b = bh / p.Hk, hk = bh % p.Hk;
   const int k0 = j * kBN;
@@ -134,7 +139,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qs_lo = k0 / kBQ;
   const int qs_hi = static_cast<int>(q_last_ll) / kBQ;
   const int nsph = qs_hi - qs_lo + 1;  // steps per head
-  const int N = p.g * nsph;
+  const int n_all = p.g * nsph;
+  const int n_begin = static_cast<int>(static_cast<long long>(part) * n_all / p.parts);
+  const int N = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.parts) - n_begin;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -145,15 +152,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(sp_full, 1);
     mbar_init(sp_free, 128);
     mbar_init(p_full, 128);
-    mbar_init(ps_empty, 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&ps_empty[s], 1);
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_empty[s], 128);
     }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
-    mbar_init(stage_free, 1);
-    mbar_init(stage_full, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __device__ int q0() const { return qs * kBQ; }
   };
-  const Cursor cur0{hk * p.g, qs_lo, hk * p.g + p.g, qs_lo, qs_hi};
+  const Cursor cur0{hk * p.g + n_begin / nsph, qs_lo + n_begin % nsph, hk * p.g + p.g, qs_lo, qs_hi};
 
   if (warp < 4) {
     regs_dec<kRegLo>();
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T
       const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV);
       const uint32_t sQ = smem_u32(smem + kOffQD), sDO = sQ + kQBytes;
-      const uint32_t sP = smem_u32(smem + kOffP), sDS = smem_u32(smem + kOffDS);
+      const uint32_t sDS = smem_u32(smem + kOffDS);
       bool ok = mbar_wait(kv_full, 0, wc);
       tc_fence_after();
 
@@ -243,8 +248,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dO_k = sdesc_sw128(sDO, 16, 1024);        // dO, K-major
       const uint64_t dQ_m = sdesc_sw128(sQ, kQPanel, 1024);    // Q, MN-major
       const uint64_t dO_m = sdesc_sw128(sDO, kQPanel, 1024);   // dO, MN-major
-      const uint64_t dP_k = sdesc_sw128(sP, 16, 1024);         // P^T, K-major
-      const uint64_t dS_k = sdesc_sw128(sDS, 16, 1024);        // dS^T, K-major
       const uint64_t dS_m = sdesc_sw128(sDS, kPBytes, 1024);   // dS^T, MN-major
       const uint64_t dK_m = sdesc_sw128(sK, kKVPanel, 1024);   // K^T, MN-major
       auto ofs = [](int bytes) { return static_cast<uint64_t>(bytes >> 4); };
@@ -271,32 +274,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
-      if (ok) ok = issue_SdP(0);
+      if (ok && N > 0) ok = issue_SdP(0);
       for (int n = 0; ok && n < N; ++n) {
         const int st = n % kQStages;
         const int db = n & 1, duse = n >> 1;  // dQ^T TMEM buffer
         // The next step's S^T/dP^T as soon as the softmax has loaded this one.
         if (n + 1 < N && !issue_SdP(n + 1)) break;
+        // The softmax has written P^T/dS^T into dQ^T buffer db (after that
+        // buffer was drained) and dS^T into shared buffer db.
         if (!mbar_wait(p_full, n & 1, wc)) break;
         tc_fence_after();
         const uint64_t qb = ofs(st * kStageBytes);
+        const uint32_t ptm = tmem + col_dq(db);  // P^T at +0, dS^T at +32
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dV += P^T dO
-          mma_ss(tmem + kColDV, dP_k + ofs(kk * 32), dO_m + qb + ofs(kk * 2048), idKV,
+          mma_ts(tmem + kColDV, ptm + kk * 8, dO_m + qb + ofs(kk * 2048), idKV,
                  (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-          mma_ss(tmem + kColDK, dS_k + ofs(kk * 32), dQ_m + qb + ofs(kk * 2048), idKV,
+          mma_ts(tmem + kColDK, ptm + 32 + kk * 8, dQ_m + qb + ofs(kk * 2048), idKV,
                  (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
-        if (duse > 0 && !mbar_wait(&dq_empty[db], (duse - 1) & 1, wc)) break;
-        tc_fence_after();
+        const uint64_t sb = ofs(db * kPBytes);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T
-          mma_ss(tmem + col_dq(db), dK_m + ofs(kk * 2048), dS_m + ofs(kk * 2048), idDQ,
-                 kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)  // dQ^T = K^T dS^T (over P^T/dS^T, read above)
+          mma_ss(ptm, dK_m + ofs(kk * 2048), dS_m + sb + ofs(kk * 2048), idDQ, kk > 0 ? 1u : 0u);
         mma_commit(&dq_full[db]);
-        mma_commit(ps_empty);
+        mma_commit(&ps_empty[db]);
+        (void)duse;
       }
       mma_commit(acc_full);
       mma_commit(mma_done);
@@ -358,22 +363,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           dd[c * 16 + i / 2] = pack_bf16x2(dsv[0], dsv[1]);
           dd[c * 16 + i / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-      got = n == 0 || mbar_wait(ps_empty, (n - 1) & 1, wc);
+      // Buffer db (TMEM dQ^T columns and shared dS^T) was last used by step
+      // n-2: wait until that step's dQ^T has been drained and its dQ^T
+      // product has read the shared dS^T.
+      const int db = n & 1, duse = n >> 1;
+      got = duse == 0 || (mbar_wait(&dq_empty[db], (duse - 1) & 1, wc) &&
+                          mbar_wait(&ps_empty[db], (duse - 1) & 1, wc));
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
-      // Row r of P^T / dS^T: 64 bf16 = 8 chunks of 16 B, 128B-swizzled.
-      uint8_t* prow = smem + kOffP + (r >> 3) * 1024 + (r & 7) * 128;
-      uint8_t* drow = smem + kOffDS + (r >> 3) * 1024 + (r & 7) * 128;
+      tc_fence_after();
+      // P^T and dS^T rows into TMEM (A operands of the dV / dK products).
+      tmem_st32(tmem + lane_off + col_dq(db), pp);
+      tmem_st32(tmem + lane_off + col_dq(db) + 32, dd);
+      // Row r of dS^T into shared memory: 64 bf16 = 8 chunks of 16 B, 128B-swizzled.
+      uint8_t* drow = smem + kOffDS + db * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         const int pos = (ch ^ (r & 7)) << 4;
-        *reinterpret_cast<uint4*>(prow + pos) =
-            make_uint4(pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
         *reinterpret_cast<uint4*>(drow + pos) =
             make_uint4(dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -383,7 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__all_sync(0xffffffffu, acc_ok)) {
       tc_fence_after();
       const bool row_ok = kj < p.T;
-      const size_t off = ((static_cast<size_t>(b) * p.T + (row_ok ? kj : 0)) * p.Hk + hk) * kD;
+      const float keep = N > 0 ? 1.f : 0.f;  // a part without steps writes zeros
+      const size_t off = static_cast<size_t>(part) * p.kv_stride +
+                         ((static_cast<size_t>(b) * p.T + (row_ok ? kj : 0)) * p.Hk + hk) * kD;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t a[32];
@@ -393,14 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           float4* dst = reinterpret_cast<float4*>(p.dv_acc + off + c * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 8; ++v4)
-            dst[v4] = make_float4(__uint_as_float(a[4 * v4]), __uint_as_float(a[4 * v4 + 1]),
-                                  __uint_as_float(a[4 * v4 + 2]), __uint_as_float(a[4 * v4 + 3]));
+            dst[v4] = make_float4(__uint_as_float(a[4 * v4]) * keep, __uint_as_float(a[4 * v4 + 1]) * keep,
+                                  __uint_as_float(a[4 * v4 + 2]) * keep, __uint_as_float(a[4 * v4 + 3]) * keep);
         }
         tmem_ld32(tmem + lane_off + kColDK + c * 32, a);
         tmem_ld_wait();
         if (row_ok) {
           float4* dst = reinterpret_cast<float4*>(p.dk_acc + off + c * 32);
-          const float sc = p.scale;
+          const float sc = p.scale * keep;
 #pragma unroll
           for (int v4 = 0; v4 < 8; ++v4)
             dst[v4] = make_float4(__uint_as_float(a[4 * v4]) * sc, __uint_as_float(a[4 * v4 + 1]) * sc,
@@ -416,8 +430,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------- dQ drain
     const int d = (warp & 3) * 32 + lane;  // TMEM lane = head_dim index of dQ^T
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const bool leader = (warp == 8 && lane == 0);
-    float* sdq = reinterpret_cast<float*>(smem + kOffDQ);
     const float sc = p.scale;
     Cursor c = cur0;
     for (int n = 0; n < N; ++n, c.next()) {
@@ -432,27 +444,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&dq_empty[st]);
-      if (leader) {
-        bulk_wait_read0();  // the previous reduction has read the staging tile
-        mbar_arrive(stage_free);
-      }
-      got = mbar_wait(stage_free, n & 1, wc);
-      if (!__all_sync(0xffffffffu, got)) break;
+      // Column q of dQ^T -> dq_acc[b][h][q0 + q][d]; the warp's 32 lanes hit
+      // 32 consecutive floats (one 128-byte reduction request per query).
+      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.T + q0) * kD + d;
+      const int nrows = min(kBQ, p.T - q0);
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sdq[(c * 32 + i) * kD + d] = __uint_as_float(a[c][i]) * sc;
-      fence_proxy_async_smem();
-      mbar_arrive(stage_full);
-      if (leader) {
-        if (!mbar_wait(stage_full, n & 1, wc)) break;
-        const int nrows = min(kBQ, p.T - q0);
-        float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.T + q0) * kD;
-        bulk_reduce_add_f32(dst, sdq, static_cast<uint32_t>(nrows) * kD * 4);
-        bulk_commit();
-      }
+        for (int i = 0; i < 32; ++i)
+          if (cc * 32 + i < nrows) red_add_f32(dst + (cc * 32 + i) * kD, __uint_as_float(a[cc][i]) * sc);
     }
-    if (leader) bulk_wait0();
   }
 
   tc_fence_before();

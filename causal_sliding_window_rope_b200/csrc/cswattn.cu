@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 #include <string>
@@ -244,6 +245,22 @@ void launch_simt_bwd(const Shape& s, const SimtParams& sp, cudaStream_t st) {
   }
 }
 
+// ---------------------------------------------------------------- self-test
+
+// One thread waits, with the kernels' bounded wait, on a barrier nothing
+// arrives on; the wait runs out and records the timeout status.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    const WaitCtx wc{&abort_flag, limit_ns};
+    (void)mbar_wait(&bar, 0, wc);
+  }
+}
+
 // ---------------------------------------------------------------- timing
 
 std::atomic<int> g_timing{0};
@@ -294,9 +311,27 @@ struct Workspace {
 
 int padded_T(int T) { return (T + 63) / 64 * 64; }
 
+// CTAs per KV tile in the tensor-core backward: heavy tiles (many query
+// steps) are split so that the largest CTA holds at most about half the
+// average work of an SM (148 SMs). 1 for the fp32 path.
+int bwd_parts(const Shape& s) {
+  if (!s.bf16) return 1;
+  const int nkv = (s.T + 127) / 128;
+  long long total = 0, nmax = 0;
+  for (int j = 0; j < nkv; ++j) {
+    const long long last = std::min<long long>(s.T - 1, static_cast<long long>(j) * 128 + 127 + s.W - 1);
+    const long long n = static_cast<long long>(s.g) * (last / 64 - 2 * j + 1);
+    total += n;
+    nmax = std::max(nmax, n);
+  }
+  total *= static_cast<long long>(s.B) * s.Hk;
+  const long long want = (2 * nmax * 148 + total - 1) / std::max(total, 1ll);
+  return static_cast<int>(std::min<long long>(8, std::max<long long>(1, want)));
+}
+
 Workspace carve(const Shape& s, void* base) {
   const size_t nq = static_cast<size_t>(s.B) * s.H * s.T * s.D;
-  const size_t nk = static_cast<size_t>(s.B) * s.T * s.Hk * s.D;
+  const size_t nk = static_cast<size_t>(s.B) * s.T * s.Hk * s.D * bwd_parts(s);
   const size_t nr = static_cast<size_t>(s.B) * s.H * padded_T(s.T);
   Workspace w;
   uint8_t* p = static_cast<uint8_t*>(base);
@@ -355,6 +390,13 @@ int cswattn_version(void) { return (1 << 16) | 0; }
 const char* cswattn_last_error(void) { return t_err.c_str(); }
 
 void cswattn_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns < 1000 ? 1000 : ns); }
+
+cswattn_status cswattn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000) limit_ns = 1000;
+  if (limit_ns > 1000000000ull) limit_ns = 1000000000ull;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return launched("self-test launch");
+}
 
 void cswattn_set_timing(int enable) { g_timing.store(enable ? 1 : 0); }
 
@@ -616,8 +658,10 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     bp.dq_acc = w.dq_acc;
     bp.dk_acc = w.dk_acc;
     bp.dv_acc = w.dv_acc;
+    bp.parts = bwd_parts(s);
+    bp.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
     bp.wait_ns = g_wait_ns.load();
-    const unsigned grid = static_cast<unsigned>(bp.nkv) * s.B * s.Hk;
+    const unsigned grid = static_cast<unsigned>(bp.nkv) * bp.parts * s.B * s.Hk;
     {
       ScopedTiming tm(CSWATTN_K_BWD, cs);
       bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, bp);
@@ -641,6 +685,8 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   ep.dq_acc = w.dq_acc;
   ep.dk_acc = w.dk_acc;
   ep.dv_acc = w.dv_acc;
+  ep.parts = bwd_parts(s);
+  ep.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
   ep.dq = dQ;
   ep.dk = dK;
   ep.dv = dV;

@@ -96,8 +96,10 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
                         const void* v_out, void* O, float* lse, void* stream);
 
 /* Bytes of device scratch attn_bwd needs for this layer: float32
- * accumulators of dq_out (B, n_head, T, head_dim), dk_out and dv_out
- * (B, T, n_kv_head, head_dim), and two row terms (dO.O and lse*log2(e)),
+ * accumulators of dq_out (B, n_head, T, head_dim), P partial sums each of
+ * dk_out and dv_out (B, T, n_kv_head, head_dim) (P = 1..8, the number of
+ * CTAs the bf16 backward splits a key tile's work into; 1 for f32), and two
+ * row terms (dO.O and lse*log2(e)),
  * each (B, n_head, Tpad) with Tpad = T rounded up to a multiple of 64;
  * every part padded to 256 bytes. Returns 0 for an invalid layer. */
 size_t attn_bwd_workspace_bytes(const cswattn_layer* layer);
@@ -159,6 +161,14 @@ cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const
  * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last check, CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
 cswattn_status cswattn_sync_status(void* stream);
+
+/* Self-test of the bounded-wait path: launches one small kernel whose thread
+ * waits on a barrier that nothing ever arrives on, using the same bounded
+ * wait as the attention kernels, with a limit of `limit_ns` (clamped to
+ * [1000, 1e9]). The wait runs out, the kernel records CSWATTN_ERR_TIMEOUT in
+ * the device status word and returns; a following cswattn_sync_status()
+ * reports (and clears) it. Touches no TMEM and issues no copies. */
+cswattn_status cswattn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* Upper bound, in nanoseconds, of every device-side wait of later launches
  * (default 2e9). Values below 1000 are raised to 1000. Process-wide. */

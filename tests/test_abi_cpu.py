@@ -101,7 +101,11 @@ def test_workspace_size_and_check(lib):
     pad = lambda x: (x + 255) // 256 * 256  # noqa: E731
     B, T, H, Hk, D = 2, 100, 6, 2, 128
     Tpad = (T + 63) // 64 * 64
-    assert n == pad(4 * B * H * T * D) + 2 * pad(4 * B * T * Hk * D) + 2 * pad(4 * B * H * Tpad)
+    # dq accumulator, P partial-sum slots each for dk and dv (1 <= P <= 8), two row terms
+    fixed = pad(4 * B * H * T * D) + 2 * pad(4 * B * H * Tpad)
+    assert any(n == fixed + 2 * pad(P * 4 * B * T * Hk * D) for P in range(1, 9))
+    f32 = cs.LayerSpec(2, 100, 6, 2, 128, 32, dtype="f32")
+    assert cs.attn_bwd_workspace_bytes(f32) == fixed + 2 * pad(4 * B * T * Hk * D)  # P = 1
     layer = ctypes.byref(spec.c())
     ptrs = [256 * (i + 1) for i in range(17)]
     st = lib.attn_bwd(layer, *ptrs[:12], *ptrs[12:17], 256 * 40, n - 1, None)
