@@ -47,58 +47,63 @@ def workload_desc(w):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled during the timed
+    region: NVML polled from a thread every ~2 ms (read-only queries). The
+    record is None when NVML is unavailable."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, indices):
-        self.indices = set(indices)
-        self.proc = None
+        self.indices = list(indices) or [0]
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = 0.0
+        self._stop = None
+        self._thread = None
+        self._nvml = None
 
     def start(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            handles = [pynvml.nvmlDeviceGetHandleByIndex(i) for i in self.indices]
+            self.max_mhz = max(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM) for h in handles)
+        except Exception:
+            self._nvml = None
+            return
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                for h in handles:
+                    try:
+                        self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                        mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        for name, const in self.REASONS:
+                            if mask & getattr(pynvml, const):
+                                self.reasons.add(name)
+                    except Exception:
+                        pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is None:
             return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in out.splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                idx = int(parts[0])
-            except ValueError:
-                continue
-            if self.indices and idx not in self.indices:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
+        self._stop.set()
+        self._thread.join(timeout=5)
+        if not self.samples:
             return None
-        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples), "source": "nvml, every ~2 ms during the timed region",
+                "reasons": sorted(self.reasons)}
 
 
 def rank_config_id(rank: int) -> int:
@@ -220,7 +225,6 @@ def run_ours(args):
     clocks = ClockSampler(visible_gpu_indices(world if world > 1 else 1) if rank == 0 else [])
     if rank == 0:
         clocks.start()
-        time.sleep(0.3)
     cs.cswattn_set_timing(True)
     cs.cswattn_kernel_times()
     total_ms = timed(step, args.steps, flush=True)
@@ -363,18 +367,23 @@ def time_oracle_sample(w, n_layers=None):
 
 
 def cpu_baseline(w, budget_s=20.0):
+    """The oracle on a bounded sample, repeated until about half the budget
+    (10-30 s of CPU work by default) has been spent."""
     import oracle
     oracle.build()
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     flops, dt, n = time_oracle_sample(w, n_layers=1)
+    reps = 1
     if dt < budget_s / 4:
-        f2, d2, n2 = time_oracle_sample(w, n_layers=None)
-        flops, dt, n = f2, d2, n2
+        flops, dt, reps = 0.0, 0.0, 0
+        while dt < budget_s / 2 and reps < 8:
+            f2, d2, n = time_oracle_sample(w, n_layers=None)
+            flops, dt, reps = flops + f2, dt + d2, reps + 1
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"float64 C oracle (prologue+fwd+bwd+chain rule), batch 1, one KV head "
                       f"with its {w.H // w.Hk} query heads, T={w.T}, first {n} of the layer windows "
-                      f"{w.windows}; FLOPs counted as 12*D per unmasked pair"}
+                      f"{w.windows}, {reps} repetition(s); FLOPs counted as 12*D per unmasked pair"}
 
 
 def run_reference(args):
