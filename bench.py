@@ -185,15 +185,47 @@ def run_ours(args):
     h2d = sum(v.numel() * v.element_size() for p in pinned for v in p.values() if v is not None)
     d2h = sum(v.numel() * v.element_size() for o in host_out for v in o.values())
 
+    # e2e step: host->device copies on one stream, kernels on the main one,
+    # device->host copies on a third, chained per layer by events, so that
+    # the two copy directions (PCIe is full duplex) and the kernels overlap.
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    fwd_names, grad_names = ("q", "k", "v", "ve", "gate"), ("dQ", "dK", "dV", "dve", "dgate")
+
     def step_e2e():
-        for x, p in zip(inp, pinned):
-            for n in names:
-                if p[n] is not None:
-                    x[n].copy_(p[n], non_blocking=True)
-        step()
-        for b, o in zip(bufs, host_out):
-            for n, t in o.items():
-                t.copy_(getattr(b, n), non_blocking=True)
+        begin = torch.cuda.Event()
+        begin.record(stream)
+        s_in.wait_event(begin)
+        s_out.wait_event(begin)
+        for s, x, p, b, o in zip(specs, inp, pinned, bufs, host_out):
+            with torch.cuda.stream(s_in):
+                for n in fwd_names:
+                    if p[n] is not None:
+                        x[n].copy_(p[n], non_blocking=True)
+                got_fwd = torch.cuda.Event()
+                got_fwd.record(s_in)
+                x["dO"].copy_(p["dO"], non_blocking=True)
+                got_dO = torch.cuda.Event()
+                got_dO.record(s_in)
+            stream.wait_event(got_fwd)
+            cs.layer_forward(s, b, x["q"], x["k"], x["v"], x["ve"], x["gate"], stream=stream)
+            fwd_done = torch.cuda.Event()
+            fwd_done.record(stream)
+            stream.wait_event(got_dO)
+            cs.layer_backward(s, b, x["q"], x["k"], x["ve"], x["gate"], x["dO"], stream=stream)
+            bwd_done = torch.cuda.Event()
+            bwd_done.record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(fwd_done)
+                o["O"].copy_(b.O, non_blocking=True)
+                s_out.wait_event(bwd_done)
+                for n in grad_names:
+                    if n in o:
+                        o[n].copy_(getattr(b, n), non_blocking=True)
+        # the next step overwrites these buffers: join both copy streams
+        for side in (s_in, s_out):
+            e = torch.cuda.Event()
+            e.record(side)
+            stream.wait_event(e)
 
     flops_layer = [12.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
     flops_fwd = [4.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]

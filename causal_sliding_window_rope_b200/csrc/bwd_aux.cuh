@@ -6,8 +6,10 @@
 //   "1. GPT 모델": RoPE, QK normalisation, value-embedding code):
 //   dq = RMSNorm'(RoPE^-1(dq~)), dk likewise, dv = dv_eff,
 //   dve = 3 s dv_eff, dgate = 3 s (1 - s) sum_d dv_eff ve with s = sigmoid(gate).
-// Both use the prologue's split-halves row layout (each lane holds matching
-// slices of both halves of a row); reductions are shuffles over a row's lanes.
+// Both stage their token block into shared memory with bulk copies issued at
+// kernel start, like the prologue, and use its split-halves row layout (each
+// lane holds matching slices of both halves of a row); reductions are
+// shuffles over a row's lanes.
 #pragma once
 #include "prologue.cuh"
 
@@ -19,52 +21,82 @@ namespace cswattn {
 struct PreParams {
   long long rows;  // B * T * H
   int T, H, Tpad;
+  int tok;                     // tokens per CTA (1..kPrologueTok)
+  unsigned long long wait_ns;  // bound of the staging wait
   const void *O, *dO;
   const float* lse;  // (B, H, T)
   float* delta;      // (B, H, Tpad)
   float* lse2;       // (B, H, Tpad)
+  float* dq_zero;    // (B, T, H, D) accumulator to clear, or null
 };
 
-// One CTA per kPrologueTok consecutive tokens; each row (token, head) is
-// owned by LPR lanes in the prologue's split-halves layout (two vector loads
-// per lane per tensor), reduced with shuffles.
-template <typename T, int D>
+__host__ __device__ inline size_t preprocess_stage_bytes(int tok, int H, int D, int esize) {
+  return 2 * static_cast<size_t>(tok) * H * D * esize;
+}
+
+// One CTA per `tok` consecutive tokens, staged like the prologue (one bulk
+// copy each for the block's O and dO rows); each row (token, head) is owned
+// by LPR lanes in the split-halves layout, reduced with shuffles.
+template <typename T, int D, bool STAGED>
 __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreParams p) {
   using RL = RowLayout<T, D>;
   using HVec = HalfVec<T, RL::HV>;
   constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
   __shared__ int s_b[kPrologueTok], s_t[kPrologueTok];
-  __shared__ bool s_valid[kPrologueTok];
+  __shared__ uint64_t s_bar;
+  extern __shared__ __align__(128) uint8_t stage_smem[];
   const long long n_tok = p.rows / p.H;
-  const long long tok0 = static_cast<long long>(blockIdx.x) * kPrologueTok;
-  if (threadIdx.x < kPrologueTok) {
+  const long long tok0 = static_cast<long long>(blockIdx.x) * p.tok;
+  const int ntt = static_cast<int>(n_tok - tok0 < p.tok ? n_tok - tok0 : p.tok);
+  const size_t orow = static_cast<size_t>(p.H) * D;
+  const T* ob = static_cast<const T*>(p.O) + tok0 * orow;
+  const T* gb = static_cast<const T*>(p.dO) + tok0 * orow;
+  const Stage stage{&s_bar};
+  if constexpr (STAGED) {
+    T* so = reinterpret_cast<T*>(stage_smem);
+    T* sg = so + p.tok * orow;
+    if (threadIdx.x == 0) {
+      const uint32_t nb = static_cast<uint32_t>(ntt * orow * sizeof(T));
+      stage.arm(2 * nb);
+      stage.copy(so, ob, nb);
+      stage.copy(sg, gb, nb);
+    }
+    ob = so;
+    gb = sg;
+  }
+  if (threadIdx.x < ntt) {
     const long long tok = tok0 + threadIdx.x;
-    s_valid[threadIdx.x] = tok < n_tok;
-    const long long tk = tok < n_tok ? tok : 0;
-    s_b[threadIdx.x] = static_cast<int>(tk / p.T);
-    s_t[threadIdx.x] = static_cast<int>(tk % p.T);
+    s_b[threadIdx.x] = static_cast<int>(tok / p.T);
+    s_t[threadIdx.x] = static_cast<int>(tok % p.T);
+  }
+  if (p.dq_zero) {
+    // The block's rows of the dq accumulator (contiguous in (B,T,H,D)).
+    float4* z = reinterpret_cast<float4*>(p.dq_zero + tok0 * orow);
+    const int n4 = static_cast<int>(ntt * orow / 4);
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
+  if constexpr (STAGED) {
+    if (!stage.wait(p.wait_ns)) return;
+  }
   const int sub = threadIdx.x % LPR;
   const int grp = threadIdx.x / LPR;
-  const int total_rows = kPrologueTok * p.H;
+  const int total_rows = ntt * p.H;
   RowCursor cur{0, 0};
   cur.advance(grp, p.H);
   for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
-    const bool in_range = base + grp < total_rows;
-    const int tt = in_range ? cur.tt : 0, h = in_range ? cur.kind_row : 0;
+    const bool valid = base + grp < total_rows;
+    const int tt = valid ? cur.tt : 0, h = valid ? cur.kind_row : 0;
     cur.advance(ROWS_PER_PASS, p.H);
-    const bool valid = in_range && s_valid[tt];
-    const long long row = (tok0 + tt) * p.H + h;  // (b*T + t)*H + h
     float acc = 0.f;
     if (valid) {
-      const size_t lo = static_cast<size_t>(row) * D + sub * HV;
+      const size_t lo = (static_cast<size_t>(tt) * p.H + h) * D + sub * HV;
       float o0[HV], o1[HV], g0[HV], g1[HV];
-      HVec::load(static_cast<const T*>(p.O) + lo, o0);
-      HVec::load(static_cast<const T*>(p.O) + lo + HALF, o1);
-      HVec::load(static_cast<const T*>(p.dO) + lo, g0);
-      HVec::load(static_cast<const T*>(p.dO) + lo + HALF, g1);
+      HVec::load(ob + lo, o0);
+      HVec::load(ob + lo + HALF, o1);
+      HVec::load(gb + lo, g0);
+      HVec::load(gb + lo + HALF, g1);
 #pragma unroll
       for (int i = 0; i < HV; ++i) acc = fmaf(o0[i], g0[i], fmaf(o1[i], g1[i], acc));
     }
@@ -87,15 +119,26 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
 struct EpiParams {
   int B, T, H, Hk;
   int has_ve;
+  int tok;                              // tokens per CTA (1..kPrologueTok)
+  unsigned long long wait_ns;           // bound of the staging wait
   float omega[kMaxHalfD];
   const void *q, *k, *ve, *gate;        // prologue inputs (layer dtype)
   const float *rstd_q, *rstd_k;
-  const float* dq_acc;                  // (B,H,T,D) dq~ (scaled)
+  const float* dq_acc;                  // (B,T,H,D) dq~ (scaled)
   const float *dk_acc, *dv_acc;         // [parts] x (B,T,Hk,D) partial dk~ (scaled), dv_eff
   int parts;                            // number of partial slots to sum
   long long kv_stride;                  // elements between partial slots
   void *dq, *dk, *dv, *dve, *dgate;     // outputs (layer dtype)
 };
+
+// Shared-memory bytes of the staged epilogue for `tok` tokens: dq~, the dk~
+// and dv_eff partial slots (float32), then q, k and ve (layer dtype).
+__host__ __device__ inline size_t epilogue_stage_bytes(int tok, int H, int Hk, int D, int esize,
+                                                       int parts, bool has_ve) {
+  return static_cast<size_t>(tok) * D *
+         ((static_cast<size_t>(H) + 2 * static_cast<size_t>(parts) * Hk) * 4 +
+          (static_cast<size_t>(H) + (has_ve ? 2 : 1) * Hk) * esize);
+}
 
 template <int VEC>
 __device__ __forceinline__ void load_f32(const float* src, float (&x)[VEC]) {
@@ -118,7 +161,7 @@ __device__ __forceinline__ void load_f32(const float* src, float (&x)[VEC]) {
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool STAGED>
 __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiParams p) {
   using RL = RowLayout<T, D>;
   using HVec = HalfVec<T, RL::HV>;
@@ -126,27 +169,71 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
 
   __shared__ __align__(16) TokenTable<HALF> tab;
+  __shared__ uint64_t s_bar;
+  extern __shared__ __align__(128) uint8_t stage_smem[];
 
   const long long n_tok = static_cast<long long>(p.B) * p.T;
-  const long long tok0 = static_cast<long long>(blockIdx.x) * kPrologueTok;
-  tab.fill(tok0, n_tok, p.T, p.omega);
+  const long long tok0 = static_cast<long long>(blockIdx.x) * p.tok;
+  const int ntt = static_cast<int>(n_tok - tok0 < p.tok ? n_tok - tok0 : p.tok);
+  // Block bases: token tt, head h of a tensor with n heads is row tt * n + h.
+  const size_t qrow = static_cast<size_t>(p.H) * D, kvrow = static_cast<size_t>(p.Hk) * D;
+  // Element stride between partial slots as seen from the block bases.
+  size_t slot = static_cast<size_t>(p.kv_stride);
+  const float* dqb = p.dq_acc + tok0 * qrow;
+  const float* dkb = p.dk_acc + tok0 * kvrow;
+  const float* dvb = p.dv_acc + tok0 * kvrow;
+  const T* qb = static_cast<const T*>(p.q) + tok0 * qrow;
+  const T* kb = static_cast<const T*>(p.k) + tok0 * kvrow;
+  const T* eb = p.has_ve ? static_cast<const T*>(p.ve) + tok0 * kvrow : nullptr;
+  const Stage stage{&s_bar};
+  if constexpr (STAGED) {
+    float* sdq = reinterpret_cast<float*>(stage_smem);
+    float* sdk = sdq + p.tok * qrow;
+    float* sdv = sdk + p.parts * p.tok * kvrow;
+    T* sq = reinterpret_cast<T*>(sdv + p.parts * p.tok * kvrow);
+    T* sk = sq + p.tok * qrow;
+    T* se = sk + p.tok * kvrow;
+    if (threadIdx.x == 0) {
+      const uint32_t qf = static_cast<uint32_t>(ntt * qrow * 4);
+      const uint32_t kf = static_cast<uint32_t>(ntt * kvrow * 4);
+      const uint32_t qh = static_cast<uint32_t>(ntt * qrow * sizeof(T));
+      const uint32_t kh = static_cast<uint32_t>(ntt * kvrow * sizeof(T));
+      stage.arm(qf + 2 * p.parts * kf + qh + (p.has_ve ? 2u : 1u) * kh);
+      stage.copy(sdq, dqb, qf);
+      for (int pi = 0; pi < p.parts; ++pi) {
+        stage.copy(sdk + pi * p.tok * kvrow, dkb + pi * slot, kf);
+        stage.copy(sdv + pi * p.tok * kvrow, dvb + pi * slot, kf);
+      }
+      stage.copy(sq, qb, qh);
+      stage.copy(sk, kb, kh);
+      if (p.has_ve) stage.copy(se, eb, kh);
+    }
+    dqb = sdq;
+    dkb = sdk;
+    dvb = sdv;
+    slot = p.tok * kvrow;
+    qb = sq;
+    kb = sk;
+    eb = se;
+  }
+  tab.fill(tok0, p.T, p.omega, ntt);
   __syncthreads();
+  if constexpr (STAGED) {
+    if (!stage.wait(p.wait_ns)) return;
+  }
 
   const int rows_per_tok = p.H + 2 * p.Hk;
-  const int total_rows = kPrologueTok * rows_per_tok;
+  const int total_rows = ntt * rows_per_tok;
   const int sub = threadIdx.x % LPR;
   const int grp = threadIdx.x / LPR;
   RowCursor cur{0, 0};
   cur.advance(grp, rows_per_tok);
 
   for (int base = 0; base < total_rows; base += ROWS_PER_PASS) {
-    const bool in_range = base + grp < total_rows;
-    const int tt = in_range ? cur.tt : 0;
-    const int kind_row = in_range ? cur.kind_row : 0;
+    const bool valid = base + grp < total_rows;
+    const int tt = valid ? cur.tt : 0;
+    const int kind_row = valid ? cur.kind_row : 0;
     cur.advance(ROWS_PER_PASS, rows_per_tok);
-    const bool valid = in_range && tab.valid[tt];
-    const int t = tab.t[tt];
-    const long long b = tab.b[tt];
     int kind, head, nheads;
     if (kind_row < p.H) {
       kind = 0; head = kind_row; nheads = p.H;
@@ -155,32 +242,27 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
     } else {
       kind = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
     }
-    const size_t row = static_cast<size_t>(valid ? tok0 + tt : 0) * nheads + head;  // (b,t,head)
+    // Row within the block (sources) and within the tensor (destinations).
+    const size_t brow = static_cast<size_t>(tt) * nheads + head;
+    const size_t row = static_cast<size_t>(tok0 + tt) * nheads + head;  // (b,t,head)
     const size_t off_lo = row * D + static_cast<size_t>(sub) * HV;
     const size_t off_hi = off_lo + HALF;
+    const size_t boff = brow * D + static_cast<size_t>(sub) * HV;
 
     // Gradient w.r.t. the rotated, normalised row (or dv_eff for value rows),
     // and the row's input (q or k) or ve.
     float dl[HV], dh[HV], xl[HV], xh[HV];
     float rs = 0.f, gl = 0.f;
     if (valid) {
-      const float* src;
-      size_t so;
-      if (kind == 0) {
-        src = p.dq_acc;
-        so = ((static_cast<size_t>(b) * p.H + head) * p.T + t) * D + sub * HV;
-      } else {
-        src = kind == 1 ? p.dk_acc : p.dv_acc;
-        so = off_lo;
-      }
-      load_f32<HV>(src + so, dl);
-      load_f32<HV>(src + so + HALF, dh);
+      const float* src = kind == 0 ? dqb : (kind == 1 ? dkb : dvb);
+      load_f32<HV>(src + boff, dl);
+      load_f32<HV>(src + boff + HALF, dh);
       if (kind != 0) {
         // dK / dV arrive as partial sums from the backward's parts.
         for (int pi = 1; pi < p.parts; ++pi) {
           float el[HV], eh[HV];
-          load_f32<HV>(src + pi * p.kv_stride + so, el);
-          load_f32<HV>(src + pi * p.kv_stride + so + HALF, eh);
+          load_f32<HV>(src + pi * slot + boff, el);
+          load_f32<HV>(src + pi * slot + boff + HALF, eh);
 #pragma unroll
           for (int i = 0; i < HV; ++i) {
             dl[i] += el[i];
@@ -189,12 +271,12 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
         }
       }
       if (kind != 2) {
-        HVec::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off_lo, xl);
-        HVec::load(static_cast<const T*>(kind == 0 ? p.q : p.k) + off_hi, xh);
+        HVec::load((kind == 0 ? qb : kb) + boff, xl);
+        HVec::load((kind == 0 ? qb : kb) + boff + HALF, xh);
         rs = (kind == 0 ? p.rstd_q : p.rstd_k)[row];
       } else if (p.has_ve) {
-        HVec::load(static_cast<const T*>(p.ve) + off_lo, xl);
-        HVec::load(static_cast<const T*>(p.ve) + off_hi, xh);
+        HVec::load(eb + boff, xl);
+        HVec::load(eb + boff + HALF, xh);
         gl = Vec16<T>::scalar(p.gate, row);
       } else {
 #pragma unroll

@@ -56,6 +56,10 @@ constexpr int kOffV = kOffK + kKVBytes;
 constexpr int kOffQD = kOffV + kKVBytes;                 // [kQStages] x (Q | dO)
 constexpr int kOffDS = kOffQD + kQStages * kStageBytes;  // dS^T [2]
 constexpr int kOffBar = kOffDS + 2 * kPBytes;
+// dK/dV write-out staging over the Q/dO ring and dS^T buffers: 2 x 4 panels
+// of 128 rows x 32 float32.
+constexpr int kF32Panel = kBN * 128;
+static_assert(kOffQD + 8 * kF32Panel <= kOffBar, "write-out staging");
 constexpr int kOffRow = kOffBar + 256;         // per Q stage: lse2[64], delta[64]
 constexpr int kSmemBytes = kOffRow + kQStages * 2 * kBQ * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -80,7 +84,7 @@ struct Params {
   float scale;       // c
   const float* lse2;   // (B,H,Tpad) lse * log2(e), +inf past T
   const float* delta;  // (B,H,Tpad) dO.O, 0 past T
-  float* dq_acc;       // (B,H,T,D), accumulated (must start at zero)
+  float* dq_acc;       // (B,T,H,D), accumulated (must start at zero)
   float* dk_acc;       // [parts] x (B,T,Hk,D) partial sums
   float* dv_acc;       // [parts] x (B,T,Hk,D) partial sums
   unsigned long long wait_ns;
@@ -103,6 +107,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -120,6 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = bars + 17;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
+  uint64_t* kv_staged = bars + 20;  // dK/dV rows written to shared memory
   float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [kQStages][64]
   float* s_delta = s_lse2 + kQStages * kBQ;                         // [kQStages][64]
 
@@ -158,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&dq_empty[s], 128);
     }
     mbar_init(acc_full, 1);
+    mbar_init(kv_staged, 128);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -197,6 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmDO);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      prefetch_tmap(&tmDK);
+      prefetch_tmap(&tmDV);
       Cursor c = cur0;
       int st = 0, use = 0;
       mbar_expect_tx(kv_full, 2 * kKVBytes);
@@ -390,36 +399,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // dK / dV write-out: thread r holds key row r of both accumulators.
+    // dK / dV write-out: thread r holds key row r of both accumulators. The
+    // rows go through shared memory (the Q/dO ring and the dS^T buffers,
+    // free once acc_full has fired) as four 32-column float32 panels per
+    // tensor in the 128B-swizzled layout of the tensor maps; eight TMA
+    // stores then write the tile (rows past T are not written).
     const bool acc_ok = ok && mbar_wait(acc_full, 0, wc);
     if (__all_sync(0xffffffffu, acc_ok)) {
       tc_fence_after();
-      const bool row_ok = kj < p.T;
       const float keep = N > 0 ? 1.f : 0.f;  // a part without steps writes zeros
-      const size_t off = static_cast<size_t>(part) * p.kv_stride +
-                         ((static_cast<size_t>(b) * p.T + (row_ok ? kj : 0)) * p.Hk + hk) * kD;
+      uint8_t* stv = smem + kOffQD;           // dV panels
+      uint8_t* stk = stv + 4 * kF32Panel;     // dK panels
+      auto stage_row = [&](uint8_t* panel, const uint32_t (&a)[32], float sc) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<float4*>(panel + r * 128 + ((k ^ (r & 7)) << 4)) =
+              make_float4(__uint_as_float(a[4 * k]) * sc, __uint_as_float(a[4 * k + 1]) * sc,
+                          __uint_as_float(a[4 * k + 2]) * sc, __uint_as_float(a[4 * k + 3]) * sc);
+      };
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t a[32];
         tmem_ld32(tmem + lane_off + kColDV + c * 32, a);
         tmem_ld_wait();
-        if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(p.dv_acc + off + c * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            dst[v4] = make_float4(__uint_as_float(a[4 * v4]) * keep, __uint_as_float(a[4 * v4 + 1]) * keep,
-                                  __uint_as_float(a[4 * v4 + 2]) * keep, __uint_as_float(a[4 * v4 + 3]) * keep);
-        }
+        stage_row(stv + c * kF32Panel, a, keep);
         tmem_ld32(tmem + lane_off + kColDK + c * 32, a);
         tmem_ld_wait();
-        if (row_ok) {
-          float4* dst = reinterpret_cast<float4*>(p.dk_acc + off + c * 32);
-          const float sc = p.scale * keep;
+        stage_row(stk + c * kF32Panel, a, p.scale * keep);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(kv_staged);
+      if (r == 0 && mbar_wait(kv_staged, 0, wc)) {
+        const int outer = part * p.B + b;  // partial slot `part` of batch b
 #pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            dst[v4] = make_float4(__uint_as_float(a[4 * v4]) * sc, __uint_as_float(a[4 * v4 + 1]) * sc,
-                                  __uint_as_float(a[4 * v4 + 2]) * sc, __uint_as_float(a[4 * v4 + 3]) * sc);
+        for (int c = 0; c < 4; ++c) {
+          tma_store_4d(&tmDV, stv + c * kF32Panel, 32 * c, hk, k0, outer);
+          tma_store_4d(&tmDK, stk + c * kF32Panel, 32 * c, hk, k0, outer);
         }
+        bulk_commit();
+        bulk_wait0();
       }
     }
   } else {
@@ -444,15 +462,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&dq_empty[st]);
-      // Column q of dQ^T -> dq_acc[b][h][q0 + q][d]; the warp's 32 lanes hit
+      // Column q of dQ^T -> dq_acc[b][q0 + q][h][d]; the warp's 32 lanes hit
       // 32 consecutive floats (one 128-byte reduction request per query).
-      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.T + q0) * kD + d;
+      const size_t qstride = static_cast<size_t>(p.H) * kD;
+      float* dst = p.dq_acc + (static_cast<size_t>(b) * p.T + q0) * qstride +
+                   static_cast<size_t>(h) * kD + d;
       const int nrows = min(kBQ, p.T - q0);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (cc * 32 + i < nrows) red_add_f32(dst + (cc * 32 + i) * kD, __uint_as_float(a[cc][i]) * sc);
+          if (cc * 32 + i < nrows) red_add_f32(dst + (cc * 32 + i) * qstride, __uint_as_float(a[cc][i]) * sc);
     }
   }
 

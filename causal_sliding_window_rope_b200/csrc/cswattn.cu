@@ -134,19 +134,25 @@ cswattn_status get_encoder(EncodeTiledFn* fn) {
 
 // (B, T, heads, 128) bf16 tensor; box = 64 head_dim elements x `rows` tokens
 // of one head, 128-byte swizzle; out-of-range rows read as zero.
-cswattn_status make_map(CUtensorMap* map, const void* base, int B, int T, int heads, int rows) {
+// Tensor map of a (outer, T, heads, 128) row-major tensor of bf16 (or
+// float32) viewed as 4-D (128, heads, T, outer); a box is one 128-byte
+// column panel (64 bf16 or 32 float32) of `rows` rows of one head, 128B-swizzled.
+cswattn_status make_map(CUtensorMap* map, const void* base, int outer, int T, int heads, int rows,
+                        bool f32 = false) {
   EncodeTiledFn enc;
   cswattn_status s = get_encoder(&enc);
   if (s != CSWATTN_OK) return s;
+  const cuuint64_t es = f32 ? 4 : 2;
   const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(T),
-                              static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(heads) * 256,
-                                 static_cast<cuuint64_t>(T) * heads * 256};
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+                              static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[3] = {128 * es, static_cast<cuuint64_t>(heads) * 128 * es,
+                                 static_cast<cuuint64_t>(T) * heads * 128 * es};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return CSWATTN_OK;
 }
@@ -166,46 +172,98 @@ cswattn_status launched(const char* what) {
   return CSWATTN_OK;
 }
 
-template <typename T>
-void launch_prologue(const Shape& s, const PrologueParams& pp, cudaStream_t st) {
-  const long long ntok = static_cast<long long>(s.B) * s.T;
-  const unsigned grid = static_cast<unsigned>((ntok + kPrologueTok - 1) / kPrologueTok);
-  switch (s.D) {
-    case 4: if constexpr (sizeof(T) == 4) prologue_kernel<T, 4><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 8: if constexpr (sizeof(T) == 4) prologue_kernel<T, 8><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 16: if constexpr (sizeof(T) == 4) prologue_kernel<T, 16><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 32: if constexpr (sizeof(T) == 4) prologue_kernel<T, 32><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 64: if constexpr (sizeof(T) == 4) prologue_kernel<T, 64><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    default: prologue_kernel<T, 128><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+// Launch shape of a row kernel (prologue, backward preprocess, backward
+// epilogue). The staged form copies a CTA's whole token block into shared
+// memory up front: it takes as many tokens as fit in kRowStageTarget bytes
+// (so that several CTAs per SM have their copies in flight), at most
+// kPrologueTok. A layer whose single token needs more than kRowStageMax
+// bytes runs the direct form (tok = 0), which reads global memory row by row.
+constexpr size_t kRowStageTarget = 64u << 10;
+constexpr size_t kRowStageMax = 200u << 10;
+
+struct RowLaunch {
+  int tok;       // tokens per CTA of the staged form, 0 for the direct form
+  size_t smem;   // dynamic shared memory of the staged form
+  unsigned grid;
+};
+
+RowLaunch row_launch(long long ntok, size_t per_tok) {
+  RowLaunch r{0, 0, 0};
+  if (per_tok > 0 && per_tok <= kRowStageMax) {
+    r.tok = static_cast<int>(std::min<size_t>(kPrologueTok, std::max<size_t>(1, kRowStageTarget / per_tok)));
+    r.smem = r.tok * per_tok;
   }
+  const int per_cta = r.tok > 0 ? r.tok : kPrologueTok;
+  r.grid = static_cast<unsigned>((ntok + per_cta - 1) / per_cta);
+  return r;
+}
+
+template <auto STAGED_K, auto DIRECT_K, typename P>
+cswattn_status launch_rows(P p, const RowLaunch& r, cudaStream_t st) {
+  p.wait_ns = g_wait_ns.load();
+  if (r.tok > 0) {
+    static std::once_flag flag;
+    static cudaError_t ferr = cudaSuccess;
+    cswattn_status e = set_smem(STAGED_K, static_cast<int>(kRowStageMax), flag, ferr);
+    if (e != CSWATTN_OK) return e;
+    p.tok = r.tok;
+    STAGED_K<<<r.grid, kPrologueThreads, r.smem, st>>>(p);
+  } else {
+    p.tok = kPrologueTok;
+    DIRECT_K<<<r.grid, kPrologueThreads, 0, st>>>(p);
+  }
+  return CSWATTN_OK;
 }
 
 template <typename T>
-void launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t st) {
-  const long long ntok = static_cast<long long>(s.B) * s.T;
-  const unsigned grid = static_cast<unsigned>((ntok + kPrologueTok - 1) / kPrologueTok);
+cswattn_status launch_prologue(const Shape& s, const PrologueParams& pp, cudaStream_t st) {
+  const RowLaunch r = row_launch(static_cast<long long>(s.B) * s.T,
+                                 prologue_stage_bytes(1, s.H, s.Hk, s.D, s.esize, pp.has_ve != 0));
+#define CSW_ROWS(D_) launch_rows<prologue_kernel<T, D_, true>, prologue_kernel<T, D_, false>>(pp, r, st)
   switch (s.D) {
-    case 4: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 4><<<grid, kPrologueThreads, 0, st>>>(ep); break;
-    case 8: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 8><<<grid, kPrologueThreads, 0, st>>>(ep); break;
-    case 16: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 16><<<grid, kPrologueThreads, 0, st>>>(ep); break;
-    case 32: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 32><<<grid, kPrologueThreads, 0, st>>>(ep); break;
-    case 64: if constexpr (sizeof(T) == 4) epilogue_kernel<T, 64><<<grid, kPrologueThreads, 0, st>>>(ep); break;
-    default: epilogue_kernel<T, 128><<<grid, kPrologueThreads, 0, st>>>(ep); break;
+    case 4: if constexpr (sizeof(T) == 4) return CSW_ROWS(4); break;
+    case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
+    case 16: if constexpr (sizeof(T) == 4) return CSW_ROWS(16); break;
+    case 32: if constexpr (sizeof(T) == 4) return CSW_ROWS(32); break;
+    case 64: if constexpr (sizeof(T) == 4) return CSW_ROWS(64); break;
+    default: return CSW_ROWS(128);
   }
+#undef CSW_ROWS
+  return fail(CSWATTN_ERR_UNSUPPORTED, "prologue: head_dim %d", s.D);
 }
 
 template <typename T>
-void launch_preprocess(const Shape& s, const PreParams& pp, cudaStream_t st) {
-  const long long ntok = static_cast<long long>(s.B) * s.T;
-  const unsigned grid = static_cast<unsigned>((ntok + kPrologueTok - 1) / kPrologueTok);
+cswattn_status launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t st) {
+  const RowLaunch r = row_launch(static_cast<long long>(s.B) * s.T,
+                                 epilogue_stage_bytes(1, s.H, s.Hk, s.D, s.esize, ep.parts, ep.has_ve != 0));
+#define CSW_ROWS(D_) launch_rows<epilogue_kernel<T, D_, true>, epilogue_kernel<T, D_, false>>(ep, r, st)
   switch (s.D) {
-    case 4: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 4><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 8: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 8><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 16: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 16><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 32: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 32><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    case 64: if constexpr (sizeof(T) == 4) preprocess_kernel<T, 64><<<grid, kPrologueThreads, 0, st>>>(pp); break;
-    default: preprocess_kernel<T, 128><<<grid, kPrologueThreads, 0, st>>>(pp); break;
+    case 4: if constexpr (sizeof(T) == 4) return CSW_ROWS(4); break;
+    case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
+    case 16: if constexpr (sizeof(T) == 4) return CSW_ROWS(16); break;
+    case 32: if constexpr (sizeof(T) == 4) return CSW_ROWS(32); break;
+    case 64: if constexpr (sizeof(T) == 4) return CSW_ROWS(64); break;
+    default: return CSW_ROWS(128);
   }
+#undef CSW_ROWS
+  return fail(CSWATTN_ERR_UNSUPPORTED, "epilogue: head_dim %d", s.D);
+}
+
+template <typename T>
+cswattn_status launch_preprocess(const Shape& s, const PreParams& pp, cudaStream_t st) {
+  const RowLaunch r = row_launch(static_cast<long long>(s.B) * s.T,
+                                 preprocess_stage_bytes(1, s.H, s.D, s.esize));
+#define CSW_ROWS(D_) launch_rows<preprocess_kernel<T, D_, true>, preprocess_kernel<T, D_, false>>(pp, r, st)
+  switch (s.D) {
+    case 4: if constexpr (sizeof(T) == 4) return CSW_ROWS(4); break;
+    case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
+    case 16: if constexpr (sizeof(T) == 4) return CSW_ROWS(16); break;
+    case 32: if constexpr (sizeof(T) == 4) return CSW_ROWS(32); break;
+    case 64: if constexpr (sizeof(T) == 4) return CSW_ROWS(64); break;
+    default: return CSW_ROWS(128);
+  }
+#undef CSW_ROWS
+  return fail(CSWATTN_ERR_UNSUPPORTED, "preprocess: head_dim %d", s.D);
 }
 
 void launch_simt_fwd(const Shape& s, const SimtParams& sp, cudaStream_t st) {
@@ -480,11 +538,9 @@ cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const vo
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   {
     ScopedTiming tm(CSWATTN_K_PROLOGUE, cs);
-    if (s.bf16)
-      launch_prologue<__nv_bfloat16>(s, pp, cs);
-    else
-      launch_prologue<float>(s, pp, cs);
+    st = s.bf16 ? launch_prologue<__nv_bfloat16>(s, pp, cs) : launch_prologue<float>(s, pp, cs);
   }
+  if (st != CSWATTN_OK) return st;
   return launched("prologue launch");
 }
 
@@ -522,6 +578,8 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
   if ((st = make_map(&mq, q_out, s.B, s.T, s.H, fwd::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, fwd::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, fwd::kBM)) != CSWATTN_OK) return st;
+  CUtensorMap mo;
+  if ((st = make_map(&mo, O, s.B, s.T, s.H, fwd::kBM)) != CSWATTN_OK) return st;
   static std::once_flag flag;
   static cudaError_t ferr;
   if ((st = set_smem(fwd::fwd_kernel, fwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
@@ -541,7 +599,7 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
   const unsigned grid = static_cast<unsigned>(fp.npairs) * s.B * s.Hk;
   {
     ScopedTiming tm(CSWATTN_K_FWD, cs);
-    fwd::fwd_kernel<<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, fp);
+    fwd::fwd_kernel<<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, mo, fp);
   }
   return launched("forward launch");
 }
@@ -597,13 +655,13 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   pre.lse = lse;
   pre.delta = w.delta;
   pre.lse2 = w.lse2;
+  // The tensor-core backward accumulates dq~ with reductions: zero it here.
+  pre.dq_zero = s.bf16 ? w.dq_acc : nullptr;
   {
     ScopedTiming tm(CSWATTN_K_BWD_PRE, cs);
-    if (s.bf16)
-      launch_preprocess<__nv_bfloat16>(s, pre, cs);
-    else
-      launch_preprocess<float>(s, pre, cs);
+    st = s.bf16 ? launch_preprocess<__nv_bfloat16>(s, pre, cs) : launch_preprocess<float>(s, pre, cs);
   }
+  if (st != CSWATTN_OK) return st;
   if ((st = launched("preprocess launch")) != CSWATTN_OK) return st;
 
   if (!s.bf16) {
@@ -631,14 +689,15 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     }
     if ((st = launched("fp32 backward launch")) != CSWATTN_OK) return st;
   } else {
-    const size_t dq_bytes = static_cast<size_t>(s.B) * s.H * s.T * s.D * 4;
-    cudaError_t e = cudaMemsetAsync(w.dq_acc, 0, dq_bytes, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     CUtensorMap mq, mdo, mk, mv;
     if ((st = make_map(&mq, q_out, s.B, s.T, s.H, bwd::kBQ)) != CSWATTN_OK) return st;
     if ((st = make_map(&mdo, dO, s.B, s.T, s.H, bwd::kBQ)) != CSWATTN_OK) return st;
     if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, bwd::kBN)) != CSWATTN_OK) return st;
     if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, bwd::kBN)) != CSWATTN_OK) return st;
+    const int parts = bwd_parts(s);
+    CUtensorMap mdk, mdv;
+    if ((st = make_map(&mdk, w.dk_acc, s.B * parts, s.T, s.Hk, bwd::kBN, true)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, true)) != CSWATTN_OK) return st;
     static std::once_flag flag;
     static cudaError_t ferr;
     if ((st = set_smem(bwd::bwd_kernel, bwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
@@ -658,13 +717,13 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     bp.dq_acc = w.dq_acc;
     bp.dk_acc = w.dk_acc;
     bp.dv_acc = w.dv_acc;
-    bp.parts = bwd_parts(s);
+    bp.parts = parts;
     bp.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
     bp.wait_ns = g_wait_ns.load();
     const unsigned grid = static_cast<unsigned>(bp.nkv) * bp.parts * s.B * s.Hk;
     {
       ScopedTiming tm(CSWATTN_K_BWD, cs);
-      bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, bp);
+      bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, bp);
     }
     if ((st = launched("backward launch")) != CSWATTN_OK) return st;
   }
@@ -694,11 +753,9 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   ep.dgate = dgate;
   {
     ScopedTiming tm(CSWATTN_K_BWD_EPI, cs);
-    if (s.bf16)
-      launch_epilogue<__nv_bfloat16>(s, ep, cs);
-    else
-      launch_epilogue<float>(s, ep, cs);
+    st = s.bf16 ? launch_epilogue<__nv_bfloat16>(s, ep, cs) : launch_epilogue<float>(s, ep, cs);
   }
+  if (st != CSWATTN_OK) return st;
   return launched("epilogue launch");
 }
 

@@ -21,7 +21,9 @@
 //   warp 1      TMEM owner + single-thread MMA issuer
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: thread r
 //               owns TMEM lane r = query row r, so the row max and sum are
-//               in-thread; P goes back to TMEM as bf16 over the S columns
+//               in-thread; P goes back to TMEM as bf16 over the S columns.
+//               At the end each warpgroup stages its O tile (bf16) in its
+//               Q buffer and writes it with two TMA stores.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
 // Per KV tile: S_X = Q_X K_j^T (SS MMA, K-major both), softmax -> P_X,
 // O_X += P_X V_j (TS MMA: P from TMEM, V MN-major from shared memory).
@@ -78,7 +80,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const Params p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -91,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = bars + 17;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
+  uint64_t* o_staged = bars + 20;  // [2] per tile: O rows written to shared memory
 
   const int warp = warp_id(), lane = lane_id();
 
@@ -126,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
       mbar_init(&o_full[s], 1);
+      mbar_init(&o_staged[s], 128);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -158,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
+      prefetch_tmap(&tmO);
       int filled[kSlots] = {0, 0, 0, 0, 0};
       mbar_expect_tx(q_full, (valid[1] ? 2 : 1) * kTileBytes);
       for (int X = 0; X < 2; ++X) {
@@ -363,28 +369,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__all_sync(0xffffffffu, o_ok)) {
         tc_fence_after();
         const float inv_l = 1.f / l;
-        const bool row_ok = qi < p.T;
-        __nv_bfloat16* orow =
-            p.O + ((static_cast<size_t>(b) * p.T + (row_ok ? qi : 0)) * p.H + head[X]) * kD;
+        // Row r of O as bf16 into this tile's Q buffer, which is free once
+        // o_full has fired (every product of the tile is complete), in the
+        // 128B-swizzled two-panel layout of the tensor map; then one TMA
+        // store per panel writes the tile (rows past T are not written).
+        uint8_t* ot = smem + kOffQ + X * kTileBytes;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
-              w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
-              w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
-              w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
-              dst[v4] = w;
-            }
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const int k = c * 4 + v4;  // 16-byte chunk of the 256-byte row
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(ot + (k >> 3) * kPanelBytes + r * 128 + (((k & 7) ^ (r & 7)) << 4)) = w;
           }
         }
-        if (row_ok)
+        fence_proxy_async_smem();
+        mbar_arrive(&o_staged[X]);
+        if (r == 0 && mbar_wait(&o_staged[X], 0, wc)) {
+          tma_store_4d(&tmO, ot, 0, head[X], q0, b);
+          tma_store_4d(&tmO, ot + kPanelBytes, 64, head[X], q0, b);
+          bulk_commit();
+          bulk_wait0();
+        }
+        if (qi < p.T)
           p.lse[(static_cast<size_t>(b) * p.H + head[X]) * p.T + qi] =
               (m2 + log2f(l)) * 0.69314718055994531f;
       }

@@ -5,26 +5,34 @@
 // value-embedding code (v + 3*sigmoid(gate)*ve, one gate per token and KV
 // head, broadcast over head_dim).
 //
-// One CTA handles kTok consecutive tokens (b, t). It first computes
-// cos/sin(t * omega_i) for its tokens into shared memory, then walks the
-// H query rows, Hk key rows and Hk value rows of each token. A row of D
-// elements is owned by LPR = D / (2 HV) lanes; lane l holds the HV-element
-// slices [l HV, (l+1) HV) of both halves of the row (elements i and
-// i + D/2), so every RoPE pair is inside one lane and each lane keeps two
-// vector loads in flight per row. Loads and stores are coalesced vector
-// accesses; the RMS is a shuffle reduction over the row's LPR lanes.
+// One CTA handles `tok` consecutive tokens (b, t). The row kernels are bound
+// by HBM bandwidth and are short (tens of microseconds), so what matters is
+// how many bytes are in flight from the start: in the staged form thread 0
+// issues one bulk copy (cp.async.bulk) per input tensor for the whole token
+// block before anything else happens, and the CTA computes cos/sin(t omega_i)
+// for its tokens into shared memory while the copies land. The rows are then
+// read from shared memory. (The direct form reads global memory row by row;
+// it serves layers whose token block does not fit in shared memory.)
+//
+// A row of D elements is owned by LPR = D / (2 HV) lanes; lane l holds the
+// HV-element slices [l HV, (l+1) HV) of both halves of the row (elements i
+// and i + D/2), so every RoPE pair is inside one lane. The RMS is a shuffle
+// reduction over the row's LPR lanes; results go to global memory as
+// coalesced vector stores.
 #pragma once
 #include "common.cuh"
 
 namespace cswattn {
 
 constexpr int kPrologueThreads = 256;
-constexpr int kPrologueTok = 8;
+constexpr int kPrologueTok = 8;   // most tokens per CTA
 constexpr int kMaxHalfD = 64;
 
 struct PrologueParams {
   int B, T, H, Hk;
   int has_ve;
+  int tok;                  // tokens per CTA (1..kPrologueTok)
+  unsigned long long wait_ns;  // bound of the staging wait
   float eps;
   float omega[kMaxHalfD];  // rope_base^(-2i/D), i < D/2, rounded from double
   const void *q, *k, *v, *ve, *gate;
@@ -119,27 +127,24 @@ __device__ __forceinline__ float row_sum(float v) {
   return v;
 }
 
-// Per-CTA token table of the row kernels: the CTA's kPrologueTok consecutive
-// tokens (b, t), and cos/sin(t * omega_i) for each of them.
+// Per-CTA token table of the row kernels: the CTA's ntt (at most
+// kPrologueTok) consecutive tokens (b, t), and cos/sin(t * omega_i) for each.
 template <int HALF>
 struct TokenTable {
   float cos_[kPrologueTok][HALF];
   float sin_[kPrologueTok][HALF];
   int b[kPrologueTok], t[kPrologueTok];
-  bool valid[kPrologueTok];
 
-  __device__ void fill(long long tok0, long long n_tok, int T, const float* omega) {
-    if (threadIdx.x < kPrologueTok) {
+  // Tokens tok0 .. tok0 + ntt - 1, all of them below B*T.
+  __device__ void fill(long long tok0, int T, const float* omega, int ntt) {
+    if (threadIdx.x < ntt) {
       const long long tok = tok0 + threadIdx.x;
-      valid[threadIdx.x] = tok < n_tok;
-      const long long tk = tok < n_tok ? tok : 0;
-      b[threadIdx.x] = static_cast<int>(tk / T);
-      t[threadIdx.x] = static_cast<int>(tk % T);
+      b[threadIdx.x] = static_cast<int>(tok / T);
+      t[threadIdx.x] = static_cast<int>(tok % T);
     }
-    for (int e = threadIdx.x; e < kPrologueTok * HALF; e += blockDim.x) {
+    for (int e = threadIdx.x; e < ntt * HALF; e += blockDim.x) {
       const int tt = e / HALF, i = e % HALF;
-      const long long tok = tok0 + tt;
-      const int t_ = tok < n_tok ? static_cast<int>(tok % T) : 0;
+      const int t_ = static_cast<int>((tok0 + tt) % T);
       float sn, cs;
       sincosf(static_cast<float>(t_) * omega[i], &sn, &cs);
       cos_[tt][i] = cs;
@@ -180,7 +185,42 @@ struct RowCursor {
   }
 };
 
-template <typename T, int D>
+// Staging of one CTA's token block into shared memory: thread 0 arms the
+// barrier with the block's byte count and issues the bulk copies; every
+// thread later waits for the bytes (bounded; a timeout is recorded in the
+// status word and the CTA computes nothing).
+struct Stage {
+  uint64_t* bar;
+  __device__ void arm(uint32_t bytes) const {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    mbar_expect_tx(bar, bytes);
+  }
+  // bytes: a multiple of 16; both addresses 16-byte aligned.
+  __device__ void copy(void* dst, const void* src, uint32_t bytes) const {
+    bulk_load(dst, src, bytes, bar);
+  }
+  __device__ bool wait(unsigned long long limit_ns) const {
+    if (mbar_try_wait(bar, 0)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, 0)) {
+      if (globaltimer() - t0 > limit_ns) {
+        atomicOr(&g_status, kStatusTimeout);
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+// Shared-memory bytes of the staged prologue for `tok` tokens.
+__host__ __device__ inline size_t prologue_stage_bytes(int tok, int H, int Hk, int D, int esize,
+                                                       bool has_ve) {
+  return static_cast<size_t>(tok) * (H + (has_ve ? 3 : 2) * Hk) * D * esize;
+}
+
+template <typename T, int D, bool STAGED>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_kernel(const PrologueParams p) {
   using RL = RowLayout<T, D>;
@@ -189,14 +229,47 @@ __global__ void __launch_bounds__(kPrologueThreads)
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
 
   __shared__ __align__(16) TokenTable<HALF> tab;
+  __shared__ uint64_t s_bar;
+  extern __shared__ __align__(128) uint8_t stage_smem[];
 
   const long long n_tok = static_cast<long long>(p.B) * p.T;
-  const long long tok0 = static_cast<long long>(blockIdx.x) * kPrologueTok;
-  tab.fill(tok0, n_tok, p.T, p.omega);
+  const long long tok0 = static_cast<long long>(blockIdx.x) * p.tok;
+  const int ntt = static_cast<int>(n_tok - tok0 < p.tok ? n_tok - tok0 : p.tok);
+  // Row bases of the block: token tt, head h of a tensor with n heads is
+  // row tt * n + h from these.
+  const size_t qrow = static_cast<size_t>(p.H) * D, kvrow = static_cast<size_t>(p.Hk) * D;
+  const T *qb = static_cast<const T*>(p.q) + tok0 * qrow;
+  const T *kb = static_cast<const T*>(p.k) + tok0 * kvrow;
+  const T *vb = static_cast<const T*>(p.v) + tok0 * kvrow;
+  const T *eb = p.has_ve ? static_cast<const T*>(p.ve) + tok0 * kvrow : nullptr;
+  const Stage stage{&s_bar};
+  if constexpr (STAGED) {
+    T* sq = reinterpret_cast<T*>(stage_smem);
+    T* sk = sq + p.tok * qrow;
+    T* sv = sk + p.tok * kvrow;
+    T* se = sv + p.tok * kvrow;
+    if (threadIdx.x == 0) {
+      const uint32_t qb_ = static_cast<uint32_t>(ntt * qrow * sizeof(T));
+      const uint32_t kb_ = static_cast<uint32_t>(ntt * kvrow * sizeof(T));
+      stage.arm(qb_ + (p.has_ve ? 3u : 2u) * kb_);
+      stage.copy(sq, qb, qb_);
+      stage.copy(sk, kb, kb_);
+      stage.copy(sv, vb, kb_);
+      if (p.has_ve) stage.copy(se, eb, kb_);
+    }
+    qb = sq;
+    kb = sk;
+    vb = sv;
+    eb = se;
+  }
+  tab.fill(tok0, p.T, p.omega, ntt);
   __syncthreads();
+  if constexpr (STAGED) {
+    if (!stage.wait(p.wait_ns)) return;
+  }
 
   const int rows_per_tok = p.H + 2 * p.Hk;
-  const int total_rows = kPrologueTok * rows_per_tok;
+  const int total_rows = ntt * rows_per_tok;
   const int sub = threadIdx.x % LPR;  // lane within the row group
   const int grp = threadIdx.x / LPR;  // row group within the CTA
   RowCursor cur{0, 0};
@@ -208,7 +281,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
     const int tt = in_range ? cur.tt : 0;
     const int kind_row = in_range ? cur.kind_row : 0;
     cur.advance(ROWS_PER_PASS, rows_per_tok);
-    const bool valid = in_range && tab.valid[tt];
+    const bool valid = in_range;  // every token of the block exists
     // Row kinds: [0, H) query heads, [H, H+Hk) key heads, then value heads.
     int kind, head, nheads;
     if (kind_row < p.H) {
@@ -218,23 +291,26 @@ __global__ void __launch_bounds__(kPrologueThreads)
     } else {
       kind = 2; head = kind_row - p.H - p.Hk; nheads = p.Hk;
     }
+    // Row within the block (source) and within the tensor (destination).
+    const size_t brow = static_cast<size_t>(tt) * nheads + head;
     const size_t row = static_cast<size_t>(valid ? tok0 + tt : 0) * nheads + head;
     const size_t off_lo = row * D + static_cast<size_t>(sub) * HV;
     const size_t off_hi = off_lo + HALF;
-    const T* src = static_cast<const T*>(kind == 0 ? p.q : (kind == 1 ? p.k : p.v));
+    const size_t boff = brow * D + static_cast<size_t>(sub) * HV;
+    const T* src = kind == 0 ? qb : (kind == 1 ? kb : vb);
     float xl[HV], xh[HV], el[HV], eh[HV];
     float gl = 0.f;
     if (valid) {
-      HVec::load(src + off_lo, xl);
-      HVec::load(src + off_hi, xh);
+      HVec::load(src + boff, xl);
+      HVec::load(src + boff + HALF, xh);
     } else {
 #pragma unroll
       for (int i = 0; i < HV; ++i) xl[i] = xh[i] = 0.f;
     }
     const bool has_e = valid && kind == 2 && p.has_ve;
     if (has_e) {
-      HVec::load(static_cast<const T*>(p.ve) + off_lo, el);
-      HVec::load(static_cast<const T*>(p.ve) + off_hi, eh);
+      HVec::load(eb + boff, el);
+      HVec::load(eb + boff + HALF, eh);
       gl = Vec16<T>::scalar(p.gate, row);
     } else {
 #pragma unroll

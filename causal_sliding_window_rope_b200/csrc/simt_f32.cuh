@@ -20,7 +20,7 @@ struct SimtParams {
   const float *O, *dO, *lse;   // backward inputs
   const float* delta;          // (B,H,Tpad) dO.O
   float *out_O, *out_lse;      // forward outputs
-  float *dq_acc;               // (B,H,T,D) dq~ (scaled)
+  float *dq_acc;               // (B,T,H,D) dq~ (scaled)
   float *dk_acc, *dv_acc;      // (B,T,Hk,D) dk~ (scaled), dv_eff
 };
 
@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const SimtParams p) {
   p.out_lse[(static_cast<size_t>(b) * p.H + h) * p.T + i] = m + logf(l);
 }
 
-// dq~_i = c * sum_j p_ij (dp_ij - Delta_i) k~_j, written to dq_acc (B,H,T,D).
+// dq~_i = c * sum_j p_ij (dp_ij - Delta_i) k~_j, written to dq_acc (B,T,H,D).
 template <int D>
 __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const SimtParams p) {
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(128) simt_bwd_dq_kernel(const SimtParams p) {
 #pragma unroll
     for (int d = 0; d < D; ++d) acc[d] = fmaf(ds, p.k[kv + d], acc[d]);
   }
-  float* out = p.dq_acc + row * D;
+  float* out = p.dq_acc + qo;
 #pragma unroll
   for (int d = 0; d < D; ++d) out[d] = acc[d] * p.scale;
 }
