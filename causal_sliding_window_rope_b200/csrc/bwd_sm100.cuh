@@ -22,11 +22,12 @@
 //   dK  += dS^T Q     (same shape)                         TS MMA (dS^T in TMEM)
 //   dQ^T = K^T dS^T   (M=128 d, N=64 queries, K=128 keys)   SS MMA, over the
 //          P^T/dS^T columns (issued after the two TS MMAs that read them),
-//          drained by the dQ warps straight from TMEM with float32
-//          reductions into the dq accumulator (one 128-byte request per warp
-//          and query).
-// Shared memory holds only the MMA operands (K, V, the Q/dO ring, dS^T), so
-// the SS products, which are bound by shared-memory bandwidth, get most of it.
+//          drained by the dQ warps from TMEM into a swizzled shared tile
+//          that four TMA float32 add-reductions send into the dq
+//          accumulator (B,T,H,D).
+// Shared memory holds the MMA operands (K, V, the Q/dO ring, dS^T) and the
+// dQ staging tile; at the end the ring and dS^T buffers stage dK/dV for
+// their TMA stores.
 // TMEM (512 columns): SP (S^T at +0, dP^T at +64) | dQ^T x2 (64 columns
 // each; also P^T at +0 and dS^T at +32 before the dQ^T product) | dV | dK.
 // The softmax warps release SP as soon as they have loaded it into
@@ -55,11 +56,14 @@ constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKVBytes;
 constexpr int kOffQD = kOffV + kKVBytes;                 // [kQStages] x (Q | dO)
 constexpr int kOffDS = kOffQD + kQStages * kStageBytes;  // dS^T [2]
-constexpr int kOffBar = kOffDS + 2 * kPBytes;
+// dQ^T drain staging: 4 panels of 64 query rows x 32 float32 (128B-swizzled).
+constexpr int kOffDQS = kOffDS + 2 * kPBytes;
+constexpr int kDQPanel = kBQ * 128;
+constexpr int kOffBar = kOffDQS + 4 * kDQPanel;
 // dK/dV write-out staging over the Q/dO ring and dS^T buffers: 2 x 4 panels
 // of 128 rows x 32 float32.
 constexpr int kF32Panel = kBN * 128;
-static_assert(kOffQD + 8 * kF32Panel <= kOffBar, "write-out staging");
+static_assert(kOffQD + 8 * kF32Panel <= kOffDQS, "write-out staging");
 constexpr int kOffRow = kOffBar + 256;         // per Q stage: lse2[64], delta[64]
 constexpr int kSmemBytes = kOffRow + kQStages * 2 * kBQ * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-               const Params p) {
+               const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -126,6 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
   uint64_t* kv_staged = bars + 20;  // dK/dV rows written to shared memory
+  uint64_t* dqs_full = bars + 21;   // dQ^T staging tile written (128 arrivals)
+  uint64_t* dqs_free = bars + 22;   // the reduction has read the staging tile
   float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [kQStages][64]
   float* s_delta = s_lse2 + kQStages * kBQ;                         // [kQStages][64]
 
@@ -165,6 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(kv_staged, 128);
+    mbar_init(dqs_full, 128);
+    mbar_init(dqs_free, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -206,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmDK);
       prefetch_tmap(&tmDV);
+      prefetch_tmap(&tmDQ);
       Cursor c = cur0;
       int st = 0, use = 0;
       mbar_expect_tx(kv_full, 2 * kKVBytes);
@@ -449,6 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = (warp & 3) * 32 + lane;  // TMEM lane = head_dim index of dQ^T
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sc = p.scale;
+    uint8_t* stile = smem + kOffDQS;
+    const bool leader = threadIdx.x == 256;
     Cursor c = cur0;
     for (int n = 0; n < N; ++n, c.next()) {
       const int st = n & 1, use = n >> 1;
@@ -462,18 +473,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&dq_empty[st]);
-      // Column q of dQ^T -> dq_acc[b][q0 + q][h][d]; the warp's 32 lanes hit
-      // 32 consecutive floats (one 128-byte reduction request per query).
-      const size_t qstride = static_cast<size_t>(p.H) * kD;
-      float* dst = p.dq_acc + (static_cast<size_t>(b) * p.T + q0) * qstride +
-                   static_cast<size_t>(h) * kD + d;
-      const int nrows = min(kBQ, p.T - q0);
+      // Column q of dQ^T is row q of the step's dQ~ tile: stage it in four
+      // 32-column panels (128B-swizzled; the warp's 32 lanes fill one
+      // 128-byte row, conflict-free) and add the tile into dq_acc with four
+      // TMA reductions (rows past T are skipped).
+      got = n == 0 || mbar_wait(dqs_free, (n - 1) & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) break;
+      uint8_t* prow = stile + (d >> 5) * kDQPanel + (d & 3) * 4;
+      const int chunk = (d & 31) >> 2;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (cc * 32 + i < nrows) red_add_f32(dst + (cc * 32 + i) * qstride, __uint_as_float(a[cc][i]) * sc);
+        for (int i = 0; i < 32; ++i) {
+          const int q = cc * 32 + i;
+          *reinterpret_cast<float*>(prow + q * 128 + ((chunk ^ (q & 7)) << 4)) = __uint_as_float(a[cc][i]) * sc;
+        }
+      fence_proxy_async_smem();
+      mbar_arrive(dqs_full);
+      if (leader) {
+        if (mbar_wait(dqs_full, n & 1, wc)) {
+#pragma unroll
+          for (int pc = 0; pc < 4; ++pc) tma_reduce_add_4d(&tmDQ, stile + pc * kDQPanel, 32 * pc, h, q0, b);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        mbar_arrive(dqs_free);
+      }
     }
+    if (leader) bulk_wait0();
   }
 
   tc_fence_before();

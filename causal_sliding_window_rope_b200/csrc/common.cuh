@@ -140,6 +140,17 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
       : "memory");
 }
 
+// 4-D tile float32 add-reduction shared -> global (bulk group; out-of-range
+// rows are skipped). The coordinates must be non-negative.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0,
+                                                  int c1, int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 // Untiled bulk copy global -> shared of `bytes` (multiple of 16, both
 // addresses 16-byte aligned), completing on an mbarrier (no multicast).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,

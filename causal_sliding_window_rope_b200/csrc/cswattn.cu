@@ -698,6 +698,8 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     CUtensorMap mdk, mdv;
     if ((st = make_map(&mdk, w.dk_acc, s.B * parts, s.T, s.Hk, bwd::kBN, true)) != CSWATTN_OK) return st;
     if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, true)) != CSWATTN_OK) return st;
+    CUtensorMap mdq;
+    if ((st = make_map(&mdq, w.dq_acc, s.B, s.T, s.H, bwd::kBQ, true)) != CSWATTN_OK) return st;
     static std::once_flag flag;
     static cudaError_t ferr;
     if ((st = set_smem(bwd::bwd_kernel, bwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
@@ -723,7 +725,7 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     const unsigned grid = static_cast<unsigned>(bp.nkv) * bp.parts * s.B * s.Hk;
     {
       ScopedTiming tm(CSWATTN_K_BWD, cs);
-      bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, bp);
+      bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, mdq, bp);
     }
     if ((st = launched("backward launch")) != CSWATTN_OK) return st;
   }
