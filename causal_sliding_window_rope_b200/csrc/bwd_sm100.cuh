@@ -1,4 +1,4 @@
-// bwd_sm100.cuh -- attention backward on tcgen05 tensor cores (bf16, D = 128).
+// bwd_sm100.cuh -- attention backward on tcgen05 tensor cores (bf16, D = 128 or 64).
 //
 // Gradient of the causal sliding-window attention of the page
 // "5만원으로 나만의 ChatGPT 훈련하는 방법" (section "5. 플래시 어텐션 통합",
@@ -108,6 +108,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   }
 }
 
+// HD: head_dim, 128 or 64 (a 64-wide head leaves the second column panel
+// zero: its loads are filled with zeros, its products skipped where they
+// only add zeros, its stores and reductions not issued).
+template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -278,12 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t qb = ofs(st * kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+          if (kk * 16 >= HD) break;  // zero columns of a 64-wide head
           const uint64_t okv = ofs((kk >> 2) * kKVPanel + (kk & 3) * 32);
           const uint64_t oq = ofs((kk >> 2) * kQPanel + (kk & 3) * 32);
           mma_ss(tmem + kColSP, dK_k + okv, dQ_k + qb + oq, idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+          if (kk * 16 >= HD) break;
           const uint64_t okv = ofs((kk >> 2) * kKVPanel + (kk & 3) * 32);
           const uint64_t oq = ofs((kk >> 2) * kQPanel + (kk & 3) * 32);
           mma_ss(tmem + kColSP + 64, dV_k + okv, dO_k + qb + oq, idS, kk > 0 ? 1u : 0u);
@@ -442,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int outer = part * p.B + b;  // partial slot `part` of batch b
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          if (32 * c >= HD) break;  // columns past head_dim are not stored
           tma_store_4d(&tmDV, stv + c * kF32Panel, 32 * c, hk, k0, outer);
           tma_store_4d(&tmDK, stk + c * kF32Panel, 32 * c, hk, k0, outer);
         }
@@ -493,7 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) {
         if (mbar_wait(dqs_full, n & 1, wc)) {
 #pragma unroll
-          for (int pc = 0; pc < 4; ++pc) tma_reduce_add_4d(&tmDQ, stile + pc * kDQPanel, 32 * pc, h, q0, b);
+          for (int pc = 0; pc < 4; ++pc)
+            if (32 * pc < HD) tma_reduce_add_4d(&tmDQ, stile + pc * kDQPanel, 32 * pc, h, q0, b);
           bulk_commit();
           bulk_wait_read0();
         }

@@ -73,8 +73,8 @@ cswattn_status check_layer(const cswattn_layer* L, Shape* s) {
   if (rows * L->head_dim >= (1ll << 40) || static_cast<long long>(L->B) * L->n_kv_head * 2048 >= (1ll << 31))
     return fail(CSWATTN_ERR_UNSUPPORTED, "layer too large");
   if (L->dtype == CSWATTN_BF16) {
-    if (L->head_dim != 128)
-      return fail(CSWATTN_ERR_UNSUPPORTED, "bf16 supports head_dim 128 only (got %d)", L->head_dim);
+    if (L->head_dim != 128 && L->head_dim != 64)
+      return fail(CSWATTN_ERR_UNSUPPORTED, "bf16 supports head_dim 64 and 128 (got %d)", L->head_dim);
   } else {
     const int d = L->head_dim;
     if (d != 4 && d != 8 && d != 16 && d != 32 && d != 64 && d != 128)
@@ -132,21 +132,22 @@ cswattn_status get_encoder(EncodeTiledFn* fn) {
   return CSWATTN_OK;
 }
 
-// (B, T, heads, 128) bf16 tensor; box = 64 head_dim elements x `rows` tokens
-// of one head, 128-byte swizzle; out-of-range rows read as zero.
-// Tensor map of a (outer, T, heads, 128) row-major tensor of bf16 (or
-// float32) viewed as 4-D (128, heads, T, outer); a box is one 128-byte
-// column panel (64 bf16 or 32 float32) of `rows` rows of one head, 128B-swizzled.
+// Tensor map of a (outer, T, heads, D) row-major tensor of bf16 (or
+// float32), D <= 128, viewed as 4-D (D, heads, T, outer); a box is one
+// 128-byte column panel (64 bf16 or 32 float32) of `rows` rows of one head,
+// 128B-swizzled; out-of-range rows and columns read as zero. The
+// tensor-core kernels always move 128 columns: for D = 64 the second bf16
+// panel lies past the tensor, loads fill it with zeros and stores skip it.
 cswattn_status make_map(CUtensorMap* map, const void* base, int outer, int T, int heads, int rows,
-                        bool f32 = false) {
+                        int D, bool f32 = false) {
   EncodeTiledFn enc;
   cswattn_status s = get_encoder(&enc);
   if (s != CSWATTN_OK) return s;
   const cuuint64_t es = f32 ? 4 : 2;
-  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(T),
-                              static_cast<cuuint64_t>(outer)};
-  const cuuint64_t strides[3] = {128 * es, static_cast<cuuint64_t>(heads) * 128 * es,
-                                 static_cast<cuuint64_t>(T) * heads * 128 * es};
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[3] = {D * es, static_cast<cuuint64_t>(heads) * D * es,
+                                 static_cast<cuuint64_t>(T) * heads * D * es};
   const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
@@ -225,7 +226,7 @@ cswattn_status launch_prologue(const Shape& s, const PrologueParams& pp, cudaStr
     case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
     case 16: if constexpr (sizeof(T) == 4) return CSW_ROWS(16); break;
     case 32: if constexpr (sizeof(T) == 4) return CSW_ROWS(32); break;
-    case 64: if constexpr (sizeof(T) == 4) return CSW_ROWS(64); break;
+    case 64: return CSW_ROWS(64);
     default: return CSW_ROWS(128);
   }
 #undef CSW_ROWS
@@ -242,7 +243,7 @@ cswattn_status launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t
     case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
     case 16: if constexpr (sizeof(T) == 4) return CSW_ROWS(16); break;
     case 32: if constexpr (sizeof(T) == 4) return CSW_ROWS(32); break;
-    case 64: if constexpr (sizeof(T) == 4) return CSW_ROWS(64); break;
+    case 64: return CSW_ROWS(64);
     default: return CSW_ROWS(128);
   }
 #undef CSW_ROWS
@@ -259,7 +260,7 @@ cswattn_status launch_preprocess(const Shape& s, const PreParams& pp, cudaStream
     case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
     case 16: if constexpr (sizeof(T) == 4) return CSW_ROWS(16); break;
     case 32: if constexpr (sizeof(T) == 4) return CSW_ROWS(32); break;
-    case 64: if constexpr (sizeof(T) == 4) return CSW_ROWS(64); break;
+    case 64: return CSW_ROWS(64);
     default: return CSW_ROWS(128);
   }
 #undef CSW_ROWS
@@ -575,14 +576,16 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
     return launched("fp32 forward launch");
   }
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q_out, s.B, s.T, s.H, fwd::kBM)) != CSWATTN_OK) return st;
-  if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, fwd::kBM)) != CSWATTN_OK) return st;
-  if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, fwd::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mq, q_out, s.B, s.T, s.H, fwd::kBM, s.D)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, fwd::kBM, s.D)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, fwd::kBM, s.D)) != CSWATTN_OK) return st;
   CUtensorMap mo;
-  if ((st = make_map(&mo, O, s.B, s.T, s.H, fwd::kBM)) != CSWATTN_OK) return st;
-  static std::once_flag flag;
-  static cudaError_t ferr;
-  if ((st = set_smem(fwd::fwd_kernel, fwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mo, O, s.B, s.T, s.H, fwd::kBM, s.D)) != CSWATTN_OK) return st;
+  static std::once_flag flag128, flag64;
+  static cudaError_t ferr128, ferr64;
+  if ((st = s.D == 64 ? set_smem(fwd::fwd_kernel<64>, fwd::kSmemBytes, flag64, ferr64)
+                      : set_smem(fwd::fwd_kernel<128>, fwd::kSmemBytes, flag128, ferr128)) != CSWATTN_OK)
+    return st;
   fwd::Params fp;
   fp.B = s.B;
   fp.T = s.T;
@@ -599,7 +602,10 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
   const unsigned grid = static_cast<unsigned>(fp.npairs) * s.B * s.Hk;
   {
     ScopedTiming tm(CSWATTN_K_FWD, cs);
-    fwd::fwd_kernel<<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, mo, fp);
+    if (s.D == 64)
+      fwd::fwd_kernel<64><<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, mo, fp);
+    else
+      fwd::fwd_kernel<128><<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, mo, fp);
   }
   return launched("forward launch");
 }
@@ -690,19 +696,21 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     if ((st = launched("fp32 backward launch")) != CSWATTN_OK) return st;
   } else {
     CUtensorMap mq, mdo, mk, mv;
-    if ((st = make_map(&mq, q_out, s.B, s.T, s.H, bwd::kBQ)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mdo, dO, s.B, s.T, s.H, bwd::kBQ)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, bwd::kBN)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, bwd::kBN)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mq, q_out, s.B, s.T, s.H, bwd::kBQ, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdo, dO, s.B, s.T, s.H, bwd::kBQ, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, bwd::kBN, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, bwd::kBN, s.D)) != CSWATTN_OK) return st;
     const int parts = bwd_parts(s);
     CUtensorMap mdk, mdv;
-    if ((st = make_map(&mdk, w.dk_acc, s.B * parts, s.T, s.Hk, bwd::kBN, true)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, true)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdk, w.dk_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
     CUtensorMap mdq;
-    if ((st = make_map(&mdq, w.dq_acc, s.B, s.T, s.H, bwd::kBQ, true)) != CSWATTN_OK) return st;
-    static std::once_flag flag;
-    static cudaError_t ferr;
-    if ((st = set_smem(bwd::bwd_kernel, bwd::kSmemBytes, flag, ferr)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdq, w.dq_acc, s.B, s.T, s.H, bwd::kBQ, s.D, true)) != CSWATTN_OK) return st;
+    static std::once_flag flag128, flag64;
+    static cudaError_t ferr128, ferr64;
+    if ((st = s.D == 64 ? set_smem(bwd::bwd_kernel<64>, bwd::kSmemBytes, flag64, ferr64)
+                        : set_smem(bwd::bwd_kernel<128>, bwd::kSmemBytes, flag128, ferr128)) != CSWATTN_OK)
+      return st;
     bwd::Params bp;
     bp.B = s.B;
     bp.T = s.T;
@@ -725,7 +733,10 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     const unsigned grid = static_cast<unsigned>(bp.nkv) * bp.parts * s.B * s.Hk;
     {
       ScopedTiming tm(CSWATTN_K_BWD, cs);
-      bwd::bwd_kernel<<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, mdq, bp);
+      if (s.D == 64)
+        bwd::bwd_kernel<64><<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, mdq, bp);
+      else
+        bwd::bwd_kernel<128><<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, mdq, bp);
     }
     if ((st = launched("backward launch")) != CSWATTN_OK) return st;
   }

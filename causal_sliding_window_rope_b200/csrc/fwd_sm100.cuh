@@ -1,4 +1,4 @@
-// fwd_sm100.cuh -- attention forward on tcgen05 tensor cores (bf16, D = 128).
+// fwd_sm100.cuh -- attention forward on tcgen05 tensor cores (bf16, D = 128 or 64).
 //
 // Computes O_i = sum_j softmax_j(c q~_i . k~_j) v_eff_j over the causal
 // sliding window (i - W < j <= i) and the row log-sum-exp, the attention
@@ -78,6 +78,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   }
 }
 
+// HD: head_dim, 128 or 64 (a 64-wide head leaves the second column panel
+// zero: its loads are filled with zeros, its products skipped, its stores
+// not issued).
+template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -224,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(X) * 128u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+          if (kk * 16 >= HD) break;  // zero columns of a 64-wide head
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
           mma_ss(d_tmem, qd + off, kd + off, idS, kk > 0 ? 1u : 0u);
         }
@@ -312,19 +317,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (kj > qi || qi - kj >= p.W) sv[c][i] = __float_as_uint(-INFINITY);
             }
         }
-        // Row max as a tree (8 independent chains, then combine).
-        float mp[8];
+        // Row max: one chain of three-input maxima per 32-column chunk.
+        float mp[4];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) mp[t] = __uint_as_float(sv[t >> 1][(t & 1) * 16]);
+        for (int c = 0; c < 4; ++c) {
+          float m = fmax3(__uint_as_float(sv[c][0]), __uint_as_float(sv[c][1]), __uint_as_float(sv[c][2]));
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i != 0 && i != 16)
-              mp[c * 2 + (i >> 4)] = fmaxf(mp[c * 2 + (i >> 4)], __uint_as_float(sv[c][i]));
-#pragma unroll
-        for (int t = 0; t < 4; ++t) mp[t] = fmaxf(mp[t], mp[t + 4]);
-        float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])) * c2;
+          for (int i = 3; i < 31; i += 2) m = fmax3(m, __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
+          mp[c] = fmaxf(m, __uint_as_float(sv[c][31]));
+        }
+        float mx = fmax3(mp[0], mp[1], fmaxf(mp[2], mp[3])) * c2;
         float alpha = 1.f;
         bool rescale = false;
         if (n == 0) {
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&o_staged[X]);
         if (r == 0 && mbar_wait(&o_staged[X], 0, wc)) {
           tma_store_4d(&tmO, ot, 0, head[X], q0, b);
-          tma_store_4d(&tmO, ot + kPanelBytes, 64, head[X], q0, b);
+          if (HD > 64) tma_store_4d(&tmO, ot + kPanelBytes, 64, head[X], q0, b);
           bulk_commit();
           bulk_wait0();
         }

@@ -64,9 +64,11 @@ typedef enum {
 
 typedef enum { CSWATTN_F32 = 0, CSWATTN_BF16 = 1 } cswattn_dtype;
 
-/* Shape of one attention layer. Supported: bf16 with head_dim 128 (tensor
- * cores), f32 with head_dim in {4, 8, 16, 32, 64, 128} (CUDA cores, fp32
- * throughout). n_head % n_kv_head == 0, window >= 1, T <= 2^20. */
+/* Shape of one attention layer. Supported: bf16 with head_dim 64 or 128
+ * (tensor cores; a 64-wide head runs the 128-wide tiles with its second half
+ * zero), f32 with head_dim in {4, 8, 16, 32, 64, 128} (CUDA cores, fp32
+ * throughout). Anything else returns CSWATTN_ERR_UNSUPPORTED.
+ * n_head % n_kv_head == 0, window >= 1, T <= 2^20. */
 typedef struct {
   int B, T, n_head, n_kv_head, head_dim;
   int window;          /* keys visible to a query, itself included */
@@ -96,7 +98,7 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
                         const void* v_out, void* O, float* lse, void* stream);
 
 /* Bytes of device scratch attn_bwd needs for this layer: float32
- * accumulators of dq_out (B, n_head, T, head_dim), P partial sums each of
+ * accumulators of dq_out (B, T, n_head, head_dim), P partial sums each of
  * dk_out and dv_out (B, T, n_kv_head, head_dim) (P = 1..8, the number of
  * CTAs the bf16 backward splits a key tile's work into; 1 for f32), and two
  * row terms (dO.O and lse*log2(e)),

@@ -55,7 +55,8 @@ def call_fwd(spec, ptrs=(16, 32, 48, 64, 80)):
     (dict(rope_base=float("inf")), cs.ERR_INVALID_ARG),
     (dict(eps=-1.0), cs.ERR_INVALID_ARG),
     (dict(softmax_scale=-0.5), cs.ERR_INVALID_ARG),
-    (dict(head_dim=64), cs.ERR_UNSUPPORTED),
+    (dict(head_dim=32), cs.ERR_UNSUPPORTED),
+    (dict(head_dim=96), cs.ERR_UNSUPPORTED),
     (dict(head_dim=6, dtype="f32"), cs.ERR_UNSUPPORTED),
     (dict(T=(1 << 20) + 1), cs.ERR_UNSUPPORTED),
 ])
@@ -68,6 +69,16 @@ def test_layer_validation(lib, change, code):
     assert lib.attn_fwd(ctypes.byref(layer), 16, 32, 48, 64, 80, None) == code
     assert lib.cswattn_last_error().decode() != ""
     assert lib.attn_bwd_workspace_bytes(ctypes.byref(layer)) == 0
+
+
+@pytest.mark.parametrize("D,dtype", [(64, "bf16"), (128, "bf16"), (4, "f32"), (64, "f32")])
+def test_supported_head_dims_pass_validation(lib, D, dtype):
+    # A supported shape fails only on its (deliberately misaligned) pointers.
+    spec = cs.LayerSpec(2, 64, 4, 2, D, 32, dtype=dtype)
+    layer = spec.c()
+    assert lib.attn_bwd_workspace_bytes(ctypes.byref(layer)) > 0
+    assert lib.attn_fwd(ctypes.byref(layer), 16 + 8, 32, 48, 64, 80, None) == cs.ERR_INVALID_ARG
+    assert b"aligned" in lib.cswattn_last_error()
 
 
 def test_bad_dtype_and_null_layer(lib):

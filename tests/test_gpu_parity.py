@@ -70,6 +70,23 @@ def test_bf16_layer_matches_oracle(B, T, H, Hk, W, has_ve):
     check_bf16(spec, got, ref)
 
 
+BF16_D64_CASES = [
+    # B, T, H, Hk, W, has_ve: head_dim 64 (second column panel zero-filled)
+    (1, 200, 4, 2, 100, True),
+    (2, 129, 2, 2, 129, False),
+    (1, 333, 6, 2, 64, True),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hk,W,has_ve", BF16_D64_CASES)
+def test_bf16_head_dim_64_matches_oracle(B, T, H, Hk, W, has_ve):
+    spec = cs.LayerSpec(B, T, H, Hk, 64, W, has_ve=has_ve, dtype="bf16")
+    inp = make_inputs(B, T, H, Hk, 64, has_ve, "bf16", config=91, layer=T % 5)
+    got, _ = run_gpu(spec, inp)
+    _, ref = oracle_layer(spec, inp)
+    check_bf16(spec, got, ref)
+
+
 F32_CASES = [
     (32, 16, 4, 4, 4, 16, False),   # the microgpt-sized layer
     (2, 40, 4, 2, 8, 7, True),
