@@ -68,6 +68,7 @@ def _get():
         _lib.oracle_prologue_bwd.argtypes = [L] + [dp] * 12
         _lib.oracle_probs_row.argtypes = [L, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp]
         _lib.oracle_probs_row.restype = ctypes.c_double
+        _lib.oracle_decode.argtypes = [L] + [dp] * 5 + [ip] + [dp] * 4
     return _lib
 
 
@@ -219,3 +220,26 @@ def layer(L: Layer, q, k, v, ve, gate, dO):
     dq, dk, dv, dve, dgate = prologue_bwd(L, q, k, ve, gate, dqt, dkt, dveff)
     return dict(qt=qt, kt=kt, veff=veff, rstd_q=rq, rstd_k=rk, O=O, lse=lse,
                 dqt=dqt, dkt=dkt, dveff=dveff, dq=dq, dk=dk, dv=dv, dve=dve, dgate=dgate)
+
+
+def decode(L: Layer, q, k, v, ve, gate, lens, kcache, vcache):
+    """One decode step with a KV cache (L.T = cache capacity). q (B,H,D);
+    k, v, ve (B,Hk,D); gate (B,Hk); lens (B,) tokens already cached; the
+    caches (B,T,Hk,D) hold k~ and v_eff rows. Returns (O (B,H,D), lse (B,H),
+    kcache', vcache') with the new token's rows written at position lens[b]."""
+    if L.has_ve and (ve is None or gate is None):
+        raise ValueError("layer has a value embedding: ve and gate are required")
+    B, H, Hk, D = L.B, L.H, L.Hk, L.D
+    q, k, v = _f64(q, (B, H, D)), _f64(k, (B, Hk, D)), _f64(v, (B, Hk, D))
+    ve = _f64(ve, (B, Hk, D)) if L.has_ve else np.zeros((B, Hk, D))
+    gate = _f64(gate, (B, Hk)) if L.has_ve else np.zeros((B, Hk))
+    lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(B))
+    if (lens < 0).any() or (lens >= L.T).any():
+        raise ValueError("cache lengths must lie in [0, T)")
+    kc = _f64(kcache, (B, L.T, Hk, D)).copy()
+    vc = _f64(vcache, (B, L.T, Hk, D)).copy()
+    O = np.zeros((B, H, D))
+    lse = np.zeros((B, H))
+    _get().oracle_decode(L.c(), _p(q), _p(k), _p(v), _p(ve), _p(gate),
+                         lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), _p(kc), _p(vc), _p(O), _p(lse))
+    return O, lse, kc, vc

@@ -379,3 +379,67 @@ void oracle_prologue_bwd(const oracle_layer *L, const double *q,
       }
     }
 }
+
+/* Decode step with a key/value cache: page section "6. 추론 엔진
+ * (nanochat/engine.py)", generation with a pre-filled KV cache
+ * (flash_attn_with_kvcache). L->T is the cache capacity. Sequence b already
+ * holds len[b] tokens: rows 0..len[b]-1 of kc (k~) and vc (v_eff), layout
+ * (B, T, Hk, D). Its new token sits at position p = len[b] (< T): the
+ * prologue is applied to it at position p, its k~ and v_eff rows are written
+ * to the caches at row p, and its query rows attend over cache rows
+ * (p - W, p]. q (B, H, D); k, v, ve (B, Hk, D); gate (B, Hk). Outputs
+ * O (B, H, D) and lse (B, H), natural log. */
+void oracle_decode(const oracle_layer *L, const double *q, const double *k,
+                   const double *v, const double *ve, const double *gate,
+                   const int *len, double *kc, double *vc, double *O,
+                   double *lse) {
+  const int B = L->B, T = L->T, H = L->H, Hk = L->Hk, D = L->D;
+  const int no_norm = (L->flags & ORACLE_NO_NORM) != 0;
+  const int no_rope = (L->flags & ORACLE_NO_ROPE) != 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int b = 0; b < B; ++b) {
+    const int p = len[b];
+    const double pos = (double)(p + L->pos_offset);
+    double n[1024];
+    double *qt = (double *)malloc(sizeof(double) * (size_t)H * D);
+    double *s = (double *)malloc(sizeof(double) * (size_t)T);
+    for (int h = 0; h < H; ++h) {
+      rms_norm_row(q + ((size_t)b * H + h) * D, n, D, L->eps, no_norm);
+      rope_row(n, qt + (size_t)h * D, D, pos, L->rope_base, 0, no_rope);
+    }
+    for (int h = 0; h < Hk; ++h) {
+      const size_t o = ((size_t)b * Hk + h) * D;
+      const size_t c = idx4(b, p, h, 0, T, Hk, D);
+      rms_norm_row(k + o, n, D, L->eps, no_norm);
+      rope_row(n, kc + c, D, pos, L->rope_base, 0, no_rope);
+      double coef = L->has_ve ? 3.0 * sigmoid(gate[(size_t)b * Hk + h]) : 0.0;
+      for (int d = 0; d < D; ++d) vc[c + d] = v[o + d] + (L->has_ve ? coef * ve[o + d] : 0.0);
+    }
+    const int lo = first_key(L, p);
+    for (int h = 0; h < H; ++h) {
+      const int hk = kv_head(L, h);
+      const double *qh = qt + (size_t)h * D;
+      double m = -INFINITY;
+      for (int j = lo; j <= p; ++j) {
+        const double *kj = kc + idx4(b, j, hk, 0, T, Hk, D);
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += qh[d] * kj[d];
+        s[j] = L->scale * dot;
+        if (s[j] > m) m = s[j];
+      }
+      double sum = 0.0;
+      for (int j = lo; j <= p; ++j) sum += exp(s[j] - m);
+      const double l = m + log(sum);
+      double *o = O + ((size_t)b * H + h) * D;
+      for (int d = 0; d < D; ++d) o[d] = 0.0;
+      for (int j = lo; j <= p; ++j) {
+        const double pj = exp(s[j] - l);
+        const double *vj = vc + idx4(b, j, hk, 0, T, Hk, D);
+        for (int d = 0; d < D; ++d) o[d] += pj * vj[d];
+      }
+      lse[(size_t)b * H + h] = l;
+    }
+    free(s);
+    free(qt);
+  }
+}

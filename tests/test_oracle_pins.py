@@ -301,3 +301,57 @@ def test_oracle_regression_fixture():
     for key, val in g["checksums"].items():
         assert abs(float(np.sum(r[key] * np.cos(np.arange(r[key].size)).reshape(r[key].shape))) - val) \
             <= 1e-9 * max(1.0, abs(val)), key
+
+
+# ---------------------------------------------------------------- decode with a KV cache
+
+def decode_case(L, lens, seed):
+    """Raw projections for all T positions, the full-sequence oracle, and the
+    decode inputs: caches holding the prologue rows of each sequence's first
+    lens[b] tokens (later rows NaN, so reading them would show), and the raw
+    projections of token lens[b]."""
+    q, k, v, ve, gate, _ = inputs(L, seed)
+    qt, kt, veff, _, _ = oracle.prologue(L, q, k, v, ve if L.has_ve else None, gate if L.has_ve else None)
+    O, lse = oracle.attn_fwd(L, qt, kt, veff)
+    kc = np.full_like(kt, np.nan)
+    vc = np.full_like(veff, np.nan)
+    B = L.B
+    tok = {n: np.stack([a[b, lens[b]] for b in range(B)]) for n, a in
+           (("q", q), ("k", k), ("v", v), ("ve", ve), ("gate", gate))}
+    for b in range(B):
+        kc[b, :lens[b]] = kt[b, :lens[b]]
+        vc[b, :lens[b]] = veff[b, :lens[b]]
+    return tok, kc, vc, (qt, kt, veff, O, lse)
+
+
+@pytest.mark.parametrize("W,H,Hk,has_ve", [(5, 4, 2, True), (40, 3, 1, False), (1, 2, 2, True),
+                                          (7, 6, 2, True)])
+def test_decode_equals_last_row_of_full_forward(W, H, Hk, has_ve):
+    """A decode step over a cache filled with the prologue rows of the first p
+    tokens is row p of the full-sequence forward (causality: row p reads no
+    later key), and the rows it writes are the prologue rows of token p."""
+    L = oracle.Layer(3, 24, H, Hk, 8, W, has_ve=has_ve)
+    lens = [0, 11, 23]
+    tok, kc, vc, (qt, kt, veff, O, lse) = decode_case(L, lens, seed=W + 10 * H)
+    Od, lsed, kc2, vc2 = oracle.decode(L, tok["q"], tok["k"], tok["v"], tok["ve"], tok["gate"],
+                                       lens, kc, vc)
+    for b, p in enumerate(lens):
+        np.testing.assert_allclose(Od[b], O[b, p], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lsed[b], lse[b, :, p], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(kc2[b, p], kt[b, p], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(vc2[b, p], veff[b, p], rtol=0, atol=1e-13)
+        assert np.isnan(kc2[b, p + 1:]).all() and np.isnan(vc2[b, p + 1:]).all()
+
+
+def test_decode_window_one_returns_own_value():
+    """W = 1: the new token sees only itself, so O = v_eff of the token and
+    lse = c q~ . k~ of the token."""
+    L = oracle.Layer(2, 10, 4, 2, 6, 1, has_ve=True)
+    lens = [3, 9]
+    tok, kc, vc, (qt, kt, veff, _, _) = decode_case(L, lens, seed=5)
+    Od, lsed, _, _ = oracle.decode(L, tok["q"], tok["k"], tok["v"], tok["ve"], tok["gate"], lens, kc, vc)
+    for b, p in enumerate(lens):
+        for h in range(L.H):
+            hk = h // (L.H // L.Hk)
+            np.testing.assert_allclose(Od[b, h], veff[b, p, hk], rtol=0, atol=1e-12)
+            assert abs(lsed[b, h] - L.scale * float(qt[b, p, h] @ kt[b, p, hk])) < 1e-12
