@@ -326,12 +326,82 @@ def run_ours(args):
                     "ms_per_step": round(e2e_ms / e2e_steps, 3)},
             "clocks": clk,
         }
+        if world == 1 and not args.no_decode and args.single_layer is None:
+            line["decode"] = decode_bench(w, dev, peaks, steps=args.steps, warmup=args.warmup)
         if world == 1 and not args.no_cpu_baseline and args.single_layer is None:
             line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+DECODE_BATCH = 32  # sequences generating together
+
+
+def decode_bench(w, dev, peaks, steps=20, warmup=5):
+    """One generation step over the workload's layer stack with a KV cache
+    (attn_decode per layer): DECODE_BATCH sequences whose caches hold T-1
+    tokens, so every layer reads its full window of K and V. HBM-bound: the
+    roofline is the window's K/V bytes per step over the step's device time
+    (the caches, 0.5 GB, exceed L2)."""
+    import torch
+
+    import causal_sliding_window_rope_b200 as cs
+    B, T, H, Hk, D = DECODE_BATCH, w.T, w.H, w.Hk, w.D
+    g = torch.Generator().manual_seed(4321)
+
+    def rnd(*shape):
+        return torch.randn(*shape, generator=g).to(torch.bfloat16).to(dev)
+
+    layers = []
+    for W, ve in zip(w.windows, w.ve):
+        spec = cs.LayerSpec(B, T, H, Hk, D, W, has_ve=ve, dtype="bf16", rope_base=w.rope_base, eps=w.eps)
+        layers.append(dict(
+            spec=spec, q=rnd(B, H, D), k=rnd(B, Hk, D), v=rnd(B, Hk, D),
+            ve=rnd(B, Hk, D) if ve else None, gate=rnd(B, Hk) if ve else None,
+            kc=rnd(B, T, Hk, D), vc=rnd(B, T, Hk, D),
+            O=torch.empty(B, H, D, dtype=torch.bfloat16, device=dev),
+            lse=torch.empty(B, H, dtype=torch.float32, device=dev),
+            ws=torch.empty(cs.attn_decode_workspace_bytes(spec), dtype=torch.uint8, device=dev)))
+    lens = torch.full((B,), T - 1, dtype=torch.int32, device=dev)
+
+    def step():
+        for x in layers:
+            cs.attn_decode(x["spec"], x["q"], x["k"], x["v"], x["ve"], x["gate"], lens, x["kc"],
+                           x["vc"], x["O"], x["lse"], x["ws"])
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    cs.cswattn_sync_status()
+    stream = torch.cuda.current_stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    cs.cswattn_set_timing(True)
+    cs.cswattn_kernel_times()
+    for a, b in evs:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    kt = cs.cswattn_kernel_times()
+    cs.cswattn_set_timing(False)
+    cs.cswattn_sync_status()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    # algorithmic bytes: the window's K and V rows, the new token's inputs and
+    # outputs, the row written back to each cache
+    kv = sum(B * Hk * min(W, T) * D * 2 * 2 for W in w.windows)
+    small = len(layers) * B * ((H + 3 * Hk) * D * 2 + H * D * 2 + H * 4 + 2 * Hk * D * 2)
+    nbytes = kv + small
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": f"one decode step of the layer stack, {B} sequences, caches of {T} rows "
+                        f"holding {T - 1} tokens, windows {w.windows}",
+            "ms_per_step": round(ms, 4), "tokens_per_s": round(B / (ms * 1e-3), 1),
+            "kernel_ms_per_step": round(kt["decode"][0] / steps, 4),
+            "launches_per_step": kt["decode"][1] // steps * 3,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": nbytes,
+                         "peak_source": "measured hbm_gbs"}}
 
 
 def traffic_for(kind):
@@ -455,6 +525,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--single-layer", type=int, default=None,
                     help="profiling case: time only this layer of the stack (no e2e, no CPU leg)")

@@ -26,10 +26,11 @@ F32, BF16 = 0, 1
 
 # Every symbol the header declares; the CPU tests check the library exports them.
 EXPORTS = ("attn_prologue", "attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
+           "attn_decode_workspace_bytes", "attn_decode",
            "cswattn_sync_status", "cswattn_set_wait_limit_ns", "cswattn_set_timing",
            "cswattn_kernel_times", "cswattn_selftest_wait_timeout", "cswattn_last_error",
            "cswattn_version")
-KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi")
+KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi", "decode")
 
 
 class CswattnLayer(ctypes.Structure):
@@ -77,6 +78,9 @@ def lib():
         L.cswattn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
         L.cswattn_selftest_wait_timeout.restype = ctypes.c_int
         L.attn_bwd_noalloc.argtypes = [lp] + [vp] * 7 + [fp, fp, vp, fp, vp] + [vp] * 5 + [vp]
+        L.attn_decode_workspace_bytes.argtypes = [lp]
+        L.attn_decode_workspace_bytes.restype = sz
+        L.attn_decode.argtypes = [lp] + [vp] * 5 + [vp, vp, vp, vp, fp, vp, sz, vp]
         for name in ("attn_prologue", "attn_fwd", "attn_bwd", "attn_bwd_noalloc",
                      "cswattn_sync_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -174,6 +178,25 @@ def attn_bwd_noalloc(spec: LayerSpec, q, k, ve, gate, q_out, k_out, v_out, rstd_
                                   _ptr(q_out), _ptr(k_out), _ptr(v_out), _ptr(rstd_q),
                                   _ptr(rstd_k), _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
                                   _ptr(dV), _ptr(dve), _ptr(dgate), _stream(stream)))
+
+
+def attn_decode_workspace_bytes(spec: LayerSpec) -> int:
+    """Scratch bytes of attn_decode; spec.T is the cache capacity."""
+    layer = spec.c()
+    return int(lib().attn_decode_workspace_bytes(ctypes.byref(layer)))
+
+
+def attn_decode(spec: LayerSpec, q, k, v, ve, gate, cache_len, k_cache, v_cache, O, lse,
+                workspace, workspace_bytes=None, stream=None):
+    """One decode step with a KV cache (spec.T = cache capacity, cache_len an
+    int32 device tensor of B lengths): writes the new token's k~ / v_eff rows
+    into the caches and its attention output O (B,H,D) and lse (B,H)."""
+    layer = spec.c()
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().attn_decode(ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate),
+                             _ptr(cache_len), _ptr(k_cache), _ptr(v_cache), _ptr(O), _ptr(lse),
+                             _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def cswattn_sync_status(stream=None):

@@ -69,9 +69,9 @@ constexpr int kSmemBytes = kOffRow + kQStages * 2 * kBQ * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 // Register budgets after setmaxnreg (launch: 384 threads x 168 registers).
-constexpr int kRegLo = 96;   // producer / MMA warpgroup
+constexpr int kRegLo = 88;   // producer / MMA warpgroup
 constexpr int kRegSm = 248;  // softmax warpgroup (S^T, dP^T rows + packed P, dS)
-constexpr int kRegDq = 160;  // dQ drain warpgroup
+constexpr int kRegDq = 168;  // dQ drain warpgroup
 static_assert(128 * (kRegLo + kRegSm + kRegDq) <= kThreads * 168, "register budget");
 
 constexpr uint32_t kColSP = 0u;  // S^T at +0, dP^T at +64
@@ -94,10 +94,6 @@ struct Params {
   unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long ns) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
@@ -118,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                const __grid_constant__ CUtensorMap tmDQ, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;      // [kQStages]

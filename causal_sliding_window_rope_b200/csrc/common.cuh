@@ -23,6 +23,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// First 1024-byte aligned address of a dynamic shared-memory array. The
+// result is the array pointer plus an offset, so the compiler still knows it
+// points into shared memory (a round trip through an integer would turn
+// every access through it into a generic one).
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* smem_raw) {
+  return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

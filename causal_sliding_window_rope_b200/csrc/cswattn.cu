@@ -18,6 +18,7 @@
 #include "bwd_aux.cuh"
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
+#include "decode.cuh"
 
 using namespace cswattn;
 
@@ -442,6 +443,55 @@ cswattn_status noalloc_scratch(void** out) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- decode
+
+struct DecodeWorkspace {
+  float *qt, *part_ml, *part_o;
+  int nsplit;
+  size_t bytes;
+};
+
+DecodeWorkspace carve_decode(const Shape& s, void* base) {
+  DecodeWorkspace w;
+  w.nsplit = dec::decode_splits(s.T, s.W);
+  const size_t rows = static_cast<size_t>(s.B) * s.H;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  w.qt = reinterpret_cast<float*>(p + off);
+  off += pad256(rows * s.D * 4);
+  w.part_ml = reinterpret_cast<float*>(p + off);
+  off += pad256(rows * w.nsplit * 2 * 4);
+  w.part_o = reinterpret_cast<float*>(p + off);
+  off += pad256(rows * w.nsplit * s.D * 4);
+  w.bytes = off;
+  return w;
+}
+
+cswattn_status check_decode_layer(const cswattn_layer* layer, Shape* s) {
+  cswattn_status st = check_layer(layer, s);
+  if (st != CSWATTN_OK) return st;
+  if (!s->bf16) return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports bf16 layers only");
+  if (s->g > dec::kMaxGroup)
+    return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports up to %d query heads per KV head (got %d)",
+                dec::kMaxGroup, s->g);
+  return CSWATTN_OK;
+}
+
+template <int D>
+cswattn_status launch_decode(const Shape& s, const dec::PrologueParams& pp, const CUtensorMap& mk,
+                             const CUtensorMap& mv, const dec::AttnParams& ap, const dec::CombineParams& cp,
+                             cudaStream_t st) {
+  constexpr int kSmem = dec::decode_attn_smem<D>();
+  static std::once_flag flag;
+  static cudaError_t ferr;
+  cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem, flag, ferr);
+  if (e != CSWATTN_OK) return e;
+  dec::decode_prologue_kernel<D><<<s.B, dec::kThreads, 0, st>>>(pp);
+  dec::decode_attn_kernel<D><<<dim3(ap.nsplit, s.Hk, s.B), dec::kThreads, kSmem, st>>>(mk, mv, ap);
+  dec::decode_combine_kernel<D><<<s.B * s.H, D, 0, st>>>(cp);
+  return CSWATTN_OK;
+}
+
 extern "C" {
 
 int cswattn_version(void) { return (1 << 16) | 0; }
@@ -493,6 +543,8 @@ cswattn_status cswattn_sync_status(void* stream) {
     e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
     if (v & kStatusTimeout) return fail(CSWATTN_ERR_TIMEOUT, "a device-side wait ran out (status 0x%x)", v);
+    if (v & kStatusRange)
+      return fail(CSWATTN_ERR_INVALID_ARG, "a decode step met a cache length outside [0, T) (status 0x%x)", v);
   }
   return CSWATTN_OK;
 }
@@ -770,6 +822,89 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   }
   if (st != CSWATTN_OK) return st;
   return launched("epilogue launch");
+}
+
+size_t attn_decode_workspace_bytes(const cswattn_layer* layer) {
+  Shape s;
+  if (check_decode_layer(layer, &s) != CSWATTN_OK) return 0;
+  return carve_decode(s, nullptr).bytes;
+}
+
+cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void* k, const void* v,
+                           const void* ve, const void* gate, const int* cache_len, void* k_cache,
+                           void* v_cache, void* O, float* lse, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  Shape s;
+  cswattn_status st = check_decode_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(k, 16);
+  CHECK_PTR(v, 16);
+  CHECK_PTR(cache_len, 4);
+  CHECK_PTR(k_cache, 16);
+  CHECK_PTR(v_cache, 16);
+  CHECK_PTR(O, 16);
+  CHECK_PTR(lse, 4);
+  CHECK_PTR(workspace, 256);
+  if (layer->has_ve) {
+    CHECK_PTR(ve, 16);
+    CHECK_PTR(gate, 2);
+  }
+  if (k_cache == v_cache) return fail(CSWATTN_ERR_INVALID_ARG, "k_cache and v_cache must differ");
+  const DecodeWorkspace w = carve_decode(s, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CSWATTN_ERR_INVALID_ARG, "decode workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
+  CUtensorMap mk, mv;
+  if ((st = make_map(&mk, k_cache, s.B, s.T, s.Hk, dec::kChunk, s.D)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mv, v_cache, s.B, s.T, s.Hk, dec::kChunk, s.D)) != CSWATTN_OK) return st;
+  dec::PrologueParams pp;
+  pp.B = s.B;
+  pp.T = s.T;
+  pp.H = s.H;
+  pp.Hk = s.Hk;
+  pp.has_ve = layer->has_ve;
+  pp.eps = layer->eps;
+  fill_omega(pp.omega, s.D, layer->rope_base);
+  pp.len = cache_len;
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.ve = static_cast<const __nv_bfloat16*>(ve);
+  pp.gate = static_cast<const __nv_bfloat16*>(gate);
+  pp.kc = static_cast<__nv_bfloat16*>(k_cache);
+  pp.vc = static_cast<__nv_bfloat16*>(v_cache);
+  pp.qt = w.qt;
+  dec::AttnParams ap;
+  ap.B = s.B;
+  ap.T = s.T;
+  ap.H = s.H;
+  ap.Hk = s.Hk;
+  ap.W = s.W;
+  ap.g = s.g;
+  ap.nsplit = w.nsplit;
+  ap.scale_log2 = s.scale * 1.4426950408889634f;
+  ap.len = cache_len;
+  ap.qt = w.qt;
+  ap.part_ml = w.part_ml;
+  ap.part_o = w.part_o;
+  ap.wait_ns = g_wait_ns.load();
+  dec::CombineParams cp;
+  cp.B = s.B;
+  cp.H = s.H;
+  cp.nsplit = w.nsplit;
+  cp.len = cache_len;
+  cp.T = s.T;
+  cp.part_ml = w.part_ml;
+  cp.part_o = w.part_o;
+  cp.O = static_cast<__nv_bfloat16*>(O);
+  cp.lse = lse;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  {
+    ScopedTiming tm(CSWATTN_K_DECODE, cs);
+    st = s.D == 64 ? launch_decode<64>(s, pp, mk, mv, ap, cp, cs) : launch_decode<128>(s, pp, mk, mv, ap, cp, cs);
+  }
+  if (st != CSWATTN_OK) return st;
+  return launched("decode launch");
 }
 
 cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const void* k,

@@ -62,10 +62,6 @@ struct Params {
   unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
 // Waits for a phase without looking at the abort flag (used to drain
 // in-flight copies and MMAs before the CTA exits). Bounded by `ns`.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long ns) {
@@ -87,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
+  uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [kSlots]

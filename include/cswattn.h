@@ -159,9 +159,42 @@ cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const
                                 const void* dO, void* dQ, void* dK, void* dV, void* dve,
                                 void* dgate, void* stream);
 
+/* Bytes of device scratch attn_decode needs for this layer (layer->T is the
+ * cache capacity): float32 q~ (B, n_head, head_dim) and, per query head, the
+ * partial results of the split-KV chunks (max, sum and head_dim partial
+ * outputs per chunk), each part padded to 256 bytes. 0 for an invalid or
+ * unsupported layer. */
+size_t attn_decode_workspace_bytes(const cswattn_layer* layer);
+
+/* Decode step with a key/value cache: page section "6. 추론 엔진
+ * (nanochat/engine.py)" (generation over a pre-filled KV cache,
+ * flash_attn_with_kvcache), one new token per sequence.
+ * layer: bf16, head_dim 64 or 128, n_head / n_kv_head <= 16; T is the cache
+ * capacity (rows per sequence), window as in attn_fwd.
+ * cache_len (device int32, B): tokens already in sequence b's cache; the
+ * new token's position is p = cache_len[b], which must lie in [0, T) (a
+ * value outside is not checked on the host: the sequence is left untouched
+ * and the next cswattn_sync_status() returns CSWATTN_ERR_INVALID_ARG).
+ * q (B, n_head, head_dim), k, v, ve (B, n_kv_head, head_dim), gate
+ * (B, n_kv_head): the new token's projections, as for attn_prologue with
+ * T = 1; ve and gate only when has_ve.
+ * k_cache, v_cache (B, T, n_kv_head, head_dim): rows 0..p-1 hold the k~ and
+ * v_eff rows of earlier tokens (prologue outputs). The call writes row p of
+ * both (k~ = RoPE_p(RMSNorm(k)), v_eff = v + 3*sigmoid(gate)*ve); it does
+ * not change cache_len (the caller advances it).
+ * O (B, n_head, head_dim), lse (B, n_head), natural log: attention of
+ * q~ = RoPE_p(RMSNorm(q)) over cache rows (p - window, p].
+ * workspace: caller-owned device scratch of at least
+ * attn_decode_workspace_bytes(layer) bytes, 256-byte aligned. */
+cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void* k,
+                           const void* v, const void* ve, const void* gate, const int* cache_len,
+                           void* k_cache, void* v_cache, void* O, float* lse, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the
  * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
- * since the last check, CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
+ * since the last check, CSWATTN_ERR_INVALID_ARG if a decode step met a cache
+ * length outside [0, T), CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
 cswattn_status cswattn_sync_status(void* stream);
 
 /* Self-test of the bounded-wait path: launches one small kernel whose thread
@@ -183,7 +216,8 @@ enum {
   CSWATTN_K_BWD_PRE = 2,  /* backward row terms Delta = rowsum(dO * O) */
   CSWATTN_K_BWD = 3,      /* attention backward main kernel(s) */
   CSWATTN_K_BWD_EPI = 4,  /* backward epilogue: RoPE^-1, RMSNorm', dv/dve/dgate */
-  CSWATTN_NUM_KERNELS = 5
+  CSWATTN_K_DECODE = 5,   /* decode step: new-token prologue, split-KV attention, combine */
+  CSWATTN_NUM_KERNELS = 6
 };
 
 /* Per-kernel device timing for measurement tools. With enable != 0, every

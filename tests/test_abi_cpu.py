@@ -122,3 +122,25 @@ def test_workspace_size_and_check(lib):
     st = lib.attn_bwd(layer, *ptrs[:12], *ptrs[12:17], 256 * 40, n - 1, None)
     assert st == cs.ERR_INVALID_ARG
     assert b"workspace" in lib.cswattn_last_error()
+
+
+def test_decode_validation(lib):
+    spec = cs.LayerSpec(2, 256, 12, 4, 128, 100, has_ve=True)
+    n = cs.attn_decode_workspace_bytes(spec)
+    # q~ (B,H,D) fp32 + per 64-key chunk (max, sum) and partial O; a window
+    # of 100 keys can straddle ceil(100/64) + 1 = 3 chunks
+    rows, chunks = 2 * 12, 3
+    def pad(x):
+        return (x + 255) // 256 * 256
+    assert n == pad(rows * 128 * 4) + pad(rows * chunks * 2 * 4) + pad(rows * chunks * 128 * 4)
+    assert cs.attn_decode_workspace_bytes(cs.LayerSpec(2, 256, 4, 2, 128, 64, dtype="f32")) == 0
+    assert cs.attn_decode_workspace_bytes(cs.LayerSpec(2, 256, 34, 2, 128, 64)) == 0  # group 17
+    layer = ctypes.byref(spec.c())
+    good = [256 * (i + 1) for i in range(5)]  # q k v ve gate
+    args = good + [4096, 8192, 12288, 16384, 20480, 24576, n, None]
+    assert lib.attn_decode(layer, *args[:5], 4096 + 2, *args[6:]) == cs.ERR_INVALID_ARG  # cache_len
+    assert b"cache_len" in lib.cswattn_last_error()
+    assert lib.attn_decode(layer, *args[:11], n - 1, None) == cs.ERR_INVALID_ARG
+    assert b"workspace" in lib.cswattn_last_error()
+    same = args[:7] + [args[6]] + args[8:]
+    assert lib.attn_decode(layer, *same) == cs.ERR_INVALID_ARG
