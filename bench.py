@@ -257,12 +257,19 @@ def run_ours(args):
     clocks = ClockSampler(visible_gpu_indices(world if world > 1 else 1) if rank == 0 else [])
     if rank == 0:
         clocks.start()
+    # Headline: K steps as a user runs them (the kernels may overlap their
+    # launches with the previous kernel's tail).
+    total_ms = timed(step, args.steps, flush=True)
+    clk = clocks.stop() if rank == 0 else None
+    cs.cswattn_sync_status()
+    # Per-kernel split: a second timed pass of K steps with CUDA events
+    # around every kernel on the launching stream (the events serialise the
+    # kernels, so this pass is a little slower than the headline).
     cs.cswattn_set_timing(True)
     cs.cswattn_kernel_times()
-    total_ms = timed(step, args.steps, flush=True)
-    ktimes = cs.cswattn_kernel_times()
+    split_ms = timed(step, args.steps, flush=True)
+    ktimes = {k: v for k, v in cs.cswattn_kernel_times().items() if v[1] > 0}
     cs.cswattn_set_timing(False)
-    clk = clocks.stop() if rank == 0 else None
     cs.cswattn_sync_status()
 
     # e2e: host buffers in, results out, copies inside the timed region
@@ -301,8 +308,10 @@ def run_ours(args):
                     "unit": "GB/s", "frac": None, "traffic": traffic_for(dom)}
         kern = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches": v[1]}
                 for k, v in ktimes.items()}
+        kern["_pass"] = {"ms_per_step": round(split_ms / args.steps, 4),
+                         "note": "second timed pass with an event pair around every kernel"}
         for k, fl in (("fwd", flops_fwd), ("bwd", flops_bwd)):
-            if ktimes[k][0] > 0:
+            if k in ktimes and ktimes[k][0] > 0:
                 kern[k]["tflops"] = round(sum(fl) * args.steps / (ktimes[k][0] * 1e-3) / 1e12, 2)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",

@@ -53,6 +53,13 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
   const T* ob = static_cast<const T*>(p.O) + tok0 * orow;
   const T* gb = static_cast<const T*>(p.dO) + tok0 * orow;
   const Stage stage{&s_bar};
+  pdl_launch_dependents();
+  if (threadIdx.x < ntt) {
+    const long long tok = tok0 + threadIdx.x;
+    s_b[threadIdx.x] = static_cast<int>(tok / p.T);
+    s_t[threadIdx.x] = static_cast<int>(tok % p.T);
+  }
+  pdl_wait();
   if constexpr (STAGED) {
     T* so = reinterpret_cast<T*>(stage_smem);
     T* sg = so + p.tok * orow;
@@ -64,11 +71,6 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
     }
     ob = so;
     gb = sg;
-  }
-  if (threadIdx.x < ntt) {
-    const long long tok = tok0 + threadIdx.x;
-    s_b[threadIdx.x] = static_cast<int>(tok / p.T);
-    s_t[threadIdx.x] = static_cast<int>(tok % p.T);
   }
   if (p.dq_zero) {
     // The block's rows of the dq accumulator (contiguous in (B,T,H,D)).
@@ -186,6 +188,9 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
   const T* kb = static_cast<const T*>(p.k) + tok0 * kvrow;
   const T* eb = p.has_ve ? static_cast<const T*>(p.ve) + tok0 * kvrow : nullptr;
   const Stage stage{&s_bar};
+  pdl_launch_dependents();
+  tab.fill(tok0, p.T, p.omega, ntt);
+  pdl_wait();
   if constexpr (STAGED) {
     float* sdq = reinterpret_cast<float*>(stage_smem);
     float* sdk = sdq + p.tok * qrow;
@@ -216,7 +221,6 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
     kb = sk;
     eb = se;
   }
-  tab.fill(tok0, p.T, p.omega, ntt);
   __syncthreads();
   if constexpr (STAGED) {
     if (!stage.wait(p.wait_ns)) return;

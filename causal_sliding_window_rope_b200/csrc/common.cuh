@@ -23,6 +23,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch. Kernels launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still
+// running: each kernel lets its successor launch as soon as it starts
+// (launch_dependents), does only work that touches no global memory the
+// previous kernels write or read (barrier setup, TMEM allocation, tables
+// from its parameters), and then waits (wait) until the previous grid has
+// completed and its writes are visible before its first global access.
+// Launched without the attribute, wait returns at once.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // First 1024-byte aligned address of a dynamic shared-memory array. The
 // result is the array pointer plus an offset, so the compiler still knows it
 // points into shared memory (a round trip through an integer would turn

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/cswattn.h"
@@ -168,6 +169,26 @@ cswattn_status set_smem(Kernel k, int bytes, std::once_flag& flag, cudaError_t& 
   return CSWATTN_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may begin
+// while the previous kernel in the stream finishes (every kernel of this
+// library waits for its predecessor before touching global memory).
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Errors surface through cudaGetLastError() in launched().
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cswattn_status launched(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -209,10 +230,10 @@ cswattn_status launch_rows(P p, const RowLaunch& r, cudaStream_t st) {
     cswattn_status e = set_smem(STAGED_K, static_cast<int>(kRowStageMax), flag, ferr);
     if (e != CSWATTN_OK) return e;
     p.tok = r.tok;
-    STAGED_K<<<r.grid, kPrologueThreads, r.smem, st>>>(p);
+    launch_pdl(STAGED_K, dim3(r.grid), dim3(kPrologueThreads), r.smem, st, p);
   } else {
     p.tok = kPrologueTok;
-    DIRECT_K<<<r.grid, kPrologueThreads, 0, st>>>(p);
+    launch_pdl(DIRECT_K, dim3(r.grid), dim3(kPrologueThreads), 0, st, p);
   }
   return CSWATTN_OK;
 }
@@ -486,9 +507,9 @@ cswattn_status launch_decode(const Shape& s, const dec::PrologueParams& pp, cons
   static cudaError_t ferr;
   cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem, flag, ferr);
   if (e != CSWATTN_OK) return e;
-  dec::decode_prologue_kernel<D><<<s.B, dec::kThreads, 0, st>>>(pp);
-  dec::decode_attn_kernel<D><<<dim3(ap.nsplit, s.Hk, s.B), dec::kThreads, kSmem, st>>>(mk, mv, ap);
-  dec::decode_combine_kernel<D><<<s.B * s.H, D, 0, st>>>(cp);
+  launch_pdl(dec::decode_prologue_kernel<D>, dim3(s.B), dim3(dec::kThreads), 0, st, pp);
+  launch_pdl(dec::decode_attn_kernel<D>, dim3(ap.nsplit, s.Hk, s.B), dim3(dec::kThreads), kSmem, st, mk, mv, ap);
+  launch_pdl(dec::decode_combine_kernel<D>, dim3(s.B * s.H), dim3(D), 0, st, cp);
   return CSWATTN_OK;
 }
 
@@ -655,9 +676,9 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
   {
     ScopedTiming tm(CSWATTN_K_FWD, cs);
     if (s.D == 64)
-      fwd::fwd_kernel<64><<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, mo, fp);
+      launch_pdl(fwd::fwd_kernel<64>, dim3(grid), dim3(fwd::kThreads), fwd::kSmemBytes, cs, mq, mk, mv, mo, fp);
     else
-      fwd::fwd_kernel<128><<<grid, fwd::kThreads, fwd::kSmemBytes, cs>>>(mq, mk, mv, mo, fp);
+      launch_pdl(fwd::fwd_kernel<128>, dim3(grid), dim3(fwd::kThreads), fwd::kSmemBytes, cs, mq, mk, mv, mo, fp);
   }
   return launched("forward launch");
 }
@@ -786,9 +807,11 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     {
       ScopedTiming tm(CSWATTN_K_BWD, cs);
       if (s.D == 64)
-        bwd::bwd_kernel<64><<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, mdq, bp);
+        launch_pdl(bwd::bwd_kernel<64>, dim3(grid), dim3(bwd::kThreads), bwd::kSmemBytes, cs, mq, mdo, mk, mv,
+                   mdk, mdv, mdq, bp);
       else
-        bwd::bwd_kernel<128><<<grid, bwd::kThreads, bwd::kSmemBytes, cs>>>(mq, mdo, mk, mv, mdk, mdv, mdq, bp);
+        launch_pdl(bwd::bwd_kernel<128>, dim3(grid), dim3(bwd::kThreads), bwd::kSmemBytes, cs, mq, mdo, mk, mv,
+                   mdk, mdv, mdq, bp);
     }
     if ((st = launched("backward launch")) != CSWATTN_OK) return st;
   }

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
   constexpr int ROWS_PER_PASS = kThreads / LPR;
   __shared__ __align__(16) float cs_[HALF], sn_[HALF];
   const int b = blockIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   const int pos = p.len[b];
   if (pos < 0 || pos >= p.T) {
     if (threadIdx.x == 0) atomicOr(&g_status, kStatusRange);
@@ -179,6 +181,8 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = p.g;
+  pdl_launch_dependents();
+  pdl_wait();
   const int pos = p.len[b];
   const bool in_range = pos >= 0 && pos < p.T;
   const int lo = in_range ? max(0, pos - p.W + 1) : 0;
@@ -362,6 +366,8 @@ struct CombineParams {
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const CombineParams p) {
   const int bh = blockIdx.x, b = bh / p.H, d = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   const int pos = p.len[b];
   if (pos < 0 || pos >= p.T) return;
   const float* ml = p.part_ml + static_cast<size_t>(bh) * p.nsplit * 2;

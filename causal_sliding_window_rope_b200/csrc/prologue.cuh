@@ -243,6 +243,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const T *vb = static_cast<const T*>(p.v) + tok0 * kvrow;
   const T *eb = p.has_ve ? static_cast<const T*>(p.ve) + tok0 * kvrow : nullptr;
   const Stage stage{&s_bar};
+  pdl_launch_dependents();
+  tab.fill(tok0, p.T, p.omega, ntt);
+  pdl_wait();
   if constexpr (STAGED) {
     T* sq = reinterpret_cast<T*>(stage_smem);
     T* sk = sq + p.tok * qrow;
@@ -262,7 +265,6 @@ __global__ void __launch_bounds__(kPrologueThreads)
     vb = sv;
     eb = se;
   }
-  tab.fill(tok0, p.T, p.omega, ntt);
   __syncthreads();
   if constexpr (STAGED) {
     if (!stage.wait(p.wait_ns)) return;
