@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_4d(&tmDK, stk + c * kF32Panel, 32 * c, hk, k0, outer);
         }
         bulk_commit();
-        bulk_wait0();
+        bulk_wait_read0();  // shared source read; the writes finish on their own
       }
     }
   } else {
@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(dqs_free);
       }
     }
-    if (leader) bulk_wait0();
+    if (leader) bulk_wait_read0();  // shared source read; the writes finish on their own
   }
 
   tc_fence_before();

@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_4d(&tmO, ot, 0, head[X], q0, b);
           if (HD > 64) tma_store_4d(&tmO, ot + kPanelBytes, 64, head[X], q0, b);
           bulk_commit();
-          bulk_wait0();
+          bulk_wait_read0();  // shared source read; the writes finish on their own
         }
         if (qi < p.T)
           p.lse[(static_cast<size_t>(b) * p.H + head[X]) * p.T + qi] =
