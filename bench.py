@@ -407,7 +407,7 @@ def decode_bench(w, dev, peaks, steps=20, warmup=5):
                         f"holding {T - 1} tokens, windows {w.windows}",
             "ms_per_step": round(ms, 4), "tokens_per_s": round(B / (ms * 1e-3), 1),
             "kernel_ms_per_step": round(kt["decode"][0] / steps, 4),
-            "launches_per_step": kt["decode"][1] // steps * 3,
+            "launches_per_step": kt["decode"][1] // steps * 2,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": nbytes,
                          "peak_source": "measured hbm_gbs"}}

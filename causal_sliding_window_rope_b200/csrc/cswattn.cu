@@ -467,7 +467,7 @@ cswattn_status noalloc_scratch(void** out) {
 // ---------------------------------------------------------------- decode
 
 struct DecodeWorkspace {
-  float *qt, *part_ml, *part_o;
+  float *part_ml, *part_o;
   int nsplit;
   size_t bytes;
 };
@@ -478,8 +478,6 @@ DecodeWorkspace carve_decode(const Shape& s, void* base) {
   const size_t rows = static_cast<size_t>(s.B) * s.H;
   uint8_t* p = static_cast<uint8_t*>(base);
   size_t off = 0;
-  w.qt = reinterpret_cast<float*>(p + off);
-  off += pad256(rows * s.D * 4);
   w.part_ml = reinterpret_cast<float*>(p + off);
   off += pad256(rows * w.nsplit * 2 * 4);
   w.part_o = reinterpret_cast<float*>(p + off);
@@ -499,15 +497,13 @@ cswattn_status check_decode_layer(const cswattn_layer* layer, Shape* s) {
 }
 
 template <int D>
-cswattn_status launch_decode(const Shape& s, const dec::PrologueParams& pp, const CUtensorMap& mk,
-                             const CUtensorMap& mv, const dec::AttnParams& ap, const dec::CombineParams& cp,
-                             cudaStream_t st) {
+cswattn_status launch_decode(const Shape& s, const CUtensorMap& mk, const CUtensorMap& mv,
+                             const dec::AttnParams& ap, const dec::CombineParams& cp, cudaStream_t st) {
   constexpr int kSmem = dec::decode_attn_smem<D>();
   static std::once_flag flag;
   static cudaError_t ferr;
   cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem, flag, ferr);
   if (e != CSWATTN_OK) return e;
-  launch_pdl(dec::decode_prologue_kernel<D>, dim3(s.B), dim3(dec::kThreads), 0, st, pp);
   launch_pdl(dec::decode_attn_kernel<D>, dim3(ap.nsplit, s.Hk, s.B), dim3(dec::kThreads), kSmem, st, mk, mv, ap);
   launch_pdl(dec::decode_combine_kernel<D>, dim3(s.B * s.H), dim3(D), 0, st, cp);
   return CSWATTN_OK;
@@ -880,23 +876,6 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   CUtensorMap mk, mv;
   if ((st = make_map(&mk, k_cache, s.B, s.T, s.Hk, dec::kChunk, s.D)) != CSWATTN_OK) return st;
   if ((st = make_map(&mv, v_cache, s.B, s.T, s.Hk, dec::kChunk, s.D)) != CSWATTN_OK) return st;
-  dec::PrologueParams pp;
-  pp.B = s.B;
-  pp.T = s.T;
-  pp.H = s.H;
-  pp.Hk = s.Hk;
-  pp.has_ve = layer->has_ve;
-  pp.eps = layer->eps;
-  fill_omega(pp.omega, s.D, layer->rope_base);
-  pp.len = cache_len;
-  pp.q = static_cast<const __nv_bfloat16*>(q);
-  pp.k = static_cast<const __nv_bfloat16*>(k);
-  pp.v = static_cast<const __nv_bfloat16*>(v);
-  pp.ve = static_cast<const __nv_bfloat16*>(ve);
-  pp.gate = static_cast<const __nv_bfloat16*>(gate);
-  pp.kc = static_cast<__nv_bfloat16*>(k_cache);
-  pp.vc = static_cast<__nv_bfloat16*>(v_cache);
-  pp.qt = w.qt;
   dec::AttnParams ap;
   ap.B = s.B;
   ap.T = s.T;
@@ -906,8 +885,17 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   ap.g = s.g;
   ap.nsplit = w.nsplit;
   ap.scale_log2 = s.scale * 1.4426950408889634f;
+  ap.has_ve = layer->has_ve;
+  ap.eps = layer->eps;
+  fill_omega(ap.omega, s.D, layer->rope_base);
   ap.len = cache_len;
-  ap.qt = w.qt;
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.k = static_cast<const __nv_bfloat16*>(k);
+  ap.v = static_cast<const __nv_bfloat16*>(v);
+  ap.ve = static_cast<const __nv_bfloat16*>(ve);
+  ap.gate = static_cast<const __nv_bfloat16*>(gate);
+  ap.kc = static_cast<__nv_bfloat16*>(k_cache);
+  ap.vc = static_cast<__nv_bfloat16*>(v_cache);
   ap.part_ml = w.part_ml;
   ap.part_o = w.part_o;
   ap.wait_ns = g_wait_ns.load();
@@ -924,7 +912,7 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   {
     ScopedTiming tm(CSWATTN_K_DECODE, cs);
-    st = s.D == 64 ? launch_decode<64>(s, pp, mk, mv, ap, cp, cs) : launch_decode<128>(s, pp, mk, mv, ap, cp, cs);
+    st = s.D == 64 ? launch_decode<64>(s, mk, mv, ap, cp, cs) : launch_decode<128>(s, mk, mv, ap, cp, cs);
   }
   if (st != CSWATTN_OK) return st;
   return launched("decode launch");

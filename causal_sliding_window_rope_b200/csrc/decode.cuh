@@ -11,14 +11,14 @@
 //   O_h = sum_j softmax_j(c q~_h . k~_j) v_eff_j over cache rows (p - W, p].
 //
 // The step reads the window of the K/V cache once: it is bound by HBM
-// bandwidth, not by the tensor cores (one query row per head). Three
-// kernels:
-//   decode_prologue: one CTA per sequence, the prologue of its new token
-//     (split-halves row layout of the row kernels);
+// bandwidth, not by the tensor cores (one query row per head). Two kernels:
 //   decode_attn: split-KV. CTA = (64-key chunk of the window, KV head,
 //     sequence), small enough that several CTAs per SM keep their copies in
 //     flight: TMA brings the chunk's K and V rows (128B-swizzled panels)
-//     into shared memory; two threads per key score it against the g query
+//     into shared memory while the CTA computes the new token's prologue
+//     (its query rows of this KV head; the chunk holding row p also its key
+//     and value rows, which it writes to the caches and over the staged
+//     row); two threads per key score it against the g query
 //     heads of the group (half of head_dim each), the CTA reduces the chunk's
 //     max and sum per head, and each thread accumulates two columns of P V
 //     over half of the keys; the partial (max, sum, O) goes to the workspace;
@@ -41,16 +41,6 @@ constexpr int kThreads = 128;
 constexpr int kMaxGroup = 16;   // query heads per KV head handled by one CTA
 constexpr int kPanel = kChunk * 128;  // kChunk rows x 128 bytes
 
-struct PrologueParams {
-  int B, T, H, Hk, has_ve;
-  float eps;
-  float omega[kMaxHalfD];
-  const int* len;
-  const __nv_bfloat16 *q, *k, *v, *ve, *gate;  // (B,H,D), (B,Hk,D), (B,Hk)
-  __nv_bfloat16 *kc, *vc;                      // (B,T,Hk,D)
-  float* qt;                                   // (B,H,D) workspace
-};
-
 // Number of kChunk-key chunks a window of W keys (in a cache of T rows) can
 // straddle: the chunks are aligned to absolute positions.
 __host__ __device__ inline int decode_splits(int T, int W) {
@@ -60,35 +50,33 @@ __host__ __device__ inline int decode_splits(int T, int W) {
   return n < cap ? n : cap;
 }
 
+struct AttnParams {
+  int B, T, H, Hk, W, g, nsplit, has_ve;
+  float scale_log2;  // softmax scale * log2(e)
+  float eps;
+  float omega[kMaxHalfD];                      // rope_base^(-2i/D)
+  const int* len;                              // (B) tokens already cached
+  const __nv_bfloat16 *q, *k, *v, *ve, *gate;  // (B,H,D), (B,Hk,D), (B,Hk)
+  __nv_bfloat16 *kc, *vc;                      // (B,T,Hk,D) caches
+  float* part_ml;     // (B,H,nsplit,2): running max (log2 units), sum
+  float* part_o;      // (B,H,nsplit,D): unnormalised partial O
+  unsigned long long wait_ns;
+};
+
+// Prologue of one row of the new token (page section "1. GPT 모델": QK
+// RMSNorm, RoPE at the token's position, value residual), in the row
+// kernels' split-halves layout: lane `sub` of the row's LPR lanes holds
+// elements [sub HV, (sub+1) HV) of both halves. kind 0: query head (scaled
+// by c log2(e) into shared fp32), 1: key (RMSNorm + RoPE), 2: value
+// (v + 3 sigmoid(gate) ve); kinds 1 and 2 return their bf16 halves.
 template <int D>
-__global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const PrologueParams p) {
+struct NewToken {
   using RL = RowLayout<__nv_bfloat16, D>;
   using HVec = HalfVec<__nv_bfloat16, RL::HV>;
-  constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
-  constexpr int ROWS_PER_PASS = kThreads / LPR;
-  __shared__ __align__(16) float cs_[HALF], sn_[HALF];
-  const int b = blockIdx.x;
-  pdl_launch_dependents();
-  pdl_wait();
-  const int pos = p.len[b];
-  if (pos < 0 || pos >= p.T) {
-    if (threadIdx.x == 0) atomicOr(&g_status, kStatusRange);
-    return;
-  }
-  for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
-    float s, c;
-    sincosf(static_cast<float>(pos) * p.omega[i], &s, &c);
-    cs_[i] = c;
-    sn_[i] = s;
-  }
-  __syncthreads();
-  const int sub = threadIdx.x % LPR, grp = threadIdx.x / LPR;
-  const int rows = p.H + 2 * p.Hk;
-  for (int base = 0; base < rows; base += ROWS_PER_PASS) {
-    const int r = base + grp;
-    const bool valid = r < rows;
-    const int kind = !valid ? 0 : (r < p.H ? 0 : (r < p.H + p.Hk ? 1 : 2));
-    const int head = !valid ? 0 : (kind == 0 ? r : (kind == 1 ? r - p.H : r - p.H - p.Hk));
+  static constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
+
+  __device__ static void row(const AttnParams& p, int b, int kind, int head, int sub, bool valid,
+                             const float* cs, const float* sn, float (&yl)[HV], float (&yh)[HV]) {
     const int nh = kind == 0 ? p.H : p.Hk;
     const size_t src = (static_cast<size_t>(b) * nh + head) * D + sub * HV;
     const __nv_bfloat16* x = kind == 0 ? p.q : (kind == 1 ? p.k : p.v);
@@ -104,13 +92,11 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
 #pragma unroll
     for (int i = 0; i < HV; ++i) ss = fmaf(xl[i], xl[i], fmaf(xh[i], xh[i], ss));
     ss = row_sum<LPR>(ss);
-    if (!valid) continue;
-    const size_t crow = ((static_cast<size_t>(b) * p.T + pos) * p.Hk + head) * D + sub * HV;
     if (kind == 2) {
       float coef = 0.f;
-      if (p.has_ve) coef = 3.0f / (1.0f + expf(-__bfloat162float(p.gate[static_cast<size_t>(b) * p.Hk + head])));
-      float el[HV], eh[HV];
-      if (p.has_ve) {
+      if (valid && p.has_ve) {
+        coef = 3.0f / (1.0f + expf(-__bfloat162float(p.gate[static_cast<size_t>(b) * p.Hk + head])));
+        float el[HV], eh[HV];
         HVec::load(p.ve + src, el);
         HVec::load(p.ve + src + HALF, eh);
 #pragma unroll
@@ -119,47 +105,28 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
           xh[i] = fmaf(coef, eh[i], xh[i]);
         }
       }
-      HVec::store(p.vc + crow, xl);
-      HVec::store(p.vc + crow + HALF, xh);
-      continue;
+#pragma unroll
+      for (int i = 0; i < HV; ++i) {
+        yl[i] = xl[i];
+        yh[i] = xh[i];
+      }
+      return;
     }
     const float rstd = rsqrtf(ss / static_cast<float>(D) + p.eps);
-    float yl[HV], yh[HV];
 #pragma unroll
     for (int i = 0; i < HV; ++i) {
-      const float c = cs_[sub * HV + i], s = sn_[sub * HV + i];
+      const float c = cs[sub * HV + i], s = sn[sub * HV + i];
       const float nl = xl[i] * rstd, nh2 = xh[i] * rstd;
       yl[i] = fmaf(nl, c, -nh2 * s);
       yh[i] = fmaf(nl, s, nh2 * c);
     }
-    if (kind == 1) {
-      HVec::store(p.kc + crow, yl);
-      HVec::store(p.kc + crow + HALF, yh);
-    } else {
-      float* o = p.qt + src;
-#pragma unroll
-      for (int i = 0; i < HV; ++i) {
-        o[i] = yl[i];
-        o[i + HALF] = yh[i];
-      }
-    }
   }
-}
-
-struct AttnParams {
-  int B, T, H, Hk, W, g, nsplit;
-  float scale_log2;  // softmax scale * log2(e)
-  const int* len;
-  const float* qt;    // (B,H,D)
-  float* part_ml;     // (B,H,nsplit,2): running max (log2 units), sum
-  float* part_o;      // (B,H,nsplit,D): unnormalised partial O
-  unsigned long long wait_ns;
 };
 
 // Shared memory of decode_attn_kernel<D> (dynamic, with 1 KB of alignment slack).
 template <int D>
 constexpr int decode_attn_smem() {
-  return 4 * kPanel + (kMaxGroup * D + kMaxGroup * kChunk + kMaxGroup * D + kMaxGroup * 6) * 4 + 1024;
+  return 4 * kPanel + (kMaxGroup * D + kMaxGroup * kChunk + kMaxGroup * D + kMaxGroup * 6 + D) * 4 + 1024;
 }
 
 template <int D>
@@ -176,6 +143,8 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
   float* so = sp + kMaxGroup * kChunk;                       // [g][D] second half of P V
   float* red = so + kMaxGroup * D;                           // [g][4] warp partials
   float* stat = red + kMaxGroup * 4;                         // [g][2] max, sum
+  float* cs = stat + kMaxGroup * 2;                          // [D/2] cos(p omega_i)
+  float* sn = cs + D / 2;                                    // [D/2] sin(p omega_i)
   __shared__ uint64_t bar;
 
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -185,9 +154,11 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
   pdl_wait();
   const int pos = p.len[b];
   const bool in_range = pos >= 0 && pos < p.T;
+  if (!in_range && split == 0 && hk == 0 && tid == 0) atomicOr(&g_status, kStatusRange);
   const int lo = in_range ? max(0, pos - p.W + 1) : 0;
   const int c0 = (lo / kChunk) * kChunk + split * kChunk;
   const bool work = in_range && c0 <= pos;
+  const bool owns_new = work && pos < c0 + kChunk;  // this chunk holds the new token's row
   auto part = [&](int h) { return (static_cast<size_t>(b) * p.H + h) * p.nsplit + split; };
   if (!work) {
     // Empty chunk: a partial that the combine step ignores.
@@ -209,8 +180,49 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
     tma_load_4d(&tmV, &bar, sV, 0, hk, c0, b);
     tma_load_4d(&tmV, &bar, sV + kPanel, 64, hk, c0, b);
   }
-  for (int i = tid; i < g * D; i += blockDim.x)
-    sq[i] = p.qt[(static_cast<size_t>(b) * p.H + hk * g) * D + i] * p.scale_log2;
+  // The new token's prologue at position pos: its g query rows of this KV
+  // head (into sq, scaled by c log2(e)), and, in the chunk that holds row
+  // pos, its key and value rows (written to the caches and, after the chunk
+  // has landed, over row pos - c0 of the staged tiles).
+  using NT = NewToken<D>;
+  for (int i = tid; i < D / 2; i += blockDim.x) {
+    float sv_, cv_;
+    sincosf(static_cast<float>(pos) * p.omega[i], &sv_, &cv_);
+    cs[i] = cv_;
+    sn[i] = sv_;
+  }
+  __syncthreads();
+  const int sub = tid % NT::LPR, grp = tid / NT::LPR;
+  constexpr int kRowsPerPass = kThreads / NT::LPR;
+  float kl[NT::HV], kh2[NT::HV];
+  bool have_k = false, have_v = false;
+  for (int base = 0; base < g + 2; base += kRowsPerPass) {
+    const int rr = base + grp;
+    const int kind = rr < g ? 0 : (rr == g ? 1 : 2);
+    const bool valid = rr < g || (owns_new && rr < g + 2);
+    float yl[NT::HV], yh[NT::HV];
+    NT::row(p, b, kind, kind == 0 ? hk * g + rr : hk, sub, valid, cs, sn, yl, yh);
+    if (!valid) continue;
+    if (kind == 0) {
+#pragma unroll
+      for (int i = 0; i < NT::HV; ++i) {
+        sq[rr * D + sub * NT::HV + i] = yl[i] * p.scale_log2;
+        sq[rr * D + NT::HALF + sub * NT::HV + i] = yh[i] * p.scale_log2;
+      }
+    } else {
+      const size_t crow = ((static_cast<size_t>(b) * p.T + pos) * p.Hk + hk) * D + sub * NT::HV;
+      __nv_bfloat16* cache = kind == 1 ? p.kc : p.vc;
+      NT::HVec::store(cache + crow, yl);
+      NT::HVec::store(cache + crow + NT::HALF, yh);
+#pragma unroll
+      for (int i = 0; i < NT::HV; ++i) {
+        kl[i] = yl[i];
+        kh2[i] = yh[i];
+      }
+      have_k = kind == 1;
+      have_v = kind == 2;
+    }
+  }
   __syncthreads();
   {
     bool ok = mbar_try_wait(&bar, 0);
@@ -224,6 +236,23 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
     }
     if (!__syncthreads_and(ok)) return;
   }
+  if (have_k || have_v) {
+    // Row pos of the staged tile (bf16, 128B-swizzled panels) gets the new
+    // token's values: the copy brought in whatever the cache held there.
+    const int rr = pos - c0;
+    uint8_t* tile = have_k ? sK : sV;
+    auto put = [&](int d0, const float (&x)[NT::HV]) {
+      uint4 u;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+      *reinterpret_cast<uint4*>(tile + (d0 >> 6) * kPanel + rr * 128 + ((((d0 & 63) >> 3) ^ (rr & 7)) << 4)) = u;
+    };
+    static_assert(NT::HV == 8, "one 16-byte chunk per half");
+    put(sub * NT::HV, kl);
+    put(NT::HALF + sub * NT::HV, kh2);
+  }
+  __syncthreads();
 
   // Scores (log2 units): threads 2r and 2r+1 take key r = tid / 2, each half
   // of its columns (one 128-byte panel of D = 128, half a panel of D = 64).
@@ -372,8 +401,10 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const CombineParams p
   if (pos < 0 || pos >= p.T) return;
   const float* ml = p.part_ml + static_cast<size_t>(bh) * p.nsplit * 2;
   float M = -INFINITY;
+#pragma unroll 8
   for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[2 * s]);
   float L = 0.f, o = 0.f;
+#pragma unroll 8
   for (int s = 0; s < p.nsplit; ++s) {
     if (ml[2 * s] == -INFINITY) continue;
     const float w = exp2f(ml[2 * s] - M);

@@ -127,12 +127,12 @@ def test_workspace_size_and_check(lib):
 def test_decode_validation(lib):
     spec = cs.LayerSpec(2, 256, 12, 4, 128, 100, has_ve=True)
     n = cs.attn_decode_workspace_bytes(spec)
-    # q~ (B,H,D) fp32 + per 64-key chunk (max, sum) and partial O; a window
+    # per 64-key chunk (max, sum) and partial O of every query head; a window
     # of 100 keys can straddle ceil(100/64) + 1 = 3 chunks
     rows, chunks = 2 * 12, 3
     def pad(x):
         return (x + 255) // 256 * 256
-    assert n == pad(rows * 128 * 4) + pad(rows * chunks * 2 * 4) + pad(rows * chunks * 128 * 4)
+    assert n == pad(rows * chunks * 2 * 4) + pad(rows * chunks * 128 * 4)
     assert cs.attn_decode_workspace_bytes(cs.LayerSpec(2, 256, 4, 2, 128, 64, dtype="f32")) == 0
     assert cs.attn_decode_workspace_bytes(cs.LayerSpec(2, 256, 34, 2, 128, 64)) == 0  # group 17
     layer = ctypes.byref(spec.c())
