@@ -406,7 +406,9 @@ int bwd_parts(const Shape& s) {
     nmax = std::max(nmax, n);
   }
   total *= static_cast<long long>(s.B) * s.Hk;
-  const long long want = (2 * nmax * 148 + total - 1) / std::max(total, 1ll);
+  // Parts per key tile: about 1.5 x (heaviest tile / average work per SM of
+  // a 148-SM B200), measured best on the d24 workload among 1, 1.5, 2 and 3.
+  const long long want = (3 * nmax * 148 + 2 * total - 1) / std::max(2 * total, 1ll);
   return static_cast<int>(std::min<long long>(8, std::max<long long>(1, want)));
 }
 
