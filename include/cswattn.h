@@ -36,7 +36,11 @@
  * scratch is the caller's `workspace`. Pointers to element tensors must be
  * 16-byte aligned; rstd/lse/gate pointers 4-byte (2-byte for bf16 gate).
  * Streams: every call is asynchronous on `stream` (a cudaStream_t; NULL is
- * the legacy default stream) and returns once the work is enqueued.
+ * the legacy default stream) and returns once the work is enqueued. The bf16
+ * kernels are launched with programmatic stream serialization: a kernel may
+ * be scheduled while the previous kernel on the stream is finishing, but it
+ * touches no global memory until that kernel has completed, so stream order
+ * holds as for ordinary launches.
  * Errors: arguments are validated on the host before anything is enqueued;
  * a rejected call returns CSWATTN_ERR_INVALID_ARG or CSWATTN_ERR_UNSUPPORTED
  * and enqueues nothing. A failed launch returns CSWATTN_ERR_CUDA. Device-side
