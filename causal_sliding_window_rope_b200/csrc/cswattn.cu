@@ -169,6 +169,10 @@ cswattn_status set_smem(Kernel k, int bytes, std::once_flag& flag, cudaError_t& 
   return CSWATTN_OK;
 }
 
+// First failed launch of the current call on this thread, reported (and
+// cleared) by launched().
+thread_local cudaError_t t_launch_error = cudaSuccess;
+
 // Launch with programmatic stream serialization: the kernel may begin
 // while the previous kernel in the stream finishes (every kernel of this
 // library waits for its predecessor before touching global memory).
@@ -185,12 +189,15 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // Errors surface through cudaGetLastError() in launched().
-  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess && t_launch_error == cudaSuccess) t_launch_error = e;
 }
 
 cswattn_status launched(const char* what) {
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = t_launch_error;
+  t_launch_error = cudaSuccess;
+  const cudaError_t last = cudaGetLastError();
+  if (e == cudaSuccess) e = last;
   if (e != cudaSuccess) return cuda_fail(e, what);
   return CSWATTN_OK;
 }
