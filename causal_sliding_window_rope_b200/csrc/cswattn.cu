@@ -502,6 +502,8 @@ cswattn_status check_decode_layer(const cswattn_layer* layer, Shape* s) {
   if (s->g > dec::kMaxGroup)
     return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports up to %d query heads per KV head (got %d)",
                 dec::kMaxGroup, s->g);
+  if (s->B > 65535 || s->Hk > 65535)  // grid dimensions of the split-KV kernel
+    return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports B, n_kv_head <= 65535");
   return CSWATTN_OK;
 }
 

@@ -135,6 +135,7 @@ def test_decode_validation(lib):
     assert n == pad(rows * chunks * 2 * 4) + pad(rows * chunks * 128 * 4)
     assert cs.attn_decode_workspace_bytes(cs.LayerSpec(2, 256, 4, 2, 128, 64, dtype="f32")) == 0
     assert cs.attn_decode_workspace_bytes(cs.LayerSpec(2, 256, 34, 2, 128, 64)) == 0  # group 17
+    assert cs.attn_decode_workspace_bytes(cs.LayerSpec(70000, 16, 4, 2, 128, 8)) == 0  # grid limit
     layer = ctypes.byref(spec.c())
     good = [256 * (i + 1) for i in range(5)]  # q k v ve gate
     args = good + [4096, 8192, 12288, 16384, 20480, 24576, n, None]
