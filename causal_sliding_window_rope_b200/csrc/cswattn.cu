@@ -160,12 +160,23 @@ cswattn_status make_map(CUtensorMap* map, const void* base, int outer, int T, in
   return CSWATTN_OK;
 }
 
+// Raises a kernel's dynamic shared-memory limit on the current device, once
+// per (kernel, device): the attribute belongs to the device's context, so a
+// process that drives several GPUs sets it on each.
 template <typename Kernel>
-cswattn_status set_smem(Kernel k, int bytes, std::once_flag& flag, cudaError_t& err) {
-  std::call_once(flag, [&] {
-    err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  });
-  if (err != cudaSuccess) return cuda_fail(err, "cudaFuncSetAttribute");
+cswattn_status set_smem(Kernel k, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const void* key = reinterpret_cast<const void*>(k);
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == key && d.second == dev) return CSWATTN_OK;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done.emplace_back(key, dev);
   return CSWATTN_OK;
 }
 
@@ -232,9 +243,7 @@ template <auto STAGED_K, auto DIRECT_K, typename P>
 cswattn_status launch_rows(P p, const RowLaunch& r, cudaStream_t st) {
   p.wait_ns = g_wait_ns.load();
   if (r.tok > 0) {
-    static std::once_flag flag;
-    static cudaError_t ferr = cudaSuccess;
-    cswattn_status e = set_smem(STAGED_K, static_cast<int>(kRowStageMax), flag, ferr);
+    cswattn_status e = set_smem(STAGED_K, static_cast<int>(kRowStageMax));
     if (e != CSWATTN_OK) return e;
     p.tok = r.tok;
     launch_pdl(STAGED_K, dim3(r.grid), dim3(kPrologueThreads), r.smem, st, p);
@@ -511,9 +520,7 @@ template <int D>
 cswattn_status launch_decode(const Shape& s, const CUtensorMap& mk, const CUtensorMap& mv,
                              const dec::AttnParams& ap, const dec::CombineParams& cp, cudaStream_t st) {
   constexpr int kSmem = dec::decode_attn_smem<D>();
-  static std::once_flag flag;
-  static cudaError_t ferr;
-  cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem, flag, ferr);
+  cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem);
   if (e != CSWATTN_OK) return e;
   launch_pdl(dec::decode_attn_kernel<D>, dim3(ap.nsplit, s.Hk, s.B), dim3(dec::kThreads), kSmem, st, mk, mv, ap);
   launch_pdl(dec::decode_combine_kernel<D>, dim3(s.B * s.H), dim3(D), 0, st, cp);
@@ -661,10 +668,8 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
   if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, fwd::kBM, s.D)) != CSWATTN_OK) return st;
   CUtensorMap mo;
   if ((st = make_map(&mo, O, s.B, s.T, s.H, fwd::kBM, s.D)) != CSWATTN_OK) return st;
-  static std::once_flag flag128, flag64;
-  static cudaError_t ferr128, ferr64;
-  if ((st = s.D == 64 ? set_smem(fwd::fwd_kernel<64>, fwd::kSmemBytes, flag64, ferr64)
-                      : set_smem(fwd::fwd_kernel<128>, fwd::kSmemBytes, flag128, ferr128)) != CSWATTN_OK)
+  if ((st = s.D == 64 ? set_smem(fwd::fwd_kernel<64>, fwd::kSmemBytes)
+                      : set_smem(fwd::fwd_kernel<128>, fwd::kSmemBytes)) != CSWATTN_OK)
     return st;
   fwd::Params fp;
   fp.B = s.B;
@@ -786,10 +791,8 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
     CUtensorMap mdq;
     if ((st = make_map(&mdq, w.dq_acc, s.B, s.T, s.H, bwd::kBQ, s.D, true)) != CSWATTN_OK) return st;
-    static std::once_flag flag128, flag64;
-    static cudaError_t ferr128, ferr64;
-    if ((st = s.D == 64 ? set_smem(bwd::bwd_kernel<64>, bwd::kSmemBytes, flag64, ferr64)
-                        : set_smem(bwd::bwd_kernel<128>, bwd::kSmemBytes, flag128, ferr128)) != CSWATTN_OK)
+    if ((st = s.D == 64 ? set_smem(bwd::bwd_kernel<64>, bwd::kSmemBytes)
+                        : set_smem(bwd::bwd_kernel<128>, bwd::kSmemBytes)) != CSWATTN_OK)
       return st;
     bwd::Params bp;
     bp.B = s.B;
