@@ -252,7 +252,11 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        return sum(a.elapsed_time(b) for a, b in evs)
+        per_step = [a.elapsed_time(b) for a, b in evs]
+        step_times.append(per_step)
+        return sum(per_step)
+
+    step_times = []  # per-step milliseconds of each timed() call, in call order
 
     clocks = ClockSampler(visible_gpu_indices(world if world > 1 else 1) if rank == 0 else [])
     if rank == 0:
@@ -316,7 +320,10 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(ms_per_step, 4),
+            "step_ms": {"median": round(statistics.median(step_times[0]), 4),
+                        "min": round(min(step_times[0]), 4), "rank": 0},
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) d24-layer-shaped tensors)",
             "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.T,
                        "parallelism": f"dp{world} (independent batch per GPU, no collective)",
