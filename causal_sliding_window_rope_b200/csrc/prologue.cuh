@@ -7,12 +7,14 @@
 //
 // One CTA handles `tok` consecutive tokens (b, t). The row kernels are bound
 // by HBM bandwidth and are short (tens of microseconds), so what matters is
-// how many bytes are in flight from the start: in the staged form thread 0
-// issues one bulk copy (cp.async.bulk) per input tensor for the whole token
-// block before anything else happens, and the CTA computes cos/sin(t omega_i)
-// for its tokens into shared memory while the copies land. The rows are then
-// read from shared memory. (The direct form reads global memory row by row;
-// it serves layers whose token block does not fit in shared memory.)
+// how many bytes are in flight from the start: the CTA computes
+// cos/sin(t omega_i) for its tokens into shared memory (which needs no
+// global memory, so it overlaps the previous kernel's tail under
+// programmatic launch), then in the staged form thread 0 issues one bulk
+// copy (cp.async.bulk) per input tensor for the whole token block and the
+// rows are read from shared memory once they have landed. (The direct form
+// reads global memory row by row; it serves layers whose token block does
+// not fit in shared memory.)
 //
 // A row of D elements is owned by LPR = D / (2 HV) lanes; lane l holds the
 // HV-element slices [l HV, (l+1) HV) of both halves of the row (elements i
