@@ -145,3 +145,17 @@ def test_decode_validation(lib):
     assert b"workspace" in lib.cswattn_last_error()
     same = args[:7] + [args[6]] + args[8:]
     assert lib.attn_decode(layer, *same) == cs.ERR_INVALID_ARG
+
+
+def test_header_enums_match_the_binding():
+    """Status codes and kernel kinds in the header are the ones the Python
+    binding uses (ctypes cannot check enums)."""
+    text = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                             "include", "cswattn.h")).read()
+    codes = dict(re.findall(r"CSWATTN_(OK|ERR_\w+)\s*=\s*(\d+)", text))
+    assert int(codes["OK"]) == cs.OK
+    for name in ("INVALID_ARG", "UNSUPPORTED", "CUDA", "TIMEOUT"):
+        assert int(codes["ERR_" + name]) == getattr(cs, "ERR_" + name)
+    kinds = re.findall(r"CSWATTN_K_(\w+)\s*=\s*(\d+)", text)
+    assert [k.lower() for k, _ in sorted(kinds, key=lambda kv: int(kv[1]))] == list(cs.KERNEL_KINDS)
+    assert int(re.search(r"CSWATTN_NUM_KERNELS\s*=\s*(\d+)", text).group(1)) == len(cs.KERNEL_KINDS)
