@@ -1,6 +1,6 @@
 """Benchmark: attention forward+backward TFLOP/s of the d24 GQA SSSL layer stack.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
     (N > 1: python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N ...)
 
 One step is the whole hot path over one batch of synthetic input: for each of
@@ -29,7 +29,8 @@ sys.path.insert(0, ROOT)
 METRIC = "attn fwd+bwd TFLOP/s (bf16, causal/windowed) and % of B200 dense BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0  # NVIDIA B200 dense BF16 (HGX B200 datasheet: 36 PF sparse per 8 GPUs)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-CONFIG_ID = 4
+DEFAULT_CONFIG = 4           # the headline workload: d24 GQA SSSL
+BF16_CONFIGS = (2, 3, 4, 5)
 
 
 def load_peaks():
@@ -106,9 +107,9 @@ class ClockSampler:
                 "reasons": sorted(self.reasons)}
 
 
-def rank_config_id(rank: int) -> int:
+def rank_config_id(rank: int, config: int = DEFAULT_CONFIG) -> int:
     """Seed component of a rank's batch: every rank draws its own inputs."""
-    return CONFIG_ID + 1000 * rank
+    return config + 1000 * rank
 
 
 def reduce_max(values, dist, device):
@@ -130,73 +131,91 @@ def visible_gpu_indices(n_local):
     return list(range(n_local))
 
 
-# ---------------------------------------------------------------------- ours
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
 
-    import causal_sliding_window_rope_b200 as cs
-    from causal_sliding_window_rope_b200 import synth
-    from causal_sliding_window_rope_b200.build import build
+def layer_flops(w):
+    """Per-layer FLOPs of one step: (fwd+bwd 12*D, fwd 4*D, bwd 8*D) per unmasked pair."""
+    fl = lambda per: [per * w.D * w.pairs(W) * w.B * w.H for W in w.windows]  # noqa: E731
+    return fl(12.0), fl(4.0), fl(8.0)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    if rank == 0:
-        build()
-    if world > 1:
-        dist.barrier()
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
 
-    w = cs.WORKLOADS[CONFIG_ID]
-    if args.single_layer is not None:
-        # Profiling case: one layer of the workload, same shapes and launches.
-        i = args.single_layer
-        w = cs.Workload(w.config, w.name + f" (layer {i} only)", w.B, w.T, w.H, w.Hk, w.D,
-                        [w.windows[i]], [w.ve[i]], w.dtype, w.rope_base, w.eps, w.dO_std)
-    specs = [cs.LayerSpec(w.B, w.T, w.H, w.Hk, w.D, W, has_ve=ve, dtype=w.dtype,
-                          rope_base=w.rope_base, eps=w.eps)
-             for W, ve in zip(w.windows, w.ve)]
-    # Per-rank shard: its own batch, seeded by rank (config id offset).
-    host = [synth.layer_inputs(w.B, w.T, w.H, w.Hk, w.D, ve, torch.bfloat16,
-                               config=rank_config_id(rank), layer=i, dO_std=w.dO_std)
-            for i, ve in enumerate(w.ve)]
-    names = ("q", "k", "v", "ve", "gate", "dO")
-    pinned = [{k: (v.pin_memory() if v is not None else None) for k, v in h.items()} for h in host]
-    inp = [{k: (v.to(dev) if v is not None else None) for k, v in h.items()} for h in host]
-    bufs = [cs.LayerBuffers(s, device=dev) for s in specs]
-    stream = torch.cuda.current_stream(dev)
-    l2_flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+def roofline(ktimes, w, steps, peaks, peak_src):
+    """Roofline object of the dominant kernel (the kind with the most device
+    time in the per-kernel pass). The tensor-core kernels are timed inside a
+    short region (tens of milliseconds at the maximum SM clock), so their
+    denominator is the burst bf16 matmul peak."""
+    _, flops_fwd, flops_bwd = layer_flops(w)
+    dom = max(ktimes, key=lambda k: ktimes[k][0])
+    dom_ms, dom_n = ktimes[dom]
+    if dom in ("fwd", "bwd"):
+        fl = flops_fwd if dom == "fwd" else flops_bwd
+        achieved = sum(fl) * steps / (dom_ms * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        return {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is short and "
+                               f"runs at the maximum SM clock)",
+                "frac_of_sustained": round(achieved / sus, 4),
+                "launches": dom_n, "avg_launch_us": round(dom_ms / max(dom_n, 1) * 1e3, 2),
+                "traffic": traffic_for(dom)}
+    return {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": None, "traffic": traffic_for(dom)}
 
-    def step():
-        for s, x, b in zip(specs, inp, bufs):
+
+class Stack:
+    """Device inputs, pinned host copies and output buffers of one workload's
+    layer stack, with the step functions the benchmark times."""
+
+    def __init__(self, w, dev, rank, cs, synth):
+        import torch
+        self.w, self.dev, self.cs = w, dev, cs
+        self.specs = [cs.LayerSpec(w.B, w.T, w.H, w.Hk, w.D, W, has_ve=ve, dtype=w.dtype,
+                                   rope_base=w.rope_base, eps=w.eps)
+                      for W, ve in zip(w.windows, w.ve)]
+        host = [synth.layer_inputs(w.B, w.T, w.H, w.Hk, w.D, ve, torch.bfloat16,
+                                   config=rank_config_id(rank, w.config), layer=i, dO_std=w.dO_std)
+                for i, ve in enumerate(w.ve)]
+        self.pinned = [{k: (v.pin_memory() if v is not None else None) for k, v in h.items()}
+                       for h in host]
+        self.inp = [{k: (v.to(dev) if v is not None else None) for k, v in h.items()} for h in host]
+        self.bufs = [cs.LayerBuffers(s, device=dev) for s in self.specs]
+        self.stream = torch.cuda.current_stream(dev)
+        out_names = ("O", "dQ", "dK", "dV", "dve", "dgate")
+        self.host_out = [{n: torch.empty_like(getattr(b, n), device="cpu").pin_memory()
+                          for n in out_names if getattr(b, n) is not None} for b in self.bufs]
+        self.h2d = sum(v.numel() * v.element_size() for p in self.pinned for v in p.values()
+                       if v is not None)
+        self.d2h = sum(v.numel() * v.element_size() for o in self.host_out for v in o.values())
+        self.s_in, self.s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def step(self):
+        cs = self.cs
+        for s, x, b in zip(self.specs, self.inp, self.bufs):
             cs.layer_forward(s, b, x["q"], x["k"], x["v"], x["ve"], x["gate"])
             cs.layer_backward(s, b, x["q"], x["k"], x["ve"], x["gate"], x["dO"])
 
-    out_names = ("O", "dQ", "dK", "dV", "dve", "dgate")
-    host_out = [{n: torch.empty_like(getattr(b, n), device="cpu").pin_memory()
-                 for n in out_names if getattr(b, n) is not None} for b in bufs]
-    h2d = sum(v.numel() * v.element_size() for p in pinned for v in p.values() if v is not None)
-    d2h = sum(v.numel() * v.element_size() for o in host_out for v in o.values())
-
-    # e2e step: host->device copies on one stream, kernels on the main one,
-    # device->host copies on a third, chained per layer by events, so that
-    # the two copy directions (PCIe is full duplex) and the kernels overlap.
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    fwd_names, grad_names = ("q", "k", "v", "ve", "gate"), ("dQ", "dK", "dV", "dve", "dgate")
-
-    def step_e2e():
+    def step_e2e(self):
+        """Host->device copies on one stream, kernels on the main one,
+        device->host copies on a third, chained per layer by events, so that
+        the two copy directions (PCIe is full duplex) and the kernels overlap."""
+        import torch
+        cs, stream, s_in, s_out = self.cs, self.stream, self.s_in, self.s_out
+        fwd_names, grad_names = ("q", "k", "v", "ve", "gate"), ("dQ", "dK", "dV", "dve", "dgate")
         begin = torch.cuda.Event()
         begin.record(stream)
         s_in.wait_event(begin)
         s_out.wait_event(begin)
-        for s, x, p, b, o in zip(specs, inp, pinned, bufs, host_out):
+        for s, x, p, b, o in zip(self.specs, self.inp, self.pinned, self.bufs, self.host_out):
             with torch.cuda.stream(s_in):
                 for n in fwd_names:
                     if p[n] is not None:
@@ -227,104 +246,170 @@ def run_ours(args):
             e.record(side)
             stream.wait_event(e)
 
-    flops_layer = [12.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
-    flops_fwd = [4.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
-    flops_bwd = [8.0 * w.D * w.pairs(W) * w.B * w.H for W in w.windows]
-    flops_step = sum(flops_layer)
 
-    for _ in range(args.warmup):
-        step()
+def timed_steps(fn, k, stream, dev, flush_buf, world, dist):
+    """Per-step device milliseconds of k calls of fn, CUDA events on the
+    launching stream, a barrier and a synchronize on both sides; the L2
+    flush buffer (if any) is written before each step, outside the events."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(k)]
+    if world > 1:
+        dist.barrier()
     torch.cuda.synchronize(dev)
+    for a, b in evs:
+        if flush_buf is not None:
+            flush_buf.zero_()  # L2 holds nothing of the next step
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+# ---------------------------------------------------------------------- ours
+
+def measure_stack(st, args, world, dist, flush_buf, warmup, steps, with_split=True):
+    """Warm-up, the headline pass and (optionally) the per-kernel pass of one
+    stack. Returns (per-step ms of the headline pass, per-kernel times)."""
+    import torch
+    cs = st.cs
+    for _ in range(warmup):
+        st.step()
+    torch.cuda.synchronize(st.dev)
     cs.cswattn_sync_status()
+    per_step = timed_steps(st.step, steps, st.stream, st.dev, flush_buf, world, dist)
+    cs.cswattn_sync_status()
+    ktimes = {}
+    if with_split:
+        # Per-kernel split: a second timed pass with CUDA events around every
+        # kernel on the launching stream (the events serialise the kernels,
+        # so this pass is a little slower than the headline).
+        cs.cswattn_set_timing(True)
+        cs.cswattn_kernel_times()
+        split = timed_steps(st.step, steps, st.stream, st.dev, flush_buf, world, dist)
+        ktimes = {k: v for k, v in cs.cswattn_kernel_times().items() if v[1] > 0}
+        ktimes["_pass_ms"] = (sum(split), 0)
+        cs.cswattn_set_timing(False)
+        cs.cswattn_sync_status()
+    return per_step, ktimes
 
-    def timed(fn, k, flush):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(k)]
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        for a, b in evs:
-            if flush:
-                l2_flush.zero_()  # outside the events: L2 holds nothing of the next step
-            a.record(stream)
-            fn()
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        per_step = [a.elapsed_time(b) for a, b in evs]
-        step_times.append(per_step)
-        return sum(per_step)
 
-    step_times = []  # per-step milliseconds of each timed() call, in call order
+def kernel_table(ktimes, w, steps):
+    _, flops_fwd, flops_bwd = layer_flops(w)
+    kern = {k: {"ms_per_step": round(v[0] / steps, 4), "launches": v[1]}
+            for k, v in ktimes.items() if not k.startswith("_")}
+    for k, fl in (("fwd", flops_fwd), ("bwd", flops_bwd)):
+        if k in ktimes and ktimes[k][0] > 0:
+            kern[k]["tflops"] = round(sum(fl) * steps / (ktimes[k][0] * 1e-3) / 1e12, 2)
+    if "_pass_ms" in ktimes:
+        kern["_pass"] = {"ms_per_step": round(ktimes["_pass_ms"][0] / steps, 4),
+                         "note": "second timed pass with an event pair around every kernel"}
+    return kern
+
+
+def other_configs(args, dev, peaks, peak_src, flush_buf, cs, synth):
+    """Device-timed throughput of the other bf16 workloads (one process only):
+    the same headline and per-kernel passes, without e2e or CPU legs."""
+    import torch
+    out = {}
+    for cid in BF16_CONFIGS:
+        if cid == args.config:
+            continue
+        w = cs.WORKLOADS[cid]
+        st = Stack(w, dev, 0, cs, synth)
+        per_step, kt = measure_stack(st, args, 1, None, flush_buf, 3, args.steps)
+        ms = sum(per_step) / args.steps
+        fl = sum(layer_flops(w)[0])
+        out[str(cid)] = {"workload": workload_desc(w), "value": round(fl / (ms * 1e-3) / 1e12, 2),
+                         "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+                         "pct_of_peak": {"measured_burst": round(fl / (ms * 1e-3) / 1e12 / peaks.get(
+                             "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]), 4),
+                             "nominal_dense": round(fl / (ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS, 4)},
+                         "roofline": roofline({k: v for k, v in kt.items() if not k.startswith("_")},
+                                              w, args.steps, peaks, peak_src),
+                         "kernels": kernel_table(kt, w, args.steps)}
+        del st
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import causal_sliding_window_rope_b200 as cs
+    from causal_sliding_window_rope_b200 import synth
+    from causal_sliding_window_rope_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    w = cs.WORKLOADS[args.config]
+    if args.single_layer is not None:
+        # Profiling case: one layer of the workload, same shapes and launches.
+        i = args.single_layer
+        w = cs.Workload(w.config, w.name + f" (layer {i} only)", w.B, w.T, w.H, w.Hk, w.D,
+                        [w.windows[i]], [w.ve[i]], w.dtype, w.rope_base, w.eps, w.dO_std)
+    st = Stack(w, dev, rank, cs, synth)
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flops_step = sum(layer_flops(w)[0])
 
     clocks = ClockSampler(visible_gpu_indices(world if world > 1 else 1) if rank == 0 else [])
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize(dev)
+    cs.cswattn_sync_status()
     if rank == 0:
         clocks.start()
     # Headline: K steps as a user runs them (the kernels may overlap their
     # launches with the previous kernel's tail).
-    total_ms = timed(step, args.steps, flush=True)
+    step_ms = timed_steps(st.step, args.steps, st.stream, dev, flush_buf, world, dist)
     clk = clocks.stop() if rank == 0 else None
     cs.cswattn_sync_status()
-    # Per-kernel split: a second timed pass of K steps with CUDA events
-    # around every kernel on the launching stream (the events serialise the
-    # kernels, so this pass is a little slower than the headline).
-    cs.cswattn_set_timing(True)
-    cs.cswattn_kernel_times()
-    split_ms = timed(step, args.steps, flush=True)
-    ktimes = {k: v for k, v in cs.cswattn_kernel_times().items() if v[1] > 0}
-    cs.cswattn_set_timing(False)
-    cs.cswattn_sync_status()
+    _, ktimes = measure_stack(st, args, world, dist, flush_buf, 0, args.steps)
 
     # e2e: host buffers in, results out, copies inside the timed region
     e2e_steps = max(1, min(args.steps, 5))
     if args.single_layer is None:
         for _ in range(2):
-            step_e2e()
+            st.step_e2e()
         torch.cuda.synchronize(dev)
-        e2e_ms = timed(step_e2e, e2e_steps, flush=False)
+        e2e_ms = sum(timed_steps(st.step_e2e, e2e_steps, st.stream, dev, None, world, dist))
     else:
         e2e_ms = float("nan")
     cs.cswattn_sync_status()
 
-    total_ms, e2e_ms = reduce_max([total_ms, e2e_ms], dist if world > 1 else None, dev)
+    total_ms, e2e_ms = reduce_max([sum(step_ms), e2e_ms], dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
     e2e_value = flops_step * world / (e2e_ms / e2e_steps * 1e-3) / 1e12
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        launches = sum(n for _, n in ktimes.values())
-        # dominant kernel: the kind with the most device time
-        dom = max(ktimes, key=lambda k: ktimes[k][0])
-        dom_ms, dom_n = ktimes[dom]
-        if dom in ("fwd", "bwd"):
-            fl = (flops_fwd if dom == "fwd" else flops_bwd)
-            achieved = sum(fl) * args.steps / (dom_ms * 1e-3) / 1e12
-            peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-            roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
-                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "peak_source": f"{peak_src} bf16_tflops_sustained",
-                    "launches": dom_n, "avg_launch_us": round(dom_ms / max(dom_n, 1) * 1e3, 2),
-                    "traffic": traffic_for(dom)}
-        else:
-            roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": None, "traffic": traffic_for(dom)}
-        kern = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches": v[1]}
-                for k, v in ktimes.items()}
-        kern["_pass"] = {"ms_per_step": round(split_ms / args.steps, 4),
-                         "note": "second timed pass with an event pair around every kernel"}
-        for k, fl in (("fwd", flops_fwd), ("bwd", flops_bwd)):
-            if k in ktimes and ktimes[k][0] > 0:
-                kern[k]["tflops"] = round(sum(fl) * args.steps / (ktimes[k][0] * 1e-3) / 1e12, 2)
+        kt = {k: v for k, v in ktimes.items() if not k.startswith("_")}
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_per_step, 4),
-            "step_ms": {"median": round(statistics.median(step_times[0]), 4),
-                        "min": round(min(step_times[0]), 4), "rank": 0},
+            "step_ms": {"median": round(statistics.median(step_ms), 4),
+                        "min": round(min(step_ms), 4), "rank": 0},
             "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) d24-layer-shaped tensors)",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) tensors shaped like the workload's layers)",
             "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.T,
                        "parallelism": f"dp{world} (independent batch per GPU, no collective)",
                        "l2": "256 MiB buffer written between timed steps, outside the events",
@@ -334,17 +419,23 @@ def run_ours(args):
                 "measured_sustained": round(value / world / peaks.get("bf16_tflops_sustained", 1400.0), 4),
                 "nominal_dense": round(value / world / NOMINAL_BF16_TFLOPS, 4),
                 "peak_source": peak_src},
-            "roofline": roof,
-            "kernels": kern,
-            "gpu_launches": launches,
+            "roofline": roofline(kt, w, args.steps, peaks, peak_src),
+            "kernels": kernel_table(ktimes, w, args.steps),
+            "gpu_launches": sum(n for _, n in kt.values()),
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "h2d_bytes_per_step": st.h2d, "d2h_bytes_per_step": st.d2h,
                     "ms_per_step": round(e2e_ms / e2e_steps, 3)},
             "clocks": clk,
         }
-        if world == 1 and not args.no_decode and args.single_layer is None:
-            line["decode"] = decode_bench(w, dev, peaks, steps=args.steps, warmup=args.warmup)
-        if world == 1 and not args.no_cpu_baseline and args.single_layer is None:
+        solo = world == 1 and args.single_layer is None
+        if solo and not args.no_decode:
+            line["decode"] = decode_bench(w, dev, peaks, steps=args.steps, warmup=args.warmup,
+                                          peak_src=peak_src)
+        if solo and not args.no_other_configs:
+            del st
+            torch.cuda.empty_cache()
+            line["other_configs"] = other_configs(args, dev, peaks, peak_src, flush_buf, cs, synth)
+        if solo and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -355,7 +446,7 @@ def run_ours(args):
 DECODE_BATCH = 32  # sequences generating together
 
 
-def decode_bench(w, dev, peaks, steps=20, warmup=5):
+def decode_bench(w, dev, peaks, steps=20, warmup=5, peak_src="measured"):
     """One generation step over the workload's layer stack with a KV cache
     (attn_decode per layer): DECODE_BATCH sequences whose caches hold T-1
     tokens, so every layer reads its full window of K and V. HBM-bound: the
@@ -417,7 +508,7 @@ def decode_bench(w, dev, peaks, steps=20, warmup=5):
             "launches_per_step": kt["decode"][1] // steps * 2,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": nbytes,
-                         "peak_source": "measured hbm_gbs"}}
+                         "peak_source": f"{peak_src} hbm_gbs"}}
 
 
 def traffic_for(kind):
@@ -498,7 +589,7 @@ def cpu_baseline(w, budget_s=20.0):
             f2, d2, n = time_oracle_sample(w, n_layers=None)
             flops, dt, reps = flops + f2, dt + d2, reps + 1
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
-            "kind": "oracle", "seconds": round(dt, 2),
+            "cpu_model": cpu_model(), "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"float64 C oracle (prologue+fwd+bwd+chain rule), batch 1, one KV head "
                       f"with its {w.H // w.Hk} query heads, T={w.T}, first {n} of the layer windows "
                       f"{w.windows}, {reps} repetition(s); FLOPs counted as 12*D per unmasked pair"}
@@ -512,7 +603,7 @@ def run_reference(args):
     import causal_sliding_window_rope_b200 as cs
     import oracle
     oracle.build()
-    w = cs.WORKLOADS[CONFIG_ID]
+    w = cs.WORKLOADS[args.config]
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     for _ in range(args.warmup and 1):
         time_oracle_sample(w, n_layers=1)
@@ -528,7 +619,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_desc(w), "sample": "one KV head group, batch 1, first layer (S window)"},
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
-                             "kind": "oracle", "sample": "float64 C oracle, batch 1, one KV head group, one S layer per step"},
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": "float64 C oracle, batch 1, one KV head group, one S layer per step"},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -540,6 +631,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", type=int, choices=BF16_CONFIGS, default=DEFAULT_CONFIG,
+                    help="workload of the headline line (2: d12, 3: d12 SSSL, 4: d24 GQA SSSL, "
+                         "5: long-context GQA)")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the device-timed summary of the other bf16 workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
     ap.add_argument("--cpu-budget", type=float, default=20.0)

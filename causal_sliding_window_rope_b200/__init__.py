@@ -68,7 +68,7 @@ def lib():
         L.attn_bwd.argtypes = [lp] + [vp] * 7 + [fp, fp, vp, fp, vp] + [vp] * 6 + [sz, vp]
         L.cswattn_sync_status.argtypes = [vp]
         L.cswattn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
-        L.cswattn_set_wait_limit_ns.restype = None
+        L.cswattn_set_wait_limit_ns.restype = ctypes.c_uint64
         L.cswattn_last_error.restype = ctypes.c_char_p
         L.cswattn_set_timing.argtypes = [ctypes.c_int]
         L.cswattn_set_timing.restype = None
@@ -203,8 +203,9 @@ def cswattn_sync_status(stream=None):
     _check(lib().cswattn_sync_status(_stream(stream)))
 
 
-def cswattn_set_wait_limit_ns(ns: int):
-    lib().cswattn_set_wait_limit_ns(int(ns))
+def cswattn_set_wait_limit_ns(ns: int) -> int:
+    """Sets the device-side wait limit; returns the limit applied (>= 1 ms)."""
+    return int(lib().cswattn_set_wait_limit_ns(int(ns)))
 
 
 def cswattn_set_timing(enable: bool):

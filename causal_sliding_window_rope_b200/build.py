@@ -8,6 +8,7 @@ a machine that has no GPU driver.
 """
 from __future__ import annotations
 
+import glob
 import os
 import subprocess
 import sys
@@ -17,8 +18,15 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcswattn.so")
 SOURCES = ["cswattn.cu"]
-DEPS = ["common.cuh", "prologue.cuh", "simt_f32.cuh", "bwd_aux.cuh", "fwd_sm100.cuh",
-        "bwd_sm100.cuh", "cswattn.cu", os.path.join("..", "..", "include", "cswattn.h")]
+HEADER = os.path.join(ROOT, "include", "cswattn.h")
+
+
+def deps() -> list[str]:
+    """Every file the library is compiled from: the translation unit, every
+    kernel header next to it and the public header."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                  + [HEADER, os.path.abspath(__file__)])
+
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -39,7 +47,7 @@ def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(os.path.join(CSRC, d)) > t for d in DEPS)
+    return any(os.path.getmtime(d) > t for d in deps())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

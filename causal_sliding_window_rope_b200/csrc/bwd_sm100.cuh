@@ -94,16 +94,6 @@ struct Params {
   unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long ns) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > ns) {
-      atomicOr(&g_status, kStatusTimeout);
-      return;
-    }
-  }
-}
-
 // HD: head_dim, 128 or 64 (a 64-wide head leaves the second column panel
 // zero: its loads are filled with zeros, its products skipped where they
 // only add zeros, its stores and reductions not issued).
@@ -244,9 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++use;
         }
       }
-      drain_wait(kv_full, 0, p.wait_ns);
+      drain_wait(kv_full, 0);
       for (int s = 0; s < kQStages; ++s)
-        if (nq[s] > 0) drain_wait(&q_full[s], (nq[s] - 1) & 1, p.wait_ns);
+        if (nq[s] > 0) drain_wait(&q_full[s], (nq[s] - 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -327,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(acc_full);
       mma_commit(mma_done);
-      drain_wait(mma_done, 0, p.wait_ns);
+      drain_wait(mma_done, 0);
     }
   }
   } else if (warp < 8) {

@@ -104,6 +104,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Bound of the drain waits: before a CTA exits (and frees its TMEM) it waits
+// for the copies and matrix products it has issued, even after another wait
+// ran out. These waits do not take the caller's limit (which may be short):
+// a copy or product in flight completes within microseconds on a working
+// GPU, so only a GPU that no longer makes progress reaches this bound.
+constexpr unsigned long long kDrainLimitNs = 10000000000ull;  // 10 s
+
+// Waits for a phase without looking at the abort flag, bounded by
+// kDrainLimitNs; records a timeout if the bound is reached.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kDrainLimitNs) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- fences
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

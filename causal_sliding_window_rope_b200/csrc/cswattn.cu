@@ -27,6 +27,10 @@ namespace {
 
 thread_local std::string t_err;
 std::atomic<unsigned long long> g_wait_ns{2000000000ull};
+// Floor of the caller's wait limit: far above the latency of any copy, matrix
+// product or hand-off between a kernel's roles, so that a short limit only
+// ends waits that would not end otherwise.
+constexpr uint64_t kMinWaitNs = 1000000ull;  // 1 ms
 
 cswattn_status fail(cswattn_status s, const char* fmt, ...) {
   char buf[512];
@@ -239,15 +243,19 @@ RowLaunch row_launch(long long ntok, size_t per_tok) {
   return r;
 }
 
+// With prepare_only, sets what the launch needs (the shared-memory limit)
+// and launches nothing: a call that may fail is made before anything of an
+// entry point is enqueued.
 template <auto STAGED_K, auto DIRECT_K, typename P>
-cswattn_status launch_rows(P p, const RowLaunch& r, cudaStream_t st) {
+cswattn_status launch_rows(P p, const RowLaunch& r, cudaStream_t st, bool prepare_only) {
   p.wait_ns = g_wait_ns.load();
   if (r.tok > 0) {
     cswattn_status e = set_smem(STAGED_K, static_cast<int>(kRowStageMax));
-    if (e != CSWATTN_OK) return e;
+    if (e != CSWATTN_OK || prepare_only) return e;
     p.tok = r.tok;
     launch_pdl(STAGED_K, dim3(r.grid), dim3(kPrologueThreads), r.smem, st, p);
   } else {
+    if (prepare_only) return CSWATTN_OK;
     p.tok = kPrologueTok;
     launch_pdl(DIRECT_K, dim3(r.grid), dim3(kPrologueThreads), 0, st, p);
   }
@@ -258,7 +266,7 @@ template <typename T>
 cswattn_status launch_prologue(const Shape& s, const PrologueParams& pp, cudaStream_t st) {
   const RowLaunch r = row_launch(static_cast<long long>(s.B) * s.T,
                                  prologue_stage_bytes(1, s.H, s.Hk, s.D, s.esize, pp.has_ve != 0));
-#define CSW_ROWS(D_) launch_rows<prologue_kernel<T, D_, true>, prologue_kernel<T, D_, false>>(pp, r, st)
+#define CSW_ROWS(D_) launch_rows<prologue_kernel<T, D_, true>, prologue_kernel<T, D_, false>>(pp, r, st, false)
   switch (s.D) {
     case 4: if constexpr (sizeof(T) == 4) return CSW_ROWS(4); break;
     case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
@@ -272,10 +280,10 @@ cswattn_status launch_prologue(const Shape& s, const PrologueParams& pp, cudaStr
 }
 
 template <typename T>
-cswattn_status launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t st) {
+cswattn_status launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t st, bool prepare_only) {
   const RowLaunch r = row_launch(static_cast<long long>(s.B) * s.T,
                                  epilogue_stage_bytes(1, s.H, s.Hk, s.D, s.esize, ep.parts, ep.has_ve != 0));
-#define CSW_ROWS(D_) launch_rows<epilogue_kernel<T, D_, true>, epilogue_kernel<T, D_, false>>(ep, r, st)
+#define CSW_ROWS(D_) launch_rows<epilogue_kernel<T, D_, true>, epilogue_kernel<T, D_, false>>(ep, r, st, prepare_only)
   switch (s.D) {
     case 4: if constexpr (sizeof(T) == 4) return CSW_ROWS(4); break;
     case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
@@ -289,10 +297,10 @@ cswattn_status launch_epilogue(const Shape& s, const EpiParams& ep, cudaStream_t
 }
 
 template <typename T>
-cswattn_status launch_preprocess(const Shape& s, const PreParams& pp, cudaStream_t st) {
+cswattn_status launch_preprocess(const Shape& s, const PreParams& pp, cudaStream_t st, bool prepare_only) {
   const RowLaunch r = row_launch(static_cast<long long>(s.B) * s.T,
                                  preprocess_stage_bytes(1, s.H, s.D, s.esize));
-#define CSW_ROWS(D_) launch_rows<preprocess_kernel<T, D_, true>, preprocess_kernel<T, D_, false>>(pp, r, st)
+#define CSW_ROWS(D_) launch_rows<preprocess_kernel<T, D_, true>, preprocess_kernel<T, D_, false>>(pp, r, st, prepare_only)
   switch (s.D) {
     case 4: if constexpr (sizeof(T) == 4) return CSW_ROWS(4); break;
     case 8: if constexpr (sizeof(T) == 4) return CSW_ROWS(8); break;
@@ -456,27 +464,17 @@ Workspace carve(const Shape& s, void* base) {
 // device memory. Every GPU that loads this library holds it until exit.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[CSWATTN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
 // Device address of g_noalloc_scratch on the current device. In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with that device current and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// that device current, on every call: the lookup is a host-side table read
+// once the module is loaded, and a fresh lookup stays right after a device
+// reset gives the array a new address. (Under lazy module loading the first
+// lookup on a device loads the module, which reserves the array there.)
 cswattn_status noalloc_scratch(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices)
-    return fail(CSWATTN_ERR_UNSUPPORTED, "device ordinal %d is outside the scratch table", dev);
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+  *out = ptr;
   return CSWATTN_OK;
 }
 
@@ -533,7 +531,11 @@ int cswattn_version(void) { return (1 << 16) | 0; }
 
 const char* cswattn_last_error(void) { return t_err.c_str(); }
 
-void cswattn_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns < 1000 ? 1000 : ns); }
+uint64_t cswattn_set_wait_limit_ns(uint64_t ns) {
+  const uint64_t v = ns < kMinWaitNs ? kMinWaitNs : ns;
+  g_wait_ns.store(v);
+  return v;
+}
 
 cswattn_status cswattn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   if (limit_ns < 1000) limit_ns = 1000;
@@ -734,6 +736,7 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   if (workspace_bytes < w.bytes)
     return fail(CSWATTN_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes, w.bytes);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int parts = bwd_parts(s);
 
   // Delta = rowsum(dO * O)
   PreParams pre;
@@ -748,9 +751,74 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   pre.lse2 = w.lse2;
   // The tensor-core backward accumulates dq~ with reductions: zero it here.
   pre.dq_zero = s.bf16 ? w.dq_acc : nullptr;
+
+  EpiParams ep;
+  ep.B = s.B;
+  ep.T = s.T;
+  ep.H = s.H;
+  ep.Hk = s.Hk;
+  ep.has_ve = layer->has_ve;
+  fill_omega(ep.omega, s.D, layer->rope_base);
+  ep.q = q;
+  ep.k = k;
+  ep.ve = ve;
+  ep.gate = gate;
+  ep.rstd_q = rstd_q;
+  ep.rstd_k = rstd_k;
+  ep.dq_acc = w.dq_acc;
+  ep.dk_acc = w.dk_acc;
+  ep.dv_acc = w.dv_acc;
+  ep.parts = parts;
+  ep.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
+  ep.dq = dQ;
+  ep.dk = dK;
+  ep.dv = dV;
+  ep.dve = dve;
+  ep.dgate = dgate;
+
+  // Everything that can fail short of a launch (tensor maps, shared-memory
+  // limits) is done before the first kernel is enqueued, so that a rejected
+  // call leaves the stream untouched.
+  CUtensorMap mq, mdo, mk, mv, mdk, mdv, mdq;
+  bwd::Params bp{};
+  if (s.bf16) {
+    if ((st = make_map(&mq, q_out, s.B, s.T, s.H, bwd::kBQ, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdo, dO, s.B, s.T, s.H, bwd::kBQ, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, bwd::kBN, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, bwd::kBN, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdk, w.dk_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
+    if ((st = make_map(&mdq, w.dq_acc, s.B, s.T, s.H, bwd::kBQ, s.D, true)) != CSWATTN_OK) return st;
+    if ((st = s.D == 64 ? set_smem(bwd::bwd_kernel<64>, bwd::kSmemBytes)
+                        : set_smem(bwd::bwd_kernel<128>, bwd::kSmemBytes)) != CSWATTN_OK)
+      return st;
+    bp.B = s.B;
+    bp.T = s.T;
+    bp.H = s.H;
+    bp.Hk = s.Hk;
+    bp.W = s.W;
+    bp.g = s.g;
+    bp.nkv = (s.T + bwd::kBN - 1) / bwd::kBN;
+    bp.scale_log2 = s.scale * 1.4426950408889634f;
+    bp.scale = s.scale;
+    bp.Tpad = w.Tpad;
+    bp.lse2 = w.lse2;
+    bp.delta = w.delta;
+    bp.dq_acc = w.dq_acc;
+    bp.dk_acc = w.dk_acc;
+    bp.dv_acc = w.dv_acc;
+    bp.parts = parts;
+    bp.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
+    bp.wait_ns = g_wait_ns.load();
+  }
+  st = s.bf16 ? launch_preprocess<__nv_bfloat16>(s, pre, cs, true) : launch_preprocess<float>(s, pre, cs, true);
+  if (st != CSWATTN_OK) return st;
+  st = s.bf16 ? launch_epilogue<__nv_bfloat16>(s, ep, cs, true) : launch_epilogue<float>(s, ep, cs, true);
+  if (st != CSWATTN_OK) return st;
+
   {
     ScopedTiming tm(CSWATTN_K_BWD_PRE, cs);
-    st = s.bf16 ? launch_preprocess<__nv_bfloat16>(s, pre, cs) : launch_preprocess<float>(s, pre, cs);
+    st = s.bf16 ? launch_preprocess<__nv_bfloat16>(s, pre, cs, false) : launch_preprocess<float>(s, pre, cs, false);
   }
   if (st != CSWATTN_OK) return st;
   if ((st = launched("preprocess launch")) != CSWATTN_OK) return st;
@@ -780,39 +848,6 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     }
     if ((st = launched("fp32 backward launch")) != CSWATTN_OK) return st;
   } else {
-    CUtensorMap mq, mdo, mk, mv;
-    if ((st = make_map(&mq, q_out, s.B, s.T, s.H, bwd::kBQ, s.D)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mdo, dO, s.B, s.T, s.H, bwd::kBQ, s.D)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mk, k_out, s.B, s.T, s.Hk, bwd::kBN, s.D)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mv, v_out, s.B, s.T, s.Hk, bwd::kBN, s.D)) != CSWATTN_OK) return st;
-    const int parts = bwd_parts(s);
-    CUtensorMap mdk, mdv;
-    if ((st = make_map(&mdk, w.dk_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
-    if ((st = make_map(&mdv, w.dv_acc, s.B * parts, s.T, s.Hk, bwd::kBN, s.D, true)) != CSWATTN_OK) return st;
-    CUtensorMap mdq;
-    if ((st = make_map(&mdq, w.dq_acc, s.B, s.T, s.H, bwd::kBQ, s.D, true)) != CSWATTN_OK) return st;
-    if ((st = s.D == 64 ? set_smem(bwd::bwd_kernel<64>, bwd::kSmemBytes)
-                        : set_smem(bwd::bwd_kernel<128>, bwd::kSmemBytes)) != CSWATTN_OK)
-      return st;
-    bwd::Params bp;
-    bp.B = s.B;
-    bp.T = s.T;
-    bp.H = s.H;
-    bp.Hk = s.Hk;
-    bp.W = s.W;
-    bp.g = s.g;
-    bp.nkv = (s.T + bwd::kBN - 1) / bwd::kBN;
-    bp.scale_log2 = s.scale * 1.4426950408889634f;
-    bp.scale = s.scale;
-    bp.Tpad = w.Tpad;
-    bp.lse2 = w.lse2;
-    bp.delta = w.delta;
-    bp.dq_acc = w.dq_acc;
-    bp.dk_acc = w.dk_acc;
-    bp.dv_acc = w.dv_acc;
-    bp.parts = parts;
-    bp.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
-    bp.wait_ns = g_wait_ns.load();
     const unsigned grid = static_cast<unsigned>(bp.nkv) * bp.parts * s.B * s.Hk;
     {
       ScopedTiming tm(CSWATTN_K_BWD, cs);
@@ -826,32 +861,9 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     if ((st = launched("backward launch")) != CSWATTN_OK) return st;
   }
 
-  EpiParams ep;
-  ep.B = s.B;
-  ep.T = s.T;
-  ep.H = s.H;
-  ep.Hk = s.Hk;
-  ep.has_ve = layer->has_ve;
-  fill_omega(ep.omega, s.D, layer->rope_base);
-  ep.q = q;
-  ep.k = k;
-  ep.ve = ve;
-  ep.gate = gate;
-  ep.rstd_q = rstd_q;
-  ep.rstd_k = rstd_k;
-  ep.dq_acc = w.dq_acc;
-  ep.dk_acc = w.dk_acc;
-  ep.dv_acc = w.dv_acc;
-  ep.parts = bwd_parts(s);
-  ep.kv_stride = static_cast<long long>(s.B) * s.T * s.Hk * s.D;
-  ep.dq = dQ;
-  ep.dk = dK;
-  ep.dv = dV;
-  ep.dve = dve;
-  ep.dgate = dgate;
   {
     ScopedTiming tm(CSWATTN_K_BWD_EPI, cs);
-    st = s.bf16 ? launch_epilogue<__nv_bfloat16>(s, ep, cs) : launch_epilogue<float>(s, ep, cs);
+    st = s.bf16 ? launch_epilogue<__nv_bfloat16>(s, ep, cs, false) : launch_epilogue<float>(s, ep, cs, false);
   }
   if (st != CSWATTN_OK) return st;
   return launched("epilogue launch");

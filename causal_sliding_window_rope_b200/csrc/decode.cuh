@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
       ok = mbar_try_wait(&bar, 0);
       if (!ok && globaltimer() - t0 > p.wait_ns) {
         atomicOr(&g_status, kStatusTimeout);
+        drain_wait(&bar, 0);  // the tile copies land before the CTA exits
         break;
       }
     }

@@ -62,18 +62,6 @@ struct Params {
   unsigned long long wait_ns;
 };
 
-// Waits for a phase without looking at the abort flag (used to drain
-// in-flight copies and MMAs before the CTA exits). Bounded by `ns`.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned long long ns) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > ns) {
-      atomicOr(&g_status, kStatusTimeout);
-      return;
-    }
-  }
-}
-
 // HD: head_dim, 128 or 64 (a 64-wide head leaves the second column panel
 // zero: its loads are filled with zeros, its products skipped, its stores
 // not issued).
@@ -190,9 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Drain: every issued copy has landed before the CTA may exit.
-      drain_wait(q_full, 0, p.wait_ns);
+      drain_wait(q_full, 0);
       for (int s2 = 0; s2 < kSlots; ++s2)
-        if (filled[s2] > 0) drain_wait(&kv_full[s2], (filled[s2] - 1) & 1, p.wait_ns);
+        if (filled[s2] > 0) drain_wait(&kv_full[s2], (filled[s2] - 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -276,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: all issued MMAs complete before TMEM is released.
       mma_commit(mma_done);
-      drain_wait(mma_done, 0, p.wait_ns);
+      drain_wait(mma_done, 0);
     }
   }
   } else {

@@ -203,12 +203,16 @@ struct Stage {
   __device__ void copy(void* dst, const void* src, uint32_t bytes) const {
     bulk_load(dst, src, bytes, bar);
   }
+  // On a timeout the copies may still be in flight: wait for them (with the
+  // fixed drain bound) before the CTA returns, so that none lands in the
+  // shared memory of a later CTA.
   __device__ bool wait(unsigned long long limit_ns) const {
     if (mbar_try_wait(bar, 0)) return true;
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait(bar, 0)) {
       if (globaltimer() - t0 > limit_ns) {
         atomicOr(&g_status, kStatusTimeout);
+        drain_wait(bar, 0);
         return false;
       }
     }

@@ -148,10 +148,15 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
  * the library holds it until the process exits. Layers whose
  * attn_bwd_workspace_bytes() exceeds that size are rejected with
  * CSWATTN_ERR_UNSUPPORTED before anything is enqueued (use attn_bwd with
- * your own workspace for those). No call allocates device memory.
- * The first call on a device looks up the array's device address on that
- * device (the device current at the call); make that first call before
- * any stream capture. All calls on a device share the one array: two calls
+ * your own workspace for those). No call allocates device memory
+ * through cudaMalloc or any allocator: the array is part of the library's
+ * device code. Under lazy module loading (the CUDA default) that code, and
+ * with it the array, is loaded onto a device by the first call of this
+ * library there, which may synchronize that device; make one warm-up call
+ * on each device outside the step loop and before any stream capture.
+ * Every call looks up the array's address on the device current at the
+ * call (a host-side lookup), so the entry point keeps working after a
+ * device reset. All calls on a device share the one array: two calls
  * that may overlap on the GPU (different streams, no ordering between
  * them) race and corrupt each other's results, so order them, for example
  * by issuing them on one stream. The array keeps whatever the last call
@@ -208,9 +213,13 @@ cswattn_status cswattn_sync_status(void* stream);
  * reports (and clears) it. Touches no TMEM and issues no copies. */
 cswattn_status cswattn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
-/* Upper bound, in nanoseconds, of every device-side wait of later launches
- * (default 2e9). Values below 1000 are raised to 1000. Process-wide. */
-void cswattn_set_wait_limit_ns(uint64_t ns);
+/* Upper bound, in nanoseconds, of the device-side waits of later launches
+ * on each other's progress (default 2e9); returns the limit applied. Values
+ * below 1e6 (1 ms) are raised to 1e6. Process-wide. This limit does not
+ * bound a kernel's final waits for its own copies and matrix products in
+ * flight (they have a fixed bound of 10 s), so a short limit never lets a
+ * kernel exit, or free its tensor memory, while they are still running. */
+uint64_t cswattn_set_wait_limit_ns(uint64_t ns);
 
 /* Kernel kinds reported by cswattn_kernel_times(). */
 enum {

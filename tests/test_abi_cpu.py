@@ -23,7 +23,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"^\s*(?:cswattn_status|size_t|void|const char\s*\*|int)\s+(\w+)\s*\(",
+    names = re.findall(r"^\s*(?:cswattn_status|size_t|uint64_t|void|const char\s*\*|int)\s+(\w+)\s*\(",
                        text, flags=re.M)
     return sorted(set(names))
 
@@ -159,3 +159,41 @@ def test_header_enums_match_the_binding():
     kinds = re.findall(r"CSWATTN_K_(\w+)\s*=\s*(\d+)", text)
     assert [k.lower() for k, _ in sorted(kinds, key=lambda kv: int(kv[1]))] == list(cs.KERNEL_KINDS)
     assert int(re.search(r"CSWATTN_NUM_KERNELS\s*=\s*(\d+)", text).group(1)) == len(cs.KERNEL_KINDS)
+
+
+def test_wait_limit_floor(lib):
+    # Short limits are raised to 1 ms, far above any copy or product latency;
+    # the kernels' final waits for their own copies have a fixed bound.
+    assert cs.cswattn_set_wait_limit_ns(5) == 1_000_000
+    assert cs.cswattn_set_wait_limit_ns(999_999) == 1_000_000
+    assert cs.cswattn_set_wait_limit_ns(3_000_000) == 3_000_000
+    assert cs.cswattn_set_wait_limit_ns(2_000_000_000) == 2_000_000_000
+
+
+def test_build_tracks_every_kernel_source(tmp_path, monkeypatch):
+    """Editing any kernel header, the translation unit or the public header
+    makes the library stale, so build() recompiles it."""
+    import shutil
+    csrc = tmp_path / "csrc"
+    shutil.copytree(cs_build.CSRC, csrc)
+    header = tmp_path / "cswattn.h"
+    shutil.copy(cs_build.HEADER, header)
+    libf = tmp_path / "libcswattn.so"
+    libf.write_bytes(b"")
+    monkeypatch.setattr(cs_build, "CSRC", str(csrc))
+    monkeypatch.setattr(cs_build, "HEADER", str(header))
+    monkeypatch.setattr(cs_build, "LIB", str(libf))
+    deps = cs_build.deps()
+    names = {os.path.basename(d) for d in deps}
+    assert {"decode.cuh", "bwd_sm100.cuh", "fwd_sm100.cuh", "cswattn.cu", "cswattn.h"} <= names
+    copied = [d for d in deps if d.startswith(str(tmp_path))]  # never touch the real tree
+    assert len(copied) == len(deps) - 1
+    t_lib = 2_000_000_000
+    for d in copied:
+        os.utime(d, (t_lib - 10, t_lib - 10))
+    os.utime(libf, (t_lib, t_lib))
+    assert not cs_build.stale()
+    for d in copied:
+        os.utime(d, (t_lib + 10, t_lib + 10))
+        assert cs_build.stale(), d
+        os.utime(d, (t_lib - 10, t_lib - 10))

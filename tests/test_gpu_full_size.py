@@ -31,7 +31,10 @@ def query_rows(B, H, T, rng):
 
 
 def key_rows(B, Hk, T, W, rng):
-    pts = {T - 1, T - 2, T - 128, T - 129}
+    """Key rows at the sequence end, in the middle of windowed layers, and in
+    the first key tiles: keys 0..129 are seen by every query of a full-causal
+    layer (the heaviest tiles, whose steps the backward splits into parts)."""
+    pts = {0, 1, 63, 64, 127, 128, 129, T - 1, T - 2, T - 128, T - 129}
     if W < T:
         pts.add(T // 2 + 3)
     rows = []
@@ -76,6 +79,7 @@ def test_full_size_layer_stack(config):
         qt, kt, veff, rq, rk = oracle.prologue(L, x["q"], x["k"], x["v"], x["ve"], x["gate"])
         assert rel_frob(got["qt"], qt) < TOL and rel_frob(got["kt"], kt) < TOL
         assert rel_frob(got["veff"], veff) < TOL and rel_frob(got["rstd_q"], rq) < TOL
+        assert rel_frob(got["rstd_k"], rk) < TOL
 
         qr = query_rows(w.B, w.H, w.T, rng)
         O, lse = oracle.fwd_rows(L, qt, kt, veff, qr)
