@@ -59,6 +59,7 @@ constexpr int kOffDS = kOffQD + kQStages * kStageBytes;  // dS^T [2]
 // dQ^T drain staging: 4 panels of 64 query rows x 32 float32 (128B-swizzled).
 constexpr int kOffDQS = kOffDS + 2 * kPBytes;
 constexpr int kDQPanel = kBQ * 128;
+constexpr int kDQHalf = kDQPanel / 2;  // one panel of 32 query rows
 constexpr int kOffBar = kOffDQS + 4 * kDQPanel;
 // dK/dV write-out staging over the Q/dO ring and dS^T buffers: 2 x 4 panels
 // of 128 rows x 32 float32.
@@ -121,8 +122,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
   uint64_t* kv_staged = bars + 20;  // dK/dV rows written to shared memory
-  uint64_t* dqs_full = bars + 21;   // dQ^T staging tile written (128 arrivals)
-  uint64_t* dqs_free = bars + 22;   // the reduction has read the staging tile
+  uint64_t* dqs_full = bars + 21;   // [2] half of the dQ staging tile written (128 arrivals)
+  uint64_t* dqs_free = bars + 23;   // [2] the reduction has read that half
   float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [kQStages][64]
   float* s_delta = s_lse2 + kQStages * kBQ;                         // [kQStages][64]
 
@@ -162,8 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(kv_staged, 128);
-    mbar_init(dqs_full, 128);
-    mbar_init(dqs_free, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&dqs_full[s], 128);
+      mbar_init(&dqs_free[s], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -468,33 +471,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&dq_empty[st]);
-      // Column q of dQ^T is row q of the step's dQ~ tile: stage it in four
-      // 32-column panels (128B-swizzled; the warp's 32 lanes fill one
-      // 128-byte row, conflict-free) and add the tile into dq_acc with four
-      // TMA reductions (rows past T are skipped).
-      got = n == 0 || mbar_wait(dqs_free, (n - 1) & 1, wc);
-      if (!__all_sync(0xffffffffu, got)) break;
-      uint8_t* prow = stile + (d >> 5) * kDQPanel + (d & 3) * 4;
+      // Column q of dQ^T is row q of the step's dQ~ tile. The tile goes out
+      // in two halves of 32 query rows (hq), each staged as four 32-column
+      // float32 panels (128B-swizzled; the warp's 32 lanes fill one 128-byte
+      // row, conflict-free) and added into dq_acc by four TMA reductions
+      // (rows past T are skipped). A half is restaged only once the
+      // reduction of its previous use has read it, so the reduction of one
+      // half overlaps the staging of the other.
       const int chunk = (d & 31) >> 2;
+      bool step_ok = true;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int q = cc * 32 + i;
-          *reinterpret_cast<float*>(prow + q * 128 + ((chunk ^ (q & 7)) << 4)) = __uint_as_float(a[cc][i]) * sc;
+      for (int hq = 0; hq < 2; ++hq) {
+        // Half hq of step n-1 has been read: signalled once per step.
+        got = n == 0 || mbar_wait(&dqs_free[hq], (n - 1) & 1, wc);
+        if (!__all_sync(0xffffffffu, got)) {
+          step_ok = false;
+          break;
         }
-      fence_proxy_async_smem();
-      mbar_arrive(dqs_full);
-      if (leader) {
-        if (mbar_wait(dqs_full, n & 1, wc)) {
+        uint8_t* prow = stile + hq * (4 * kDQHalf) + (d >> 5) * kDQHalf + (d & 3) * 4;
 #pragma unroll
-          for (int pc = 0; pc < 4; ++pc)
-            if (32 * pc < HD) tma_reduce_add_4d(&tmDQ, stile + pc * kDQPanel, 32 * pc, h, q0, b);
+        for (int i = 0; i < 32; ++i)
+          *reinterpret_cast<float*>(prow + i * 128 + ((chunk ^ (i & 7)) << 4)) = __uint_as_float(a[hq][i]) * sc;
+        fence_proxy_async_smem();
+        mbar_arrive(&dqs_full[hq]);
+        if (leader) {
+          if (mbar_wait(&dqs_full[hq], n & 1, wc)) {
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc)
+              if (32 * pc < HD)
+                tma_reduce_add_4d(&tmDQ, stile + hq * (4 * kDQHalf) + pc * kDQHalf, 32 * pc, h, q0 + 32 * hq, b);
+          }
           bulk_commit();
-          bulk_wait_read0();
+          // Every group but this one has been read: the other half's
+          // previous use (half 1 of step n-1, or half 0 of this step).
+          bulk_wait_read1();
+          if (hq == 1 || n > 0) mbar_arrive(&dqs_free[hq ^ 1]);
         }
-        mbar_arrive(dqs_free);
       }
+      if (!step_ok) break;
     }
     if (leader) bulk_wait_read0();  // shared source read; the writes finish on their own
   }
