@@ -184,29 +184,6 @@ cswattn_status set_smem(Kernel k, int bytes) {
   return CSWATTN_OK;
 }
 
-// Number of SMs of the current device (the persistent kernels launch one
-// CTA per SM), looked up once per device.
-cswattn_status sm_count(int* out) {
-  static std::mutex mu;
-  static std::vector<std::pair<int, int>> known;  // (device, SMs)
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  std::lock_guard<std::mutex> lock(mu);
-  for (const auto& k : known)
-    if (k.first == dev) {
-      *out = k.second;
-      return CSWATTN_OK;
-    }
-  int n = 0;
-  e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  if (n < 1) return fail(CSWATTN_ERR_CUDA, "device reports %d SMs", n);
-  known.emplace_back(dev, n);
-  *out = n;
-  return CSWATTN_OK;
-}
-
 // First failed launch of the current call on this thread, reported (and
 // cleared) by launched().
 thread_local cudaError_t t_launch_error = cudaSuccess;
