@@ -69,6 +69,9 @@ def _get():
         _lib.oracle_probs_row.argtypes = [L, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp]
         _lib.oracle_probs_row.restype = ctypes.c_double
         _lib.oracle_decode.argtypes = [L] + [dp] * 5 + [ip] + [dp] * 4
+        ci = ctypes.c_int
+        _lib.oracle_gate_logits.argtypes = [ci] * 5 + [dp] * 3
+        _lib.oracle_gate_bwd.argtypes = [ci] * 5 + [dp] * 5
     return _lib
 
 
@@ -243,3 +246,28 @@ def decode(L: Layer, q, k, v, ve, gate, lens, kcache, vcache):
     _get().oracle_decode(L.c(), _p(q), _p(k), _p(v), _p(ve), _p(gate),
                          lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), _p(kc), _p(vc), _p(O), _p(lse))
     return O, lse, kc, vc
+
+
+def gate_logits(x, w, C):
+    """Gate logits of the value-embedding gate: x[..., :C] @ w.T, x (B, T, X)
+    with X >= C, w (Hk, C); returns (B, T, Hk)."""
+    x = _f64(x)
+    w = _f64(w)
+    B, T, X = x.shape
+    Hk = w.shape[0]
+    if w.shape[1] != C or X < C:
+        raise ValueError("w must be (Hk, C) and x must have at least C channels")
+    out = np.empty((B, T, Hk))
+    _get().oracle_gate_logits(B, T, Hk, C, X, _p(x), _p(w), _p(out))
+    return out
+
+
+def gate_bwd(x, w, C, dgate):
+    """dx (B, T, C) and dw (Hk, C) of the gate projection given dL/dgate."""
+    x, w, dgate = _f64(x), _f64(w), _f64(dgate)
+    B, T, X = x.shape
+    Hk = w.shape[0]
+    dx = np.empty((B, T, C))
+    dw = np.empty((Hk, C))
+    _get().oracle_gate_bwd(B, T, Hk, C, X, _p(x), _p(w), _p(dgate), _p(dx), _p(dw))
+    return dx, dw

@@ -443,3 +443,41 @@ void oracle_decode(const oracle_layer *L, const double *q, const double *k,
     free(qt);
   }
 }
+
+/* The value-embedding gate's projection: page "5만원으로 나만의 ChatGPT
+ * 훈련하는 방법", section "1. GPT 모델", value-embedding code: the gate is a
+ * linear map (no bias: the page shows none) of the first C channels of the
+ * block input x, one output per KV head, before 3*sigmoid(.):
+ *   gate[b,t,h] = sum_{c<C} x[b,t,c] w[h,c].
+ * x (B, T, ldx) with ldx >= C (only the first C entries of a row are read);
+ * w (Hk, C); gate (B, T, Hk). */
+void oracle_gate_logits(int B, int T, int Hk, int C, int ldx, const double *x,
+                        const double *w, double *gate) {
+  for (long n = 0; n < (long)B * T; ++n)
+    for (int h = 0; h < Hk; ++h) {
+      double s = 0.0;
+      for (int c = 0; c < C; ++c) s += x[n * ldx + c] * w[(long)h * C + c];
+      gate[n * Hk + h] = s;
+    }
+}
+
+/* Its backward, given dgate = dL/dgate (B, T, Hk):
+ *   dx[b,t,c] = sum_h dgate[b,t,h] w[h,c]   (dx (B, T, C): the first C
+ *                                            channels of x; the rest get 0)
+ *   dw[h,c]   = sum_{b,t} dgate[b,t,h] x[b,t,c]. */
+void oracle_gate_bwd(int B, int T, int Hk, int C, int ldx, const double *x,
+                     const double *w, const double *dgate, double *dx,
+                     double *dw) {
+  for (long n = 0; n < (long)B * T; ++n)
+    for (int c = 0; c < C; ++c) {
+      double s = 0.0;
+      for (int h = 0; h < Hk; ++h) s += dgate[n * Hk + h] * w[(long)h * C + c];
+      dx[n * C + c] = s;
+    }
+  for (int h = 0; h < Hk; ++h)
+    for (int c = 0; c < C; ++c) {
+      double s = 0.0;
+      for (long n = 0; n < (long)B * T; ++n) s += dgate[n * Hk + h] * x[n * ldx + c];
+      dw[(long)h * C + c] = s;
+    }
+}

@@ -355,3 +355,72 @@ def test_decode_window_one_returns_own_value():
             hk = h // (L.H // L.Hk)
             np.testing.assert_allclose(Od[b, h], veff[b, p, hk], rtol=0, atol=1e-12)
             assert abs(lsed[b, h] - L.scale * float(qt[b, p, h] @ kt[b, p, hk])) < 1e-12
+
+
+# ---------------------------------------------------------------- value-embedding gate projection
+
+def test_gate_projection_hand_worked():
+    """Gate logits and their gradients on a hand-worked token (derivation in
+    the fixture)."""
+    with open(os.path.join(GOLDEN, "gate_by_hand.json")) as f:
+        g = json.load(f)
+    x = np.array(g["x"]).reshape(1, 1, 3)
+    w = np.array(g["w"])
+    logits = oracle.gate_logits(x, w, g["C"])
+    np.testing.assert_allclose(logits.reshape(2), g["logits"], atol=1e-15)
+    dx, dw = oracle.gate_bwd(x, w, g["C"], np.array(g["dgate"]).reshape(1, 1, 2))
+    np.testing.assert_allclose(dx.reshape(2), g["dx"], atol=1e-15)
+    np.testing.assert_allclose(dw, g["dw"], atol=1e-15)
+
+
+def test_gate_projection_matches_torch_linear_and_autograd():
+    """Against torch's float64 linear map and its autograd (library routines
+    the oracle does not use)."""
+    B, T, X, C, Hk = 2, 5, 9, 6, 3
+    x = rnd((B, T, X), 70)
+    w = rnd((Hk, C), 71)
+    dg = rnd((B, T, Hk), 72)
+    xt = torch.tensor(x, requires_grad=True)
+    wt = torch.tensor(w, requires_grad=True)
+    out = F.linear(xt[..., :C], wt)
+    np.testing.assert_allclose(oracle.gate_logits(x, w, C), out.detach().numpy(), atol=1e-13)
+    out.backward(torch.tensor(dg))
+    dx, dw = oracle.gate_bwd(x, w, C, dg)
+    np.testing.assert_allclose(dx, xt.grad.numpy()[..., :C], atol=1e-13)
+    assert np.all(xt.grad.numpy()[..., C:] == 0)  # channels past C are not read
+    np.testing.assert_allclose(dw, wt.grad.numpy(), atol=1e-13)
+
+
+def test_gate_projection_gradients_match_central_differences():
+    """The whole layer with its gate computed from x and w: dL/dx and dL/dw
+    of L = sum(O * dO) from the layer's dgate through the projection's
+    backward, against central differences of L itself."""
+    L = oracle.Layer(1, 12, 4, 2, 6, 5, has_ve=True)
+    q, k, v, ve, _, dO = inputs(L, 77)
+    C, X = 4, 7
+    x = rnd((1, L.T, X), 78)
+    w = rnd((L.Hk, C), 79)
+
+    def loss(x_, w_):
+        return _loss(L, q, k, v, ve, oracle.gate_logits(x_, w_, C), dO)
+
+    gate = oracle.gate_logits(x, w, C)
+    dgate = oracle.layer(L, q, k, v, ve, gate, dO)["dgate"]
+    dx, dw = oracle.gate_bwd(x, w, C, dgate)
+    h = 1e-6
+    rng = np.random.default_rng(5)
+    for _ in range(10):
+        t, c = int(rng.integers(0, L.T)), int(rng.integers(0, X))
+        xp, xm = x.copy(), x.copy()
+        xp[0, t, c] += h
+        xm[0, t, c] -= h
+        fd = (loss(xp, w) - loss(xm, w)) / (2 * h)
+        an = dx[0, t, c] if c < C else 0.0
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), ("x", t, c, fd, an)
+    for hh in range(L.Hk):
+        for c in range(C):
+            wp, wm = w.copy(), w.copy()
+            wp[hh, c] += h
+            wm[hh, c] -= h
+            fd = (loss(x, wp) - loss(x, wm)) / (2 * h)
+            assert abs(fd - dw[hh, c]) <= 1e-6 * max(1.0, abs(dw[hh, c])), ("w", hh, c, fd, dw[hh, c])
