@@ -271,3 +271,34 @@ def gate_bwd(x, w, C, dgate):
     dw = np.empty((Hk, C))
     _get().oracle_gate_bwd(B, T, Hk, C, X, _p(x), _p(w), _p(dgate), _p(dx), _p(dw))
     return dx, dw
+
+
+# ---------------------------------------------------------------- Muon orthogonalisation
+
+# The coefficient triples (a, b, c) the page prints for the first two steps of
+# the "Polar Express" iteration (page "5만원으로 나만의 ChatGPT 훈련하는 방법",
+# section "2. Muon 옵티마이저 (nanochat/optim.py)"); the rest of its list is
+# elided there, so callers pass the triples they want to apply.
+POLAR_EXPRESS_PRINTED = ((8.156, -22.483, 15.879), (4.043, -2.809, 0.500))
+
+
+def newton_schulz(X, coeffs):
+    """The quintic Newton-Schulz iteration of the same section, in float64,
+    one step per (a, b, c) triple, in the page's order and notation:
+        A = X^T X;  B = b A + c A A;  X = a X + X B.
+    X is (m, n); returns the iterate after len(coeffs) steps."""
+    X = np.array(X, dtype=np.float64, copy=True)
+    for a, b, c in coeffs:
+        A = X.T @ X
+        B = b * A + c * (A @ A)
+        X = a * X + X @ B
+    return X
+
+
+def gemm(A, B, alpha=1.0, D=None, beta=0.0):
+    """C = alpha A B + beta D in float64 (the product the iteration's steps
+    are made of)."""
+    C = alpha * (np.asarray(A, np.float64) @ np.asarray(B, np.float64))
+    if D is not None and beta != 0.0:
+        C = C + beta * np.asarray(D, np.float64)
+    return C

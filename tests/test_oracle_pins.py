@@ -424,3 +424,57 @@ def test_gate_projection_gradients_match_central_differences():
             wm[hh, c] -= h
             fd = (loss(x, wp) - loss(x, wm)) / (2 * h)
             assert abs(fd - dw[hh, c]) <= 1e-6 * max(1.0, abs(dw[hh, c])), ("w", hh, c, fd, dw[hh, c])
+
+
+# ---------------------------------------------------------------- Muon Newton-Schulz
+
+COEFFS = oracle.POLAR_EXPRESS_PRINTED
+
+
+def test_newton_schulz_scalar_closed_form():
+    """On a 1 x 1 matrix every step is the quintic x -> a x + b x^3 + c x^5."""
+    x = 0.37
+    want = x
+    for a, b, c in COEFFS:
+        want = a * want + b * want ** 3 + c * want ** 5
+    got = oracle.newton_schulz(np.array([[x]]), COEFFS)
+    assert abs(got[0, 0] - want) < 1e-15
+
+
+def test_newton_schulz_acts_on_singular_values():
+    """X = U S V^T maps to U p(S) V^T with p the composed quintic (numpy's
+    SVD, a routine the oracle does not use)."""
+    X = rnd((7, 5), 90)
+    X /= np.linalg.norm(X)
+    U, S, Vt = np.linalg.svd(X, full_matrices=False)
+    for a, b, c in COEFFS:
+        S = a * S + b * S ** 3 + c * S ** 5
+    np.testing.assert_allclose(oracle.newton_schulz(X, COEFFS), (U * S) @ Vt, atol=1e-12)
+
+
+def test_newton_schulz_orthogonal_equivariance_and_transpose():
+    """NS(P X Q) = P NS(X) Q for orthogonal P, Q, and NS(X^T) = NS(X)^T."""
+    X = rnd((6, 4), 91) / 4.0
+    P, _ = np.linalg.qr(rnd((6, 6), 92))
+    Q, _ = np.linalg.qr(rnd((4, 4), 93))
+    Y = oracle.newton_schulz(X, COEFFS)
+    np.testing.assert_allclose(oracle.newton_schulz(P @ X @ Q, COEFFS), P @ Y @ Q, atol=1e-12)
+    np.testing.assert_allclose(oracle.newton_schulz(X.T, COEFFS), Y.T, atol=1e-12)
+
+
+def test_newton_schulz_one_step_by_hand():
+    """One step on a diagonal 2 x 2 matrix, worked by hand: A = diag(x^2),
+    B = diag(b x^2 + c x^4), X' = diag(a x + b x^3 + c x^5)."""
+    a, b, c = 2.0, -1.0, 0.5
+    X = np.diag([1.0, 0.5])
+    want = np.diag([2.0 - 1.0 + 0.5, 1.0 - 0.125 + 0.015625])
+    np.testing.assert_allclose(oracle.newton_schulz(X, [(a, b, c)]), want, atol=1e-15)
+
+
+def test_gemm_matches_explicit_sums():
+    A, B, D = rnd((3, 4), 94), rnd((4, 2), 95), rnd((3, 2), 96)
+    C = oracle.gemm(A, B, 0.5, D, -2.0)
+    for i in range(3):
+        for j in range(2):
+            s = sum(A[i, k] * B[k, j] for k in range(4))
+            assert abs(C[i, j] - (0.5 * s - 2.0 * D[i, j])) < 1e-13
