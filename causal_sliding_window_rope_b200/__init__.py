@@ -25,12 +25,14 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
 
 # Every symbol the header declares; the CPU tests check the library exports them.
-EXPORTS = ("attn_prologue", "attn_fwd", "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
-           "attn_decode_workspace_bytes", "attn_decode",
+EXPORTS = ("attn_prologue", "attn_prologue_gated", "attn_gate_bwd", "attn_fwd",
+           "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
+           "attn_decode_workspace_bytes", "attn_decode", "cswattn_gemm_bf16",
+           "muon_ns_workspace_bytes", "muon_newton_schulz",
            "cswattn_sync_status", "cswattn_set_wait_limit_ns", "cswattn_set_timing",
            "cswattn_kernel_times", "cswattn_selftest_wait_timeout", "cswattn_last_error",
            "cswattn_version")
-KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi", "decode")
+KERNEL_KINDS = ("prologue", "fwd", "bwd_pre", "bwd", "bwd_epi", "decode", "gate_bwd", "gemm")
 
 
 class CswattnLayer(ctypes.Structure):
@@ -63,6 +65,16 @@ def lib():
         lp = ctypes.POINTER(CswattnLayer)
         L.attn_prologue.argtypes = [lp] + [vp] * 8 + [fp, fp, vp]
         L.attn_fwd.argtypes = [lp, vp, vp, vp, vp, fp, vp]
+        ll, ci = ctypes.c_longlong, ctypes.c_int
+        L.attn_prologue_gated.argtypes = [lp] + [vp] * 5 + [ll, ci, vp, vp, vp, vp, vp, fp, fp, vp]
+        L.attn_gate_bwd.argtypes = [lp, vp, ll, ci, vp, vp, vp, fp, vp]
+        cf = ctypes.c_float
+        L.cswattn_gemm_bf16.argtypes = [ci, ci, ci, ci, vp, ll, ci, vp, ll, cf, cf, vp, ll, vp, ll, vp]
+        L.cswattn_gemm_bf16.restype = ci
+        L.muon_ns_workspace_bytes.argtypes = [ci, ci]
+        L.muon_ns_workspace_bytes.restype = sz
+        L.muon_newton_schulz.argtypes = [ci, ci, ctypes.POINTER(cf), ci, vp, vp, vp, sz, vp]
+        L.muon_newton_schulz.restype = ci
         L.attn_bwd_workspace_bytes.argtypes = [lp]
         L.attn_bwd_workspace_bytes.restype = sz
         L.attn_bwd.argtypes = [lp] + [vp] * 7 + [fp, fp, vp, fp, vp] + [vp] * 6 + [sz, vp]
@@ -81,8 +93,8 @@ def lib():
         L.attn_decode_workspace_bytes.argtypes = [lp]
         L.attn_decode_workspace_bytes.restype = sz
         L.attn_decode.argtypes = [lp] + [vp] * 5 + [vp, vp, vp, vp, fp, vp, sz, vp]
-        for name in ("attn_prologue", "attn_fwd", "attn_bwd", "attn_bwd_noalloc",
-                     "cswattn_sync_status"):
+        for name in ("attn_prologue", "attn_prologue_gated", "attn_gate_bwd", "attn_fwd", "attn_bwd",
+                     "attn_bwd_noalloc", "cswattn_sync_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -139,6 +151,25 @@ def attn_prologue(spec: LayerSpec, q, k, v, ve, gate, q_out, k_out, v_out, rstd_
     _check(lib().attn_prologue(ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(v), _ptr(ve),
                                _ptr(gate), _ptr(q_out), _ptr(k_out), _ptr(v_out),
                                _ptr(rstd_q), _ptr(rstd_k), _stream(stream)))
+
+
+def attn_prologue_gated(spec: LayerSpec, q, k, v, ve, x, gate_channels, w_gate, gate_out, q_out,
+                        k_out, v_out, rstd_q, rstd_k, stream=None):
+    """attn_prologue with the gate logits computed from the block input:
+    gate_out = x[..., :gate_channels] @ w_gate.T (x (B, T, X) contiguous)."""
+    layer = spec.c()
+    _check(lib().attn_prologue_gated(ctypes.byref(layer), _ptr(q), _ptr(k), _ptr(v), _ptr(ve),
+                                     _ptr(x), int(x.shape[-1]), int(gate_channels), _ptr(w_gate),
+                                     _ptr(gate_out), _ptr(q_out), _ptr(k_out), _ptr(v_out),
+                                     _ptr(rstd_q), _ptr(rstd_k), _stream(stream)))
+
+
+def attn_gate_bwd(spec: LayerSpec, x, gate_channels, w_gate, dgate, dx, dw_gate, stream=None):
+    """dx (B, T, gate_channels) and float32 dw_gate (Hk, gate_channels) of the
+    gate projection, from dgate (the attention backward's dgate)."""
+    layer = spec.c()
+    _check(lib().attn_gate_bwd(ctypes.byref(layer), _ptr(x), int(x.shape[-1]), int(gate_channels),
+                               _ptr(w_gate), _ptr(dgate), _ptr(dx), _ptr(dw_gate), _stream(stream)))
 
 
 def attn_fwd(spec: LayerSpec, q_out, k_out, v_out, O, lse, stream=None):
@@ -268,3 +299,30 @@ def layer_backward(spec: LayerSpec, buf: LayerBuffers, q, k, ve, gate, dO, strea
     attn_bwd(spec, q, k, ve, gate, buf.q_out, buf.k_out, buf.v_out, buf.rstd_q, buf.rstd_k,
              buf.O, buf.lse, dO, buf.dQ, buf.dK, buf.dV, buf.dve, buf.dgate, buf.workspace,
              stream=stream)
+
+
+# ------------------------------------------------------------------ Muon
+
+def gemm_bf16(A, B, C, alpha=1.0, beta=0.0, D=None, a_mn=False, b_mn=True, stream=None):
+    """C = alpha Aop Bop^T + beta D on the tensor cores (see the C header for
+    Aop/Bop). Defaults: the plain product of row-major A (M x K), B (K x N)."""
+    M, N = C.shape
+    K = A.shape[0] if a_mn else A.shape[1]
+    _check(lib().cswattn_gemm_bf16(M, N, K, int(a_mn), _ptr(A), A.stride(0), int(b_mn), _ptr(B),
+                                   B.stride(0), float(alpha), float(beta), _ptr(D),
+                                   D.stride(0) if D is not None else N, _ptr(C), C.stride(0),
+                                   _stream(stream)))
+
+
+def muon_ns_workspace_bytes(m: int, n: int) -> int:
+    return int(lib().muon_ns_workspace_bytes(m, n))
+
+
+def muon_newton_schulz(X, Y, coeffs, workspace, stream=None):
+    """Muon's Newton-Schulz iteration, one step per (a, b, c) triple, from the
+    bf16 m x n matrix X into Y (see the C header)."""
+    m, n = X.shape
+    flat = [float(v) for t in coeffs for v in t]
+    arr = (ctypes.c_float * len(flat))(*flat)
+    _check(lib().muon_newton_schulz(m, n, arr, len(coeffs), _ptr(X), _ptr(Y), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))

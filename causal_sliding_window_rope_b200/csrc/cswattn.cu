@@ -20,6 +20,8 @@
 #include "fwd_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "decode.cuh"
+#include "gate.cuh"
+#include "gemm_sm100.cuh"
 
 using namespace cswattn;
 
@@ -159,6 +161,26 @@ cswattn_status make_map(CUtensorMap* map, const void* base, int outer, int T, in
   CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CSWATTN_OK;
+}
+
+// Tensor map of a row-major bf16 matrix of `rows` rows of `inner`
+// contiguous elements, `ld` elements apart, viewed as 2-D (inner, rows);
+// a box is box_inner x box_rows (128B swizzle, box_inner = 64), out-of-range
+// elements read as zero.
+cswattn_status make_map_2d(CUtensorMap* map, const void* base, long long inner, long long rows, long long ld,
+                           int box_inner, int box_rows) {
+  EncodeTiledFn enc;
+  cswattn_status s = get_encoder(&enc);
+  if (s != CSWATTN_OK) return s;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return CSWATTN_OK;
@@ -480,6 +502,105 @@ cswattn_status noalloc_scratch(void** out) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- matrix product
+
+struct GemmArgs {
+  int M, N, K;
+  bool a_mn, b_mn;
+  const void *A, *B, *D;
+  long long lda, ldb, ldd, ldc;
+  float alpha, beta;
+  void* C;
+};
+
+cswattn_status check_gemm(const GemmArgs& g) {
+  if (g.M < 1 || g.N < 1 || g.K < 1) return fail(CSWATTN_ERR_INVALID_ARG, "M, N, K must be >= 1");
+  if (g.M > (1 << 30) || g.N > (1 << 30) || g.K > (1 << 30)) return fail(CSWATTN_ERR_UNSUPPORTED, "matrix too large");
+  if (g.N % 8 != 0) return fail(CSWATTN_ERR_UNSUPPORTED, "N must be a multiple of 8 (got %d)", g.N);
+  const long long a_inner = g.a_mn ? g.M : g.K, b_inner = g.b_mn ? g.N : g.K;
+  if (g.lda < a_inner || g.ldb < b_inner || g.ldc < g.N || (g.beta != 0.f && g.ldd < g.N))
+    return fail(CSWATTN_ERR_INVALID_ARG, "a leading dimension is smaller than its row");
+  if (g.lda % 8 || g.ldb % 8 || g.ldc % 8 || (g.beta != 0.f && g.ldd % 8))
+    return fail(CSWATTN_ERR_INVALID_ARG, "leading dimensions must be multiples of 8 elements");
+  CHECK_PTR(g.A, 16);
+  CHECK_PTR(g.B, 16);
+  CHECK_PTR(g.C, 16);
+  if (g.beta != 0.f) CHECK_PTR(g.D, 16);
+  if (g.C == g.A || g.C == g.B) return fail(CSWATTN_ERR_INVALID_ARG, "C must not alias A or B");
+  if (!std::isfinite(g.alpha) || !std::isfinite(g.beta)) return fail(CSWATTN_ERR_INVALID_ARG, "alpha, beta must be finite");
+  return CSWATTN_OK;
+}
+
+template <bool AMN, bool BMN>
+void launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& gp, dim3 grid, cudaStream_t st) {
+  launch_pdl(gemm::gemm_kernel<AMN, BMN>, grid, dim3(gemm::kThreads), gemm::kSmemBytes, st, ma, mb, gp);
+}
+
+// Validated product, tensor maps built before the launch; nothing is
+// enqueued when a check fails.
+cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st) {
+  cswattn_status e = check_gemm(g);
+  if (e != CSWATTN_OK) return e;
+  CUtensorMap ma, mb;
+  // K-major operand: (K, rows) with 64 x 128 boxes; MN-major: (rows, K) with 64 x 64 boxes.
+  if ((e = g.a_mn ? make_map_2d(&ma, g.A, g.M, g.K, g.lda, 64, 64) : make_map_2d(&ma, g.A, g.K, g.M, g.lda, 64, 128)) !=
+      CSWATTN_OK)
+    return e;
+  if ((e = g.b_mn ? make_map_2d(&mb, g.B, g.N, g.K, g.ldb, 64, 64) : make_map_2d(&mb, g.B, g.K, g.N, g.ldb, 64, 128)) !=
+      CSWATTN_OK)
+    return e;
+  const int which = (g.a_mn ? 2 : 0) + (g.b_mn ? 1 : 0);
+  switch (which) {
+    case 0: e = set_smem(gemm::gemm_kernel<false, false>, gemm::kSmemBytes); break;
+    case 1: e = set_smem(gemm::gemm_kernel<false, true>, gemm::kSmemBytes); break;
+    case 2: e = set_smem(gemm::gemm_kernel<true, false>, gemm::kSmemBytes); break;
+    default: e = set_smem(gemm::gemm_kernel<true, true>, gemm::kSmemBytes); break;
+  }
+  if (e != CSWATTN_OK) return e;
+  gemm::Params gp;
+  gp.M = g.M;
+  gp.N = g.N;
+  gp.K = g.K;
+  gp.alpha = g.alpha;
+  gp.beta = g.beta;
+  gp.D = static_cast<const __nv_bfloat16*>(g.D);
+  gp.ldd = g.ldd;
+  gp.C = static_cast<__nv_bfloat16*>(g.C);
+  gp.ldc = g.ldc;
+  gp.wait_ns = g_wait_ns.load();
+  const dim3 grid((g.N + gemm::kBN - 1) / gemm::kBN, (g.M + gemm::kBM - 1) / gemm::kBM);
+  if (grid.y > 65535) return fail(CSWATTN_ERR_UNSUPPORTED, "M too large");
+  {
+    ScopedTiming tm(CSWATTN_K_GEMM, st);
+    switch (which) {
+      case 0: launch_gemm_t<false, false>(ma, mb, gp, grid, st); break;
+      case 1: launch_gemm_t<false, true>(ma, mb, gp, grid, st); break;
+      case 2: launch_gemm_t<true, false>(ma, mb, gp, grid, st); break;
+      default: launch_gemm_t<true, true>(ma, mb, gp, grid, st); break;
+    }
+  }
+  return launched("matrix product launch");
+}
+
+struct NsWorkspace {
+  void *A, *B, *X;
+  size_t bytes;
+};
+
+NsWorkspace carve_ns(int m, int n, void* base) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  NsWorkspace w;
+  size_t off = 0;
+  w.A = p + off;
+  off += pad256(static_cast<size_t>(n) * n * 2);
+  w.B = p + off;
+  off += pad256(static_cast<size_t>(n) * n * 2);
+  w.X = p + off;
+  off += pad256(static_cast<size_t>(m) * n * 2);
+  w.bytes = off;
+  return w;
+}
+
 // ---------------------------------------------------------------- decode
 
 struct DecodeWorkspace {
@@ -586,10 +707,22 @@ cswattn_status cswattn_sync_status(void* stream) {
   return CSWATTN_OK;
 }
 
-cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const void* k,
-                             const void* v, const void* ve, const void* gate, void* q_out,
-                             void* k_out, void* v_out, float* rstd_q, float* rstd_k,
-                             void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The gate's projection inputs of attn_prologue_gated (null for attn_prologue).
+struct GateIn {
+  const void* x;
+  long long x_stride;
+  int channels;
+  const void* w;
+  void* logits_out;
+};
+
+cswattn_status prologue_impl(const cswattn_layer* layer, const void* q, const void* k, const void* v,
+                             const void* ve, const void* gate, const GateIn* gi, void* q_out,
+                             void* k_out, void* v_out, float* rstd_q, float* rstd_k, void* stream) {
   Shape s;
   cswattn_status st = check_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
@@ -603,7 +736,17 @@ cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const vo
   CHECK_PTR(rstd_k, 4);
   if (layer->has_ve) {
     CHECK_PTR(ve, 16);
-    CHECK_PTR(gate, s.esize);
+    if (!gi) CHECK_PTR(gate, s.esize);
+  }
+  if (gi) {
+    if (!layer->has_ve)
+      return fail(CSWATTN_ERR_INVALID_ARG, "the gate projection needs a value embedding (has_ve = 1)");
+    if (gi->channels < 1 || gi->x_stride < gi->channels)
+      return fail(CSWATTN_ERR_INVALID_ARG, "gate_channels must be >= 1 and <= x_stride (got %d, %lld)",
+                  gi->channels, gi->x_stride);
+    CHECK_PTR(gi->x, s.esize);
+    CHECK_PTR(gi->w, s.esize);
+    CHECK_PTR(gi->logits_out, s.esize);
   }
   if (q_out == q || k_out == k || v_out == v || q_out == k_out || k_out == v_out || q_out == v_out)
     return fail(CSWATTN_ERR_INVALID_ARG, "prologue outputs must not alias its inputs or each other");
@@ -625,6 +768,11 @@ cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const vo
   pp.v_out = v_out;
   pp.rstd_q = rstd_q;
   pp.rstd_k = rstd_k;
+  pp.xg = gi ? gi->x : nullptr;
+  pp.x_stride = gi ? gi->x_stride : 0;
+  pp.gc = gi ? gi->channels : 0;
+  pp.w_gate = gi ? gi->w : nullptr;
+  pp.gate_out = gi ? gi->logits_out : nullptr;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   {
     ScopedTiming tm(CSWATTN_K_PROLOGUE, cs);
@@ -632,6 +780,67 @@ cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const vo
   }
   if (st != CSWATTN_OK) return st;
   return launched("prologue launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const void* k,
+                             const void* v, const void* ve, const void* gate, void* q_out,
+                             void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                             void* stream) {
+  return prologue_impl(layer, q, k, v, ve, gate, nullptr, q_out, k_out, v_out, rstd_q, rstd_k, stream);
+}
+
+cswattn_status attn_prologue_gated(const cswattn_layer* layer, const void* q, const void* k,
+                                   const void* v, const void* ve, const void* x, long long x_stride,
+                                   int gate_channels, const void* w_gate, void* gate_out, void* q_out,
+                                   void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                   void* stream) {
+  const GateIn gi{x, x_stride, gate_channels, w_gate, gate_out};
+  return prologue_impl(layer, q, k, v, ve, nullptr, &gi, q_out, k_out, v_out, rstd_q, rstd_k, stream);
+}
+
+cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long long x_stride,
+                             int gate_channels, const void* w_gate, const void* dgate, void* dx,
+                             float* dw_gate, void* stream) {
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  if (!layer->has_ve)
+    return fail(CSWATTN_ERR_INVALID_ARG, "the gate projection needs a value embedding (has_ve = 1)");
+  if (gate_channels < 1 || x_stride < gate_channels)
+    return fail(CSWATTN_ERR_INVALID_ARG, "gate_channels must be >= 1 and <= x_stride (got %d, %lld)",
+                gate_channels, x_stride);
+  CHECK_PTR(x, s.esize);
+  CHECK_PTR(w_gate, s.esize);
+  CHECK_PTR(dgate, s.esize);
+  CHECK_PTR(dx, s.esize);
+  CHECK_PTR(dw_gate, 4);
+  GateBwdParams gp;
+  gp.ntok = static_cast<long long>(s.B) * s.T;
+  gp.x_stride = x_stride;
+  gp.Hk = s.Hk;
+  gp.C = gate_channels;
+  gp.dw_blocks = s.Hk * ((gate_channels + 31) / 32);
+  gp.x = x;
+  gp.w = w_gate;
+  gp.dgate = dgate;
+  gp.dx = dx;
+  gp.dw = dw_gate;
+  const long long dx_blocks = (gp.ntok * gate_channels + kGateDwThreads - 1) / kGateDwThreads;
+  if (gp.dw_blocks + dx_blocks > 0x7fffffffll) return fail(CSWATTN_ERR_UNSUPPORTED, "gate backward too large");
+  const dim3 grid(static_cast<unsigned>(gp.dw_blocks + dx_blocks));
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  {
+    ScopedTiming tm(CSWATTN_K_GATE_BWD, cs);
+    if (s.bf16)
+      launch_pdl(gate_bwd_kernel<__nv_bfloat16>, grid, dim3(kGateDwThreads), 0, cs, gp);
+    else
+      launch_pdl(gate_bwd_kernel<float>, grid, dim3(kGateDwThreads), 0, cs, gp);
+  }
+  return launched("gate backward launch");
 }
 
 cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const void* k_out,
@@ -942,6 +1151,53 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   }
   if (st != CSWATTN_OK) return st;
   return launched("decode launch");
+}
+
+cswattn_status cswattn_gemm_bf16(int M, int N, int K, int a_mn, const void* A, long long lda, int b_mn,
+                                 const void* B, long long ldb, float alpha, float beta, const void* D,
+                                 long long ldd, void* C, long long ldc, void* stream) {
+  const GemmArgs g{M, N, K, a_mn != 0, b_mn != 0, A, B, D, lda, ldb, ldd, ldc, alpha, beta, C};
+  return run_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+size_t muon_ns_workspace_bytes(int m, int n) {
+  if (m < 1 || n < 1) return 0;
+  return carve_ns(m, n, nullptr).bytes;
+}
+
+cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, const void* X, void* Y,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (m < 1 || n < 1) return fail(CSWATTN_ERR_INVALID_ARG, "m, n must be >= 1");
+  if (n % 8 != 0) return fail(CSWATTN_ERR_UNSUPPORTED, "n must be a multiple of 8 (got %d)", n);
+  if (steps < 1 || steps > 64) return fail(CSWATTN_ERR_INVALID_ARG, "steps must be in [1, 64]");
+  if (!coeffs) return fail(CSWATTN_ERR_INVALID_ARG, "coeffs is NULL");
+  for (int i = 0; i < 3 * steps; ++i)
+    if (!std::isfinite(coeffs[i])) return fail(CSWATTN_ERR_INVALID_ARG, "coefficients must be finite");
+  CHECK_PTR(X, 16);
+  CHECK_PTR(Y, 16);
+  CHECK_PTR(workspace, 256);
+  if (X == Y) return fail(CSWATTN_ERR_INVALID_ARG, "X and Y must be different buffers");
+  const NsWorkspace w = carve_ns(m, n, workspace);
+  if (workspace_bytes < w.bytes)
+    return fail(CSWATTN_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes, w.bytes);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const void* cur = X;
+  for (int st_i = 0; st_i < steps; ++st_i) {
+    const float a = coeffs[3 * st_i], b = coeffs[3 * st_i + 1], c = coeffs[3 * st_i + 2];
+    void* out = ((steps - 1 - st_i) % 2 == 0) ? Y : w.X;  // the last step writes Y
+    // A = X^T X (n x n): both operands are X read MN-major, K = m.
+    GemmArgs g1{n, n, m, true, true, cur, cur, nullptr, n, n, 0, n, 1.f, 0.f, w.A};
+    // B = c A A + b A: A K-major, A again as the MN-major (K x N) operand.
+    GemmArgs g2{n, n, n, false, true, w.A, w.A, w.A, n, n, n, n, c, b, w.B};
+    // X' = X B + a X: X K-major (m x n), B MN-major.
+    GemmArgs g3{m, n, n, false, true, cur, w.B, cur, n, n, n, n, 1.f, a, out};
+    cswattn_status e;
+    if ((e = run_gemm(g1, cs)) != CSWATTN_OK) return e;
+    if ((e = run_gemm(g2, cs)) != CSWATTN_OK) return e;
+    if ((e = run_gemm(g3, cs)) != CSWATTN_OK) return e;
+    cur = out;
+  }
+  return CSWATTN_OK;
 }
 
 cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const void* k,

@@ -1,0 +1,202 @@
+// gemm_sm100.cuh -- bf16 matrix product on tcgen05 tensor cores, the step
+// Muon's orthogonalisation is made of (page "5만원으로 나만의 ChatGPT 훈련하는
+// 방법", section "2. Muon 옵티마이저 (nanochat/optim.py)": the quintic
+// Newton-Schulz iteration A = X^T X; B = b A + c A A; X = a X + X B).
+//
+//   C[m][n] = alpha * sum_k Aop[m][k] Bop[n][k] + beta * D[m][n]
+//
+// Aop[m][k] is A[m][k] of a row-major (M x K) A (K-major, A_MN = false) or
+// A[k][m] of a row-major (K x M) A (MN-major, A_MN = true); Bop[n][k] is
+// B[n][k] of a row-major (N x K) B or B[k][n] of a row-major (K x N) B. So
+// X^T X is A_MN = B_MN = true with A = B = X, and X B is A_MN = false,
+// B_MN = true. bf16 inputs and outputs (C, D), float32 accumulation.
+//
+// One CTA per 128 x 128 tile of C. Warp 0 (one thread) loads 64-wide K
+// chunks of both operands by TMA into a 6-stage ring (128B swizzle: a
+// K-major chunk is one panel of 128 rows x 64 K, an MN-major chunk two
+// panels of 64 K-rows x 64 elements); warp 1 owns the 128-column TMEM
+// accumulator and issues 4 MMAs (M = N = 128, K = 16) per chunk; warps 2-5
+// read the accumulator (thread = row of the tile), apply alpha and beta D
+// and store the row. Out-of-range rows, columns and K entries of a partial
+// tile read as zero and are not stored.
+#pragma once
+#include "common.cuh"
+
+namespace cswattn {
+namespace gemm {
+
+constexpr int kBM = 128, kBN = 128, kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kStages = 6;
+constexpr int kOpBytes = kBM * kBK * 2;   // 16 KB per operand per stage
+constexpr int kStageBytes = 2 * kOpBytes;
+constexpr int kOffBar = kStages * kStageBytes;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
+
+struct Params {
+  int M, N, K;
+  float alpha, beta;
+  const __nv_bfloat16* D;  // (M x N) row-major with ldd, or null when beta == 0
+  long long ldd;
+  __nv_bfloat16* C;        // (M x N) row-major with ldc
+  long long ldc;
+  unsigned long long wait_ns;
+};
+
+// TMA loads of one K chunk of an operand: rows r0.. of the tile, K from k0.
+// K-major: one 128-row x 64-K panel. MN-major: two 64-K-row panels of 64
+// M/N elements.
+template <bool MN>
+__device__ __forceinline__ void load_operand(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int r0,
+                                             int k0) {
+  if constexpr (MN) {
+    tma_load_2d(map, bar, dst, r0, k0);
+    tma_load_2d(map, bar, dst + kOpBytes / 2, r0 + 64, k0);
+  } else {
+    tma_load_2d(map, bar, dst, k0, r0);
+  }
+}
+
+// Shared-memory descriptor of an operand chunk and the offset (in 16-byte
+// units) of its K-step kk (16 K entries).
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
+  return MN ? sdesc_sw128(saddr, kOpBytes / 2, 1024)  // 64-element chunks 8 KB apart
+            : sdesc_sw128(saddr, 16, 1024);           // 128-byte rows, 8-row groups
+}
+template <bool MN>
+__device__ __forceinline__ uint64_t kstep_ofs(int kk) {
+  return static_cast<uint64_t>((MN ? kk * 16 * 128 : kk * 32) >> 4);
+}
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  pdl_launch_dependents();
+  uint8_t* smem = smem_align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = bars;                // [kStages]
+  uint64_t* empty = bars + kStages;     // [kStages]
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kStages + 2);
+  const int warp = warp_id(), lane = lane_id();
+  const int n0 = static_cast<int>(blockIdx.x) * kBN, m0 = static_cast<int>(blockIdx.y) * kBM;
+  const int nk = (p.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  const WaitCtx wc{abort_flag, p.wait_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      int issued[kStages] = {0, 0, 0, 0, 0, 0};
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % kStages, use = kc / kStages;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, wc)) break;
+        uint8_t* st = smem + s * kStageBytes;
+        mbar_expect_tx(&full[s], kStageBytes);
+        load_operand<A_MN>(&tmA, &full[s], st, m0, kc * kBK);
+        load_operand<B_MN>(&tmB, &full[s], st + kOpBytes, n0, kc * kBK);
+        ++issued[s];
+      }
+      for (int s = 0; s < kStages; ++s)
+        if (issued[s] > 0) drain_wait(&full[s], (issued[s] - 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t id = idesc_bf16(128, 128, A_MN ? 1 : 0, B_MN ? 1 : 0);
+      const uint32_t s0 = smem_u32(smem);
+      bool ok = true;
+      for (int kc = 0; ok && kc < nk; ++kc) {
+        const int s = kc % kStages, use = kc / kStages;
+        if (!mbar_wait(&full[s], use & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t da = operand_desc<A_MN>(s0 + s * kStageBytes);
+        const uint64_t db = operand_desc<B_MN>(s0 + s * kStageBytes + kOpBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          mma_ss(tmem, da + kstep_ofs<A_MN>(kk), db + kstep_ofs<B_MN>(kk), id, (kc > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(acc_full);  // also the drain: every issued product completes before it fires
+      drain_wait(acc_full, 0);
+    }
+  } else {
+    // -------------------------------------------------- epilogue (warps 2-5)
+    const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31
+    const int r = quad * 32 + lane;
+    const int m = m0 + r;
+    const bool got = mbar_wait(acc_full, 0, wc);
+    if (__all_sync(0xffffffffu, got)) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c * 32, a);
+        tmem_ld_wait();
+        if (m >= p.M) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int n = n0 + c * 32 + q * 8;  // 8 columns = 16 bytes
+          if (n >= p.N) break;
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = p.alpha * __uint_as_float(a[q * 8 + e]);
+          if (p.beta != 0.f) {
+            const uint4 u = *reinterpret_cast<const uint4*>(p.D + m * p.ldd + n);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h2[e]);
+              v[2 * e] = fmaf(p.beta, f.x, v[2 * e]);
+              v[2 * e + 1] = fmaf(p.beta, f.y, v[2 * e + 1]);
+            }
+          }
+          uint4 w;
+          w.x = pack_bf16x2(v[0], v[1]);
+          w.y = pack_bf16x2(v[2], v[3]);
+          w.z = pack_bf16x2(v[4], v[5]);
+          w.w = pack_bf16x2(v[6], v[7]);
+          *reinterpret_cast<uint4*>(p.C + m * p.ldc + n) = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace gemm
+}  // namespace cswattn

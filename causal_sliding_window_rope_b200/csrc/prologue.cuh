@@ -40,6 +40,14 @@ struct PrologueParams {
   const void *q, *k, *v, *ve, *gate;
   void *q_out, *k_out, *v_out;
   float *rstd_q, *rstd_k;
+  // Gate from the block input instead of given logits (xg non-null): the
+  // logits are x[b,t,:gc] . w_gate[h,:], rounded to the layer dtype and
+  // written to gate_out (B,T,Hk) for the backward.
+  const void* xg;        // (B,T,x_stride) block input, layer dtype
+  long long x_stride;    // elements between consecutive tokens of xg
+  int gc;                // gate channels C (the first C entries of a row)
+  const void* w_gate;    // (Hk, C), layer dtype
+  void* gate_out;        // (B,T,Hk), layer dtype
 };
 
 template <typename T>
@@ -319,10 +327,32 @@ __global__ void __launch_bounds__(kPrologueThreads)
     if (has_e) {
       HVec::load(eb + boff, el);
       HVec::load(eb + boff + HALF, eh);
-      gl = Vec16<T>::scalar(p.gate, row);
+      if (!p.xg) gl = Vec16<T>::scalar(p.gate, row);
     } else {
 #pragma unroll
       for (int i = 0; i < HV; ++i) el[i] = eh[i] = 0.f;
+    }
+    if (p.xg) {
+      // Gate logit of value rows: the row's LPR lanes split the C channels
+      // of x; the reduction runs on every lane (uniform shuffles).
+      float gp = 0.f;
+      if (has_e) {
+        const T* xr = static_cast<const T*>(p.xg) + (tok0 + tt) * p.x_stride;
+        const T* wr = static_cast<const T*>(p.w_gate) + static_cast<size_t>(head) * p.gc;
+        for (int c = sub; c < p.gc; c += LPR) gp = fmaf(Vec16<T>::scalar(xr, c), Vec16<T>::scalar(wr, c), gp);
+      }
+      gp = row_sum<LPR>(gp);
+      if (has_e) {
+        // Rounded to the layer dtype: the backward reads the stored logit.
+        if constexpr (sizeof(T) == 2) {
+          const __nv_bfloat16 g16 = __float2bfloat16_rn(gp);
+          gl = __bfloat162float(g16);
+          if (sub == 0) static_cast<__nv_bfloat16*>(p.gate_out)[row] = g16;
+        } else {
+          gl = gp;
+          if (sub == 0) static_cast<float*>(p.gate_out)[row] = gp;
+        }
+      }
     }
 
     // RMSNorm: mean of squares over the row (shuffle reduction over its lanes).

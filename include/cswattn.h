@@ -94,6 +94,37 @@ cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const vo
                              void* q_out, void* k_out, void* v_out, float* rstd_q,
                              float* rstd_k, void* stream);
 
+/* Prologue with the value-embedding gate computed from the block input
+ * instead of given as logits: page section "1. GPT 모델", value-embedding
+ * code, where the gate is 3*sigmoid(ve_gate(x[..., :C])) and ve_gate is a
+ * linear map from the first C channels of the block input x to one logit
+ * per KV head (no bias: the page shows none).
+ *   gate_out[b,t,h] = sum_{c<C} x[b,t,c] * w_gate[h,c], rounded to the layer
+ *   dtype; v_out = v + 3*sigmoid(gate_out)*ve; q_out, k_out, rstd_q, rstd_k
+ *   as for attn_prologue.
+ * x: (B, T, x_stride) in the layer dtype, only the first gate_channels
+ * entries of each token's row are read (1 <= gate_channels <= x_stride);
+ * w_gate: (n_kv_head, gate_channels); gate_out: (B, T, n_kv_head), the
+ * logits, to be passed as `gate` to attn_bwd. Requires has_ve = 1 (else
+ * CSWATTN_ERR_INVALID_ARG). Pointers aligned to the element size. */
+cswattn_status attn_prologue_gated(const cswattn_layer* layer, const void* q, const void* k,
+                                   const void* v, const void* ve, const void* x, long long x_stride,
+                                   int gate_channels, const void* w_gate, void* gate_out, void* q_out,
+                                   void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                   void* stream);
+
+/* Backward of the gate's projection (same page section), given dgate, the
+ * gradient of the loss with respect to the gate logits (attn_bwd's dgate):
+ *   dx[b,t,c]      = sum_h dgate[b,t,h] * w_gate[h,c]    (B, T, gate_channels)
+ *   dw_gate[h,c]   = sum_{b,t} dgate[b,t,h] * x[b,t,c]   (n_kv_head, gate_channels)
+ * dx is the contribution to the gradient of x[..., :gate_channels] (the
+ * caller adds it to its own); dx in the layer dtype, dw_gate float32 and
+ * deterministic (a fixed summation order). x, x_stride, gate_channels,
+ * w_gate as for attn_prologue_gated. Requires has_ve = 1. */
+cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long long x_stride,
+                             int gate_channels, const void* w_gate, const void* dgate, void* dx,
+                             float* dw_gate, void* stream);
+
 /* Forward: O_i = sum_j softmax_j(scale * q_out_i . k_out_j) v_out_j over the
  * causal window, and lse_i = log sum_j exp(scale * q_out_i . k_out_j).
  * Page section "5. 플래시 어텐션 통합" (causal call with window_size).
@@ -199,6 +230,42 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
                            void* k_cache, void* v_cache, void* O, float* lse, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* bf16 matrix product on the tensor cores, the step Muon's orthogonalisation
+ * is made of (page section "2. Muon 옵티마이저 (nanochat/optim.py)"):
+ *   C[m][n] = alpha * sum_k Aop[m][k] * Bop[n][k] + beta * D[m][n]
+ * Aop[m][k] = A[m*lda + k] (a_mn = 0: A is M x K, K contiguous) or
+ * A[k*lda + m] (a_mn = 1: A is K x M, M contiguous); Bop[n][k] = B[n*ldb + k]
+ * (b_mn = 0) or B[k*ldb + n] (b_mn = 1). So a_mn = 0, b_mn = 1 is the plain
+ * product of row-major A (M x K) and B (K x N). C and D: M x N, row-major
+ * with ldc, ldd (D read only when beta != 0; D may be C). bf16 A, B, C, D,
+ * float32 accumulation. N and every leading dimension a multiple of 8
+ * elements, pointers 16-byte aligned, C not aliasing A or B; other sizes
+ * are free (partial tiles read zeros past the edges). */
+cswattn_status cswattn_gemm_bf16(int M, int N, int K, int a_mn, const void* A, long long lda, int b_mn,
+                                 const void* B, long long ldb, float alpha, float beta, const void* D,
+                                 long long ldd, void* C, long long ldc, void* stream);
+
+/* Bytes of device scratch muon_newton_schulz needs for an m x n matrix:
+ * A and B (n x n) and one m x n iterate, bf16, each padded to 256 bytes.
+ * 0 for m or n < 1. */
+size_t muon_ns_workspace_bytes(int m, int n);
+
+/* Muon's orthogonalisation by the quintic Newton-Schulz ("Polar Express")
+ * iteration of page section "2. Muon 옵티마이저 (nanochat/optim.py)", in
+ * the page's order and notation, one step per coefficient triple:
+ *   A = X^T X;  B = b*A + c*(A A);  X = a*X + X B
+ * coeffs: host array of 3*steps floats (a, b, c per step; the page prints
+ * the first two triples, (8.156, -22.483, 15.879) and (4.043, -2.809, 0.5),
+ * and elides the rest). X (m x n, row-major, bf16) is the input iterate
+ * (the caller scales it as it wishes beforehand; the iteration is
+ * equivariant under transposition, so a wide matrix may be passed
+ * transposed to make A the smaller product); Y (m x n, bf16) receives the
+ * result and must not alias X. Every product is a cswattn_gemm_bf16 with
+ * bf16 intermediates. n a multiple of 8, 1 <= steps <= 64; workspace of at
+ * least muon_ns_workspace_bytes(m, n), 256-byte aligned. */
+cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, const void* X, void* Y,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the
  * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last check, CSWATTN_ERR_INVALID_ARG if a decode step met a cache
@@ -229,7 +296,9 @@ enum {
   CSWATTN_K_BWD = 3,      /* attention backward main kernel(s) */
   CSWATTN_K_BWD_EPI = 4,  /* backward epilogue: RoPE^-1, RMSNorm', dv/dve/dgate */
   CSWATTN_K_DECODE = 5,   /* decode step: new-token prologue, split-KV attention, combine */
-  CSWATTN_NUM_KERNELS = 6
+  CSWATTN_K_GATE_BWD = 6, /* backward of the value-embedding gate's projection */
+  CSWATTN_K_GEMM = 7,     /* bf16 matrix product (the Newton-Schulz steps) */
+  CSWATTN_NUM_KERNELS = 8
 };
 
 /* Per-kernel device timing for measurement tools. With enable != 0, every

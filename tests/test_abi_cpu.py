@@ -197,3 +197,18 @@ def test_build_tracks_every_kernel_source(tmp_path, monkeypatch):
         os.utime(d, (t_lib + 10, t_lib + 10))
         assert cs_build.stale(), d
         os.utime(d, (t_lib - 10, t_lib - 10))
+
+
+def test_gate_entry_point_validation(lib):
+    """The gate projection needs a value embedding and 1 <= C <= x_stride."""
+    ptrs = [256 * (i + 1) for i in range(12)]
+    no_ve = cs.LayerSpec(1, 16, 2, 1, 128, 16, has_ve=False)
+    st = lib.attn_prologue_gated(ctypes.byref(no_ve.c()), *ptrs[:5], 32, 32, *ptrs[5:12], None)
+    assert st == cs.ERR_INVALID_ARG and b"value embedding" in lib.cswattn_last_error()
+    spec = cs.LayerSpec(1, 16, 2, 1, 128, 16, has_ve=True)
+    st = lib.attn_prologue_gated(ctypes.byref(spec.c()), *ptrs[:5], 16, 32, *ptrs[5:12], None)
+    assert st == cs.ERR_INVALID_ARG and b"gate_channels" in lib.cswattn_last_error()
+    st = lib.attn_gate_bwd(ctypes.byref(spec.c()), ptrs[0], 64, 0, *ptrs[1:5], None)
+    assert st == cs.ERR_INVALID_ARG
+    st = lib.attn_gate_bwd(ctypes.byref(no_ve.c()), ptrs[0], 64, 32, *ptrs[1:5], None)
+    assert st == cs.ERR_INVALID_ARG
