@@ -212,3 +212,29 @@ def test_gate_entry_point_validation(lib):
     assert st == cs.ERR_INVALID_ARG
     st = lib.attn_gate_bwd(ctypes.byref(no_ve.c()), ptrs[0], 64, 32, *ptrs[1:5], None)
     assert st == cs.ERR_INVALID_ARG
+
+
+def test_gemm_and_newton_schulz_validation(lib):
+    g = lib.cswattn_gemm_bf16
+    ok_args = dict(M=128, N=128, K=64, a_mn=0, A=256, lda=64, b_mn=1, B=512, ldb=128,
+                   alpha=1.0, beta=0.0, D=None, ldd=128, C=768, ldc=128)
+
+    def call(**kw):
+        a = {**ok_args, **kw}
+        return g(a["M"], a["N"], a["K"], a["a_mn"], a["A"], a["lda"], a["b_mn"], a["B"], a["ldb"],
+                 a["alpha"], a["beta"], a["D"], a["ldd"], a["C"], a["ldc"], None)
+
+    assert call(N=12, ldb=16, ldc=16) == cs.ERR_UNSUPPORTED          # N not a multiple of 8
+    assert call(lda=32) == cs.ERR_INVALID_ARG                        # row shorter than K
+    assert call(lda=68) == cs.ERR_INVALID_ARG                        # not a multiple of 8
+    assert call(C=256) == cs.ERR_INVALID_ARG                         # C aliases A
+    assert call(beta=1.0, D=None) == cs.ERR_INVALID_ARG              # beta needs D
+    assert call(M=0) == cs.ERR_INVALID_ARG
+    coeffs = (ctypes.c_float * 6)(8.156, -22.483, 15.879, 4.043, -2.809, 0.5)
+    n = lib.muon_ns_workspace_bytes(256, 128)
+    assert n == 2 * 128 * 128 * 2 + 256 * 128 * 2
+    ns = lib.muon_newton_schulz
+    assert ns(256, 128, coeffs, 2, 256, 256, 1024, n, None) == cs.ERR_INVALID_ARG      # X == Y
+    assert ns(256, 128, coeffs, 2, 256, 512, 1024, n - 1, None) == cs.ERR_INVALID_ARG  # workspace
+    assert ns(256, 128, coeffs, 0, 256, 512, 1024, n, None) == cs.ERR_INVALID_ARG      # steps
+    assert ns(256, 12, coeffs, 2, 256, 512, 1024, n, None) == cs.ERR_UNSUPPORTED       # n % 8
