@@ -358,6 +358,17 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
+    if args.muon_only:
+        # Profiling case: only the Newton-Schulz measurement.
+        if rank == 0:
+            peaks, peak_src = load_peaks()
+            print(json.dumps({"muon_ns": muon_bench(dev, peaks, peak_src, steps=args.steps,
+                                                    warmup=args.warmup)}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
     w = cs.WORKLOADS[args.config]
     if args.single_layer is not None:
         # Profiling case: one layer of the workload, same shapes and launches.
@@ -431,6 +442,8 @@ def run_ours(args):
         if solo and not args.no_decode:
             line["decode"] = decode_bench(w, dev, peaks, steps=args.steps, warmup=args.warmup,
                                           peak_src=peak_src)
+        if solo and not args.no_muon:
+            line["muon_ns"] = muon_bench(dev, peaks, peak_src, steps=args.steps, warmup=args.warmup)
         if solo and not args.no_other_configs:
             del st
             torch.cuda.empty_cache()
@@ -509,6 +522,61 @@ def decode_bench(w, dev, peaks, steps=20, warmup=5, peak_src="measured"):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": nbytes,
                          "peak_source": f"{peak_src} hbm_gbs"}}
+
+
+# Muon's orthogonalisation on the d24 model's MLP weight shapes (4 x 1536 by
+# 1536, and its transpose): the page prints two coefficient triples of the
+# Polar-Express iteration, so a step here is those two iteration steps.
+MUON_SHAPES = ((6144, 1536), (1536, 6144))
+
+
+def muon_bench(dev, peaks, peak_src, steps=20, warmup=5):
+    """Device time of muon_newton_schulz (three tensor-core products per
+    iteration step: X^T X, b A + c A A, a X + X B) on MUON_SHAPES. FLOPs per
+    iteration step: 2 m n^2 + 2 n^3 + 2 m n^2; the roofline divides them by
+    the matrix-product kernel's own event time."""
+    import torch
+
+    import causal_sliding_window_rope_b200 as cs
+    import oracle
+    coeffs = oracle.POLAR_EXPRESS_PRINTED
+    g = torch.Generator().manual_seed(4322)
+    out = {}
+    for m, n in MUON_SHAPES:
+        X = torch.randn(m, n, generator=g, dtype=torch.float64)
+        X = (X / X.norm()).to(torch.bfloat16).to(dev)
+        Y = torch.empty_like(X)
+        ws = torch.empty(cs.muon_ns_workspace_bytes(m, n), dtype=torch.uint8, device=dev)
+        for _ in range(max(warmup, 3)):
+            cs.muon_newton_schulz(X, Y, coeffs, ws)
+        torch.cuda.synchronize(dev)
+        stream = torch.cuda.current_stream(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        cs.cswattn_set_timing(True)
+        cs.cswattn_kernel_times()
+        for a, b in evs:
+            a.record(stream)
+            cs.muon_newton_schulz(X, Y, coeffs, ws)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        kt = cs.cswattn_kernel_times()
+        cs.cswattn_set_timing(False)
+        cs.cswattn_sync_status()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        # per iteration step: X^T X (2 m n^2), A A (2 n^3), X B (2 m n^2)
+        flops = len(coeffs) * (2 * m * n * n + 2 * n ** 3 + 2 * m * n * n)
+        tf = flops / (ms * 1e-3) / 1e12
+        ktf = flops * steps / (kt["gemm"][0] * 1e-3) / 1e12 if kt["gemm"][1] else None
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        out[f"{m}x{n}"] = {
+            "workload": f"Newton-Schulz of a {m} x {n} bf16 matrix, {len(coeffs)} iteration steps "
+                        f"(the printed Polar-Express coefficients)",
+            "ms_per_call": round(ms, 4), "tflops": round(tf, 1),
+            "gemm_launches_per_call": kt["gemm"][1] // steps,
+            "roofline": {"kernel": "gemm", "bound": "tensor", "achieved": round(ktf, 1) if ktf else None,
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(ktf / peak, 4) if ktf else None,
+                         "peak_source": f"{peak_src} bf16_tflops"}}
+    return out
 
 
 def traffic_for(kind):
@@ -637,6 +705,9 @@ def main():
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the device-timed summary of the other bf16 workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-muon", action="store_true", help="skip the Newton-Schulz measurement")
+    ap.add_argument("--muon-only", action="store_true",
+                    help="profiling case: only the Newton-Schulz measurement")
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--single-layer", type=int, default=None,

@@ -12,6 +12,8 @@
 #include <utility>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/cswattn.h"
 #include "common.cuh"
 #include "prologue.cuh"
@@ -28,6 +30,14 @@ using namespace cswattn;
 namespace {
 
 thread_local std::string t_err;
+
+// NVTX range around each entry point, so a profiler's timeline shows which
+// call enqueued which kernels (header-only NVTX: a few instructions when no
+// tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 std::atomic<unsigned long long> g_wait_ns{2000000000ull};
 // Floor of the caller's wait limit: far above the latency of any copy, matrix
 // product or hand-off between a kernel's roles, so that a short limit only
@@ -790,6 +800,7 @@ cswattn_status attn_prologue(const cswattn_layer* layer, const void* q, const vo
                              const void* v, const void* ve, const void* gate, void* q_out,
                              void* k_out, void* v_out, float* rstd_q, float* rstd_k,
                              void* stream) {
+  const NvtxRange nvtx_range("attn_prologue");
   return prologue_impl(layer, q, k, v, ve, gate, nullptr, q_out, k_out, v_out, rstd_q, rstd_k, stream);
 }
 
@@ -798,6 +809,7 @@ cswattn_status attn_prologue_gated(const cswattn_layer* layer, const void* q, co
                                    int gate_channels, const void* w_gate, void* gate_out, void* q_out,
                                    void* k_out, void* v_out, float* rstd_q, float* rstd_k,
                                    void* stream) {
+  const NvtxRange nvtx_range("attn_prologue_gated");
   const GateIn gi{x, x_stride, gate_channels, w_gate, gate_out};
   return prologue_impl(layer, q, k, v, ve, nullptr, &gi, q_out, k_out, v_out, rstd_q, rstd_k, stream);
 }
@@ -805,6 +817,7 @@ cswattn_status attn_prologue_gated(const cswattn_layer* layer, const void* q, co
 cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long long x_stride,
                              int gate_channels, const void* w_gate, const void* dgate, void* dx,
                              float* dw_gate, void* stream) {
+  const NvtxRange nvtx_range("attn_gate_bwd");
   Shape s;
   cswattn_status st = check_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
@@ -845,6 +858,7 @@ cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long lon
 
 cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const void* k_out,
                         const void* v_out, void* O, float* lse, void* stream) {
+  const NvtxRange nvtx_range("attn_fwd");
   Shape s;
   cswattn_status st = check_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
@@ -918,6 +932,7 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
                         const float* rstd_k, const void* O, const float* lse, const void* dO,
                         void* dQ, void* dK, void* dV, void* dve, void* dgate, void* workspace,
                         size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("attn_bwd");
   Shape s;
   cswattn_status st = check_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
@@ -1088,6 +1103,7 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
                            const void* ve, const void* gate, const int* cache_len, void* k_cache,
                            void* v_cache, void* O, float* lse, void* workspace, size_t workspace_bytes,
                            void* stream) {
+  const NvtxRange nvtx_range("attn_decode");
   Shape s;
   cswattn_status st = check_decode_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
@@ -1156,6 +1172,7 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
 cswattn_status cswattn_gemm_bf16(int M, int N, int K, int a_mn, const void* A, long long lda, int b_mn,
                                  const void* B, long long ldb, float alpha, float beta, const void* D,
                                  long long ldd, void* C, long long ldc, void* stream) {
+  const NvtxRange nvtx_range("cswattn_gemm_bf16");
   const GemmArgs g{M, N, K, a_mn != 0, b_mn != 0, A, B, D, lda, ldb, ldd, ldc, alpha, beta, C};
   return run_gemm(g, static_cast<cudaStream_t>(stream));
 }
@@ -1167,6 +1184,7 @@ size_t muon_ns_workspace_bytes(int m, int n) {
 
 cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, const void* X, void* Y,
                                   void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("muon_newton_schulz");
   if (m < 1 || n < 1) return fail(CSWATTN_ERR_INVALID_ARG, "m, n must be >= 1");
   if (n % 8 != 0) return fail(CSWATTN_ERR_UNSUPPORTED, "n must be a multiple of 8 (got %d)", n);
   if (steps < 1 || steps > 64) return fail(CSWATTN_ERR_INVALID_ARG, "steps must be in [1, 64]");
@@ -1206,6 +1224,7 @@ cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const
                                 const float* rstd_k, const void* O, const float* lse,
                                 const void* dO, void* dQ, void* dK, void* dV, void* dve,
                                 void* dgate, void* stream) {
+  const NvtxRange nvtx_range("attn_bwd_noalloc");
   Shape s;
   cswattn_status st = check_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
