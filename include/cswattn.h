@@ -132,7 +132,8 @@ cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long lon
 cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const void* k_out,
                         const void* v_out, void* O, float* lse, void* stream);
 
-/* Bytes of device scratch attn_bwd needs for this layer: float32
+/* Bytes of device scratch attn_bwd needs for this layer (the backward of
+ * the page section "5. 플래시 어텐션 통합" call, see attn_bwd): float32
  * accumulators of dq_out (B, T, n_head, head_dim), P partial sums each of
  * dk_out and dv_out (B, T, n_kv_head, head_dim) (P = 1..8, the number of
  * CTAs the bf16 backward splits a key tile's work into; 1 for f32), and two
@@ -141,7 +142,15 @@ cswattn_status attn_fwd(const cswattn_layer* layer, const void* q_out, const voi
  * every part padded to 256 bytes. Returns 0 for an invalid layer. */
 size_t attn_bwd_workspace_bytes(const cswattn_layer* layer);
 
-/* Backward of prologue + forward for the loss L with dL/dO = dO:
+/* Backward of prologue + forward for the loss L with dL/dO = dO: the
+ * gradient of the causal windowed attention call of page section
+ * "5. 플래시 어텐션 통합 (nanochat/flash_attention.py)" and of the
+ * steps before it in section "1. GPT 모델" (RoPE and QK normalisation of
+ * the architecture list, the value-embedding code), written out:
+ *   p = softmax(scale q_out k_out^T) over the window, dp = dO v_out^T,
+ *   ds = p (dp - rowsum(dO * O)), dq_out = scale ds k_out,
+ *   dk_out = scale ds^T q_out and dv_out = p^T dO summed over each KV
+ *   head's group of query heads, then back through RoPE and RMSNorm:
  * dQ, dK (through RoPE^-1 and RMSNorm), dV = dL/dv_out, and when has_ve
  * dve = 3*sigmoid(gate)*dV and dgate = 3*sigmoid(gate)*(1-sigmoid(gate)) *
  * sum_d dV*ve. q, k, ve, gate are the prologue's inputs; q_out, k_out, v_out,
@@ -266,7 +275,9 @@ size_t muon_ns_workspace_bytes(int m, int n);
 cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, const void* X, void* Y,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
-/* Waits for `stream`, then returns and clears the device status word of the
+/* Error reporting of the device side (no counterpart on the pages, which
+ * describe no error handling): waits for `stream`, then returns and clears
+ * the device status word of the
  * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last check, CSWATTN_ERR_INVALID_ARG if a decode step met a cache
  * length outside [0, T), CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
