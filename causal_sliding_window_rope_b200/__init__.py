@@ -19,9 +19,13 @@ from dataclasses import dataclass
 from .configs import WORKLOADS, Workload, alternating_ve, window_pattern  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcswattn.so")
+# CSWATTN_CHECK=1 in the environment selects the checked build (device-side
+# bounds checks that report CSWATTN_ERR_BOUNDS instead of faulting); build it
+# with `python -m causal_sliding_window_rope_b200.build --check`.
+CHECKED = os.environ.get("CSWATTN_CHECK", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libcswattn_check.so" if CHECKED else "libcswattn.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, 1, 2, 3, 4, 5
 F32, BF16 = 0, 1
 
 # Every symbol the header declares; the CPU tests check the library exports them.

@@ -17,6 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcswattn.so")
+LIB_CHECK = os.path.join(PKG, "libcswattn_check.so")  # CSWATTN_CHECK=1: device-side bounds checks
 SOURCES = ["cswattn.cu"]
 HEADER = os.path.join(ROOT, "include", "cswattn.h")
 
@@ -43,26 +44,30 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str | None = None) -> bool:
+    lib = lib or LIB
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(d) > t for d in deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, verbose: bool = False, check: bool = False) -> str:
+    """Compile libcswattn.so (or, with check, libcswattn_check.so: the same
+    library with CSWATTN_CHECK=1 device-side bounds checks)."""
+    lib = LIB_CHECK if check else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
+           *(["-DCSWATTN_CHECK=1"] if check else []),
            *(os.path.join(CSRC, s) for s in SOURCES), "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose="-v" in sys.argv, check="--check" in sys.argv))

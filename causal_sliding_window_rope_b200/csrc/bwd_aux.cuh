@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
       for (int i = 0; i < HV; ++i) acc = fmaf(o0[i], g0[i], fmaf(o1[i], g1[i], acc));
     }
     acc = row_sum<LPR>(acc);
-    if (valid && sub == 0) {
+    if (valid && sub == 0 && check_bounds(s_b[tt] < p.rows / p.H / p.T && s_t[tt] < p.T && h < p.H)) {
       const long long b = s_b[tt], t = s_t[tt];
       const long long o = (b * p.H + h) * p.Tpad;
       p.delta[o + t] = acc;
@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
     // Row within the block (sources) and within the tensor (destinations).
     const size_t brow = static_cast<size_t>(tt) * nheads + head;
     const size_t row = static_cast<size_t>(tok0 + tt) * nheads + head;  // (b,t,head)
+    if (valid && !check_bounds(row < static_cast<size_t>(n_tok) * nheads && tt < ntt)) continue;
     const size_t off_lo = row * D + static_cast<size_t>(sub) * HV;
     const size_t off_hi = off_lo + HALF;
     const size_t boff = brow * D + static_cast<size_t>(sub) * HV;

@@ -146,6 +146,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_all = p.g * nsph;
   const int n_begin = static_cast<int>(static_cast<long long>(part) * n_all / p.parts);
   const int N = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.parts) - n_begin;
+  // Checked build: the work unit lies inside the tensors and the row-term
+  // copies of its last step stay inside the padded (B, H, Tpad) arrays.
+  if (!check_bounds(b < p.B && hk < p.Hk && j < p.nkv && part < p.parts && qs_lo <= qs_hi &&
+                    (qs_hi + 1) * kBQ <= p.Tpad && n_begin + N <= n_all))
+    return;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);

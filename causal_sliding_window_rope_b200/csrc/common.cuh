@@ -18,6 +18,22 @@ namespace cswattn {
 __device__ unsigned int g_status;
 
 constexpr unsigned int kStatusTimeout = 4u;
+constexpr unsigned int kStatusBounds = 16u;
+
+// Bounds checks of the CSWATTN_CHECK=1 build: a failed check records
+// kStatusBounds in the status word (reported by cswattn_sync_status) and
+// evaluates to false so the caller skips the access; no trap. In the
+// release build the checks compile away.
+#ifndef CSWATTN_CHECK
+#define CSWATTN_CHECK 0
+#endif
+__device__ __forceinline__ bool check_bounds(bool ok) {
+  if (CSWATTN_CHECK && !ok) {
+    atomicOr(&g_status, kStatusBounds);
+    return false;
+  }
+  return true;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -710,6 +710,8 @@ cswattn_status cswattn_sync_status(void* stream) {
   if (v != 0) {
     e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    if (v & kStatusBounds)
+      return fail(CSWATTN_ERR_BOUNDS, "a device-side bounds check failed; the access was skipped (status 0x%x)", v);
     if (v & kStatusTimeout) return fail(CSWATTN_ERR_TIMEOUT, "a device-side wait ran out (status 0x%x)", v);
     if (v & kStatusRange)
       return fail(CSWATTN_ERR_INVALID_ARG, "a decode step met a cache length outside [0, T) (status 0x%x)", v);

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
   const bool work = in_range && c0 <= pos;
   const bool owns_new = work && pos < c0 + kChunk;  // this chunk holds the new token's row
   auto part = [&](int h) { return (static_cast<size_t>(b) * p.H + h) * p.nsplit + split; };
+  if (!check_bounds(b < p.B && hk < p.Hk && split < p.nsplit && (hk + 1) * g <= p.H)) return;
   if (!work) {
     // Empty chunk: a partial that the combine step ignores.
     for (int i = tid; i < g * D; i += blockDim.x) p.part_o[part(hk * g + i / D) * D + i % D] = 0.f;

@@ -108,6 +108,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int lo = valid[1] ? min(lo_t[0], lo_t[1]) : lo_t[0];
   const int hi = valid[1] ? max(hi_t[0], hi_t[1]) : hi_t[0];
+  // Checked build: the unit lies inside the tensors (uniform over the CTA,
+  // before any barrier or TMEM is set up).
+  if (!check_bounds(pr >= 0 && b < p.B && hk < p.Hk && lo >= 0 && hi < p.nq && head[0] < p.H &&
+                    head[1] < p.H && qblk[1] < p.nq))
+    return;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);

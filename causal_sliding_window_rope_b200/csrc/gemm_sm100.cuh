@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   const int n0 = static_cast<int>(blockIdx.x) * kBN, m0 = static_cast<int>(blockIdx.y) * kBM;
   const int nk = (p.K + kBK - 1) / kBK;
+  if (!check_bounds(m0 < p.M && n0 < p.N && nk >= 1)) return;  // checked build
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {

@@ -314,6 +314,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
     const size_t off_hi = off_lo + HALF;
     const size_t boff = brow * D + static_cast<size_t>(sub) * HV;
     const T* src = kind == 0 ? qb : (kind == 1 ? kb : vb);
+    if (valid && !check_bounds(row < static_cast<size_t>(n_tok) * nheads && tt < ntt && head < nheads))
+      continue;  // checked build: a row outside the tensor is skipped
     float xl[HV], xh[HV], el[HV], eh[HV];
     float gl = 0.f;
     if (valid) {

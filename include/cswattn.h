@@ -63,7 +63,8 @@ typedef enum {
   CSWATTN_ERR_INVALID_ARG = 1,
   CSWATTN_ERR_UNSUPPORTED = 2,
   CSWATTN_ERR_CUDA = 3,
-  CSWATTN_ERR_TIMEOUT = 4
+  CSWATTN_ERR_TIMEOUT = 4,
+  CSWATTN_ERR_BOUNDS = 5 /* a device-side bounds check failed (CSWATTN_CHECK=1 build only) */
 } cswattn_status;
 
 typedef enum { CSWATTN_F32 = 0, CSWATTN_BF16 = 1 } cswattn_dtype;
@@ -280,7 +281,10 @@ cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, 
  * the device status word of the
  * current device: CSWATTN_ERR_TIMEOUT if a kernel's bounded wait ran out
  * since the last check, CSWATTN_ERR_INVALID_ARG if a decode step met a cache
- * length outside [0, T), CSWATTN_ERR_CUDA on a CUDA error, else CSWATTN_OK. */
+ * length outside [0, T), CSWATTN_ERR_BOUNDS if a bounds check of the
+ * checked build (libcswattn_check.so, compiled with CSWATTN_CHECK=1) failed
+ * (the access was skipped), CSWATTN_ERR_CUDA on a CUDA error, else
+ * CSWATTN_OK. */
 cswattn_status cswattn_sync_status(void* stream);
 
 /* Self-test of the bounded-wait path: launches one small kernel whose thread

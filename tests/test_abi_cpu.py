@@ -238,3 +238,13 @@ def test_gemm_and_newton_schulz_validation(lib):
     assert ns(256, 128, coeffs, 2, 256, 512, 1024, n - 1, None) == cs.ERR_INVALID_ARG  # workspace
     assert ns(256, 128, coeffs, 0, 256, 512, 1024, n, None) == cs.ERR_INVALID_ARG      # steps
     assert ns(256, 12, coeffs, 2, 256, 512, 1024, n, None) == cs.ERR_UNSUPPORTED       # n % 8
+
+
+def test_checked_build_compiles_and_exports_the_same_symbols():
+    """The CSWATTN_CHECK=1 build (device-side bounds checks that report
+    CSWATTN_ERR_BOUNDS) compiles and exports what the header declares."""
+    path = cs_build.build(check=True)
+    assert path.endswith("libcswattn_check.so")
+    checked = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(checked, n), n
