@@ -302,3 +302,32 @@ def gemm(A, B, alpha=1.0, D=None, beta=0.0):
     if D is not None and beta != 0.0:
         C = C + beta * np.asarray(D, np.float64)
     return C
+
+
+# ---------------------------------------------------------------- QKV projection
+
+def qkv_projection(x, w_qkv, H, Hk, D):
+    """q, k, v of the layer from the block input x (B, T, C) and the stacked
+    bias-free projection weight w_qkv ((H + 2 Hk) D, C) (rows: the H query
+    heads, then the Hk key heads, then the Hk value heads), float64:
+    q = x w_q^T viewed (B, T, H, D), likewise k and v with Hk heads."""
+    x = _f64(x)
+    w = _f64(w_qkv)
+    B, T, C = x.shape
+    if w.shape != ((H + 2 * Hk) * D, C):
+        raise ValueError("w_qkv must be ((H + 2 Hk) D, C)")
+    y = x.reshape(B * T, C) @ w.T
+    q = y[:, :H * D].reshape(B, T, H, D)
+    k = y[:, H * D:(H + Hk) * D].reshape(B, T, Hk, D)
+    v = y[:, (H + Hk) * D:].reshape(B, T, Hk, D)
+    return q, k, v
+
+
+def qkv_projection_bwd(x, w_qkv, dq, dk, dv):
+    """dx (B, T, C) and dw_qkv of the projection given the gradients of q, k, v."""
+    x = _f64(x)
+    w = _f64(w_qkv)
+    B, T, C = x.shape
+    dy = np.concatenate([_f64(dq).reshape(B * T, -1), _f64(dk).reshape(B * T, -1),
+                         _f64(dv).reshape(B * T, -1)], axis=1)
+    return (dy @ w).reshape(B, T, C), dy.T @ x.reshape(B * T, C)

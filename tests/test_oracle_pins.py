@@ -478,3 +478,59 @@ def test_gemm_matches_explicit_sums():
         for j in range(2):
             s = sum(A[i, k] * B[k, j] for k in range(4))
             assert abs(C[i, j] - (0.5 * s - 2.0 * D[i, j])) < 1e-13
+
+
+# ---------------------------------------------------------------- QKV projection
+
+def test_qkv_projection_matches_torch_linear_and_autograd():
+    B, T, C, H, Hk, D = 2, 5, 12, 4, 2, 6
+    x = rnd((B, T, C), 100)
+    w = rnd(((H + 2 * Hk) * D, C), 101)
+    xt = torch.tensor(x, requires_grad=True)
+    wt = torch.tensor(w, requires_grad=True)
+    y = F.linear(xt, wt)
+    q, k, v = oracle.qkv_projection(x, w, H, Hk, D)
+    np.testing.assert_allclose(q, y[..., :H * D].detach().numpy().reshape(B, T, H, D), atol=1e-13)
+    np.testing.assert_allclose(k, y[..., H * D:(H + Hk) * D].detach().numpy().reshape(B, T, Hk, D), atol=1e-13)
+    np.testing.assert_allclose(v, y[..., (H + Hk) * D:].detach().numpy().reshape(B, T, Hk, D), atol=1e-13)
+    gq, gk, gv = rnd(q.shape, 102), rnd(k.shape, 103), rnd(v.shape, 104)
+    y.backward(torch.cat([torch.tensor(gq).reshape(B, T, -1), torch.tensor(gk).reshape(B, T, -1),
+                          torch.tensor(gv).reshape(B, T, -1)], dim=-1))
+    dx, dw = oracle.qkv_projection_bwd(x, w, gq, gk, gv)
+    np.testing.assert_allclose(dx, xt.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(dw, wt.grad.numpy(), atol=1e-12)
+
+
+def test_qkv_projection_gradients_match_central_differences():
+    """dL/dx and dL/dW of the whole layer fed by the projection, from the
+    layer's dq, dk, dv through the projection's backward, against central
+    differences of L = sum(O * dO)."""
+    L = oracle.Layer(1, 10, 4, 2, 4, 4, has_ve=True)
+    C = 6
+    x = rnd((1, L.T, C), 105)
+    w = rnd(((L.H + 2 * L.Hk) * L.D, C), 106) / 2
+    _, _, _, ve, gate, dO = inputs(L, 107)
+
+    def loss(x_, w_):
+        q, k, v = oracle.qkv_projection(x_, w_, L.H, L.Hk, L.D)
+        return _loss(L, q, k, v, ve, gate, dO)
+
+    q, k, v = oracle.qkv_projection(x, w, L.H, L.Hk, L.D)
+    r = oracle.layer(L, q, k, v, ve, gate, dO)
+    dx, dw = oracle.qkv_projection_bwd(x, w, r["dq"], r["dk"], r["dv"])
+    h = 1e-6
+    rng = np.random.default_rng(9)
+    for _ in range(8):
+        t, c = int(rng.integers(0, L.T)), int(rng.integers(0, C))
+        xp, xm = x.copy(), x.copy()
+        xp[0, t, c] += h
+        xm[0, t, c] -= h
+        fd = (loss(xp, w) - loss(xm, w)) / (2 * h)
+        assert abs(fd - dx[0, t, c]) <= 1e-6 * max(1.0, abs(dx[0, t, c])), ("x", t, c)
+    for _ in range(12):
+        o, c = int(rng.integers(0, w.shape[0])), int(rng.integers(0, C))
+        wp, wm = w.copy(), w.copy()
+        wp[o, c] += h
+        wm[o, c] -= h
+        fd = (loss(x, wp) - loss(x, wm)) / (2 * h)
+        assert abs(fd - dw[o, c]) <= 1e-6 * max(1.0, abs(dw[o, c])), ("w", o, c)
