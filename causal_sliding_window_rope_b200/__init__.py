@@ -29,7 +29,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, 1, 
 F32, BF16 = 0, 1
 
 # Every symbol the header declares; the CPU tests check the library exports them.
-EXPORTS = ("attn_prologue", "attn_prologue_gated", "attn_gate_bwd", "attn_fwd",
+EXPORTS = ("attn_prologue", "attn_prologue_gated", "attn_gate_bwd", "attn_qkv_prologue",
+           "attn_qkv_bwd", "attn_fwd",
            "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
            "attn_decode_workspace_bytes", "attn_decode", "cswattn_gemm_bf16",
            "muon_ns_workspace_bytes", "muon_newton_schulz",
@@ -72,6 +73,10 @@ def lib():
         ll, ci = ctypes.c_longlong, ctypes.c_int
         L.attn_prologue_gated.argtypes = [lp] + [vp] * 5 + [ll, ci, vp, vp, vp, vp, vp, fp, fp, vp]
         L.attn_gate_bwd.argtypes = [lp, vp, ll, ci, vp, vp, vp, fp, vp]
+        L.attn_qkv_prologue.argtypes = [lp, vp, ll, ci] + [vp] * 8 + [fp, fp, vp]
+        L.attn_qkv_prologue.restype = ci
+        L.attn_qkv_bwd.argtypes = [lp, vp, ll, ci] + [vp] * 5 + [fp, vp]
+        L.attn_qkv_bwd.restype = ci
         cf = ctypes.c_float
         L.cswattn_gemm_bf16.argtypes = [ci, ci, ci, ci, vp, ll, ci, vp, ll, cf, cf, vp, ll, vp, ll, vp]
         L.cswattn_gemm_bf16.restype = ci
@@ -174,6 +179,23 @@ def attn_gate_bwd(spec: LayerSpec, x, gate_channels, w_gate, dgate, dx, dw_gate,
     layer = spec.c()
     _check(lib().attn_gate_bwd(ctypes.byref(layer), _ptr(x), int(x.shape[-1]), int(gate_channels),
                                _ptr(w_gate), _ptr(dgate), _ptr(dx), _ptr(dw_gate), _stream(stream)))
+
+
+def attn_qkv_prologue(spec: LayerSpec, x, C, w_qkv, ve, gate, q, k, q_out, k_out, v_out, rstd_q,
+                      rstd_k, stream=None):
+    """The QKV projection of x[..., :C] by the stacked weight w_qkv, fused with
+    the prologue (see the C header); q and k receive the raw projections."""
+    layer = spec.c()
+    _check(lib().attn_qkv_prologue(ctypes.byref(layer), _ptr(x), int(x.shape[-1]), int(C), _ptr(w_qkv),
+                                   _ptr(ve), _ptr(gate), _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out),
+                                   _ptr(v_out), _ptr(rstd_q), _ptr(rstd_k), _stream(stream)))
+
+
+def attn_qkv_bwd(spec: LayerSpec, x, C, w_qkv, dQ, dK, dV, dx, dw_qkv, stream=None):
+    """dx (B, T, C) and float32 dw_qkv of the projection from attn_bwd's dQ, dK, dV."""
+    layer = spec.c()
+    _check(lib().attn_qkv_bwd(ctypes.byref(layer), _ptr(x), int(x.shape[-1]), int(C), _ptr(w_qkv),
+                              _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dx), _ptr(dw_qkv), _stream(stream)))
 
 
 def attn_fwd(spec: LayerSpec, q_out, k_out, v_out, O, lse, stream=None):

@@ -24,6 +24,7 @@
 #include "decode.cuh"
 #include "gate.cuh"
 #include "gemm_sm100.cuh"
+#include "qkv_sm100.cuh"
 
 using namespace cswattn;
 
@@ -190,6 +191,26 @@ cswattn_status make_map_2d(CUtensorMap* map, const void* base, long long inner, 
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CSWATTN_OK;
+}
+
+// Tensor map of a bf16 (rows, heads, D) row-major tensor (tokens flattened),
+// viewed as 3-D (D, heads, rows); a box is one 128-byte column panel of
+// `box_rows` rows of one head (128B swizzle); rows past the end are not
+// written by stores.
+cswattn_status make_map_3d(CUtensorMap* map, const void* base, long long rows, int heads, int D, int box_rows) {
+  EncodeTiledFn enc;
+  cswattn_status s = get_encoder(&enc);
+  if (s != CSWATTN_OK) return s;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(heads) * D * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -521,6 +542,7 @@ struct GemmArgs {
   long long lda, ldb, ldd, ldc;
   float alpha, beta;
   void* C;
+  bool c_f32 = false;  // C is float32 (else bf16)
 };
 
 cswattn_status check_gemm(const GemmArgs& g) {
@@ -532,6 +554,7 @@ cswattn_status check_gemm(const GemmArgs& g) {
     return fail(CSWATTN_ERR_INVALID_ARG, "a leading dimension is smaller than its row");
   if (g.lda % 8 || g.ldb % 8 || g.ldc % 8 || (g.beta != 0.f && g.ldd % 8))
     return fail(CSWATTN_ERR_INVALID_ARG, "leading dimensions must be multiples of 8 elements");
+  if (g.c_f32 && g.beta != 0.f) return fail(CSWATTN_ERR_UNSUPPORTED, "a float32 C takes no beta D term");
   CHECK_PTR(g.A, 16);
   CHECK_PTR(g.B, 16);
   CHECK_PTR(g.C, 16);
@@ -575,7 +598,8 @@ cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st) {
   gp.beta = g.beta;
   gp.D = static_cast<const __nv_bfloat16*>(g.D);
   gp.ldd = g.ldd;
-  gp.C = static_cast<__nv_bfloat16*>(g.C);
+  gp.C = g.c_f32 ? nullptr : static_cast<__nv_bfloat16*>(g.C);
+  gp.C32 = g.c_f32 ? static_cast<float*>(g.C) : nullptr;
   gp.ldc = g.ldc;
   gp.wait_ns = g_wait_ns.load();
   const dim3 grid((g.N + gemm::kBN - 1) / gemm::kBN, (g.M + gemm::kBM - 1) / gemm::kBM);
@@ -1217,6 +1241,105 @@ cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, 
     if ((e = run_gemm(g3, cs)) != CSWATTN_OK) return e;
     cur = out;
   }
+  return CSWATTN_OK;
+}
+
+cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                                 const void* w_qkv, const void* ve, const void* gate, void* q, void* k,
+                                 void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                 void* stream) {
+  const NvtxRange nvtx_range("attn_qkv_prologue");
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  if (!s.bf16) return fail(CSWATTN_ERR_UNSUPPORTED, "attn_qkv_prologue supports bf16 layers only");
+  if (C < 1 || C % 8 != 0 || x_stride < C || x_stride % 8 != 0)
+    return fail(CSWATTN_ERR_INVALID_ARG, "C must be a positive multiple of 8 and x_stride >= C a multiple of 8");
+  const long long BT = static_cast<long long>(s.B) * s.T;
+  if (BT > 65535ll * qkv::kBM) return fail(CSWATTN_ERR_UNSUPPORTED, "too many tokens (%lld)", BT);
+  CHECK_PTR(x, 16);
+  CHECK_PTR(w_qkv, 16);
+  CHECK_PTR(q, 16);
+  CHECK_PTR(k, 16);
+  CHECK_PTR(q_out, 16);
+  CHECK_PTR(k_out, 16);
+  CHECK_PTR(v_out, 16);
+  CHECK_PTR(rstd_q, 4);
+  CHECK_PTR(rstd_k, 4);
+  if (layer->has_ve) {
+    CHECK_PTR(ve, 16);
+    CHECK_PTR(gate, 2);
+  }
+  const int nh = s.H + 2 * s.Hk;
+  CUtensorMap mx, mw, mq, mk, mqo, mko, mvo;
+  if ((st = make_map_2d(&mx, x, C, BT, x_stride, 64, qkv::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map_2d(&mw, w_qkv, C, static_cast<long long>(nh) * s.D, C, 64, s.D)) != CSWATTN_OK) return st;
+  if ((st = make_map_3d(&mq, q, BT, s.H, s.D, qkv::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map_3d(&mk, k, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map_3d(&mqo, q_out, BT, s.H, s.D, qkv::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map_3d(&mko, k_out, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
+  if ((st = make_map_3d(&mvo, v_out, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
+  if ((st = s.D == 64 ? set_smem(qkv::qkv_kernel<64>, qkv::kSmemBytes) : set_smem(qkv::qkv_kernel<128>, qkv::kSmemBytes)) !=
+      CSWATTN_OK)
+    return st;
+  qkv::Params qp;
+  qp.BT = static_cast<int>(BT);
+  qp.T = s.T;
+  qp.H = s.H;
+  qp.Hk = s.Hk;
+  qp.C = C;
+  qp.has_ve = layer->has_ve;
+  qp.eps = layer->eps;
+  fill_omega(qp.omega, s.D, layer->rope_base);
+  qp.ve = static_cast<const __nv_bfloat16*>(ve);
+  qp.gate = static_cast<const __nv_bfloat16*>(gate);
+  qp.rstd_q = rstd_q;
+  qp.rstd_k = rstd_k;
+  qp.wait_ns = g_wait_ns.load();
+  const dim3 grid(static_cast<unsigned>(nh), static_cast<unsigned>((BT + qkv::kBM - 1) / qkv::kBM));
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  {
+    ScopedTiming tm(CSWATTN_K_PROLOGUE, cs);
+    if (s.D == 64)
+      launch_pdl(qkv::qkv_kernel<64>, grid, dim3(qkv::kThreads), qkv::kSmemBytes, cs, mx, mw, mq, mk, mqo, mko, mvo, qp);
+    else
+      launch_pdl(qkv::qkv_kernel<128>, grid, dim3(qkv::kThreads), qkv::kSmemBytes, cs, mx, mw, mq, mk, mqo, mko, mvo, qp);
+  }
+  return launched("QKV projection launch");
+}
+
+cswattn_status attn_qkv_bwd(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                            const void* w_qkv, const void* dQ, const void* dK, const void* dV, void* dx,
+                            float* dw_qkv, void* stream) {
+  const NvtxRange nvtx_range("attn_qkv_bwd");
+  Shape s;
+  cswattn_status st = check_layer(layer, &s);
+  if (st != CSWATTN_OK) return st;
+  if (!s.bf16) return fail(CSWATTN_ERR_UNSUPPORTED, "attn_qkv_bwd supports bf16 layers only");
+  if (C < 1 || C % 8 != 0 || x_stride < C || x_stride % 8 != 0)
+    return fail(CSWATTN_ERR_INVALID_ARG, "C must be a positive multiple of 8 and x_stride >= C a multiple of 8");
+  const long long BT = static_cast<long long>(s.B) * s.T;
+  if (BT > (1ll << 30)) return fail(CSWATTN_ERR_UNSUPPORTED, "too many tokens");
+  CHECK_PTR(dx, 16);
+  CHECK_PTR(dw_qkv, 16);
+  const int M = static_cast<int>(BT);
+  const long long hq = static_cast<long long>(s.H) * s.D, hk = static_cast<long long>(s.Hk) * s.D;
+  const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(w_qkv);
+  // dx = dQ W_q + dK W_k + dV W_v (W_* rows of the stacked weight, MN-major operands).
+  const GemmArgs g[6] = {
+      {M, C, static_cast<int>(hq), false, true, dQ, w, nullptr, hq, C, 0, C, 1.f, 0.f, dx},
+      {M, C, static_cast<int>(hk), false, true, dK, w + hq * C, dx, hk, C, C, C, 1.f, 1.f, dx},
+      {M, C, static_cast<int>(hk), false, true, dV, w + (hq + hk) * C, dx, hk, C, C, C, 1.f, 1.f, dx},
+      // dW_q = dQ^T x, dW_k = dK^T x, dW_v = dV^T x (float32 rows of the stacked gradient).
+      {static_cast<int>(hq), C, M, true, true, dQ, x, nullptr, hq, x_stride, 0, C, 1.f, 0.f, dw_qkv, true},
+      {static_cast<int>(hk), C, M, true, true, dK, x, nullptr, hk, x_stride, 0, C, 1.f, 0.f, dw_qkv + hq * C, true},
+      {static_cast<int>(hk), C, M, true, true, dV, x, nullptr, hk, x_stride, 0, C, 1.f, 0.f, dw_qkv + (hq + hk) * C, true},
+  };
+  for (const auto& a : g)
+    if ((st = check_gemm(a)) != CSWATTN_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  for (const auto& a : g)
+    if ((st = run_gemm(a, cs)) != CSWATTN_OK) return st;
   return CSWATTN_OK;
 }
 

@@ -9,7 +9,7 @@
 // A[k][m] of a row-major (K x M) A (MN-major, A_MN = true); Bop[n][k] is
 // B[n][k] of a row-major (N x K) B or B[k][n] of a row-major (K x N) B. So
 // X^T X is A_MN = B_MN = true with A = B = X, and X B is A_MN = false,
-// B_MN = true. bf16 inputs and outputs (C, D), float32 accumulation.
+// B_MN = true. bf16 inputs and D, bf16 (or float32) C, float32 accumulation.
 //
 // One CTA per 128 x 128 tile of C. Warp 0 (one thread) loads 64-wide K
 // chunks of both operands by TMA into a 6-stage ring (128B swizzle: a
@@ -39,7 +39,8 @@ struct Params {
   float alpha, beta;
   const __nv_bfloat16* D;  // (M x N) row-major with ldd, or null when beta == 0
   long long ldd;
-  __nv_bfloat16* C;        // (M x N) row-major with ldc
+  __nv_bfloat16* C;        // (M x N) row-major with ldc (bf16 output), or null
+  float* C32;              // (M x N) row-major with ldc (float32 output), or null
   long long ldc;
   unsigned long long wait_ns;
 };
@@ -180,12 +181,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[2 * e + 1] = fmaf(p.beta, f.y, v[2 * e + 1]);
             }
           }
-          uint4 w;
-          w.x = pack_bf16x2(v[0], v[1]);
-          w.y = pack_bf16x2(v[2], v[3]);
-          w.z = pack_bf16x2(v[4], v[5]);
-          w.w = pack_bf16x2(v[6], v[7]);
-          *reinterpret_cast<uint4*>(p.C + m * p.ldc + n) = w;
+          if (p.C32) {
+            float4* dst = reinterpret_cast<float4*>(p.C32 + m * p.ldc + n);
+            dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+            dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+          } else {
+            uint4 w;
+            w.x = pack_bf16x2(v[0], v[1]);
+            w.y = pack_bf16x2(v[2], v[3]);
+            w.z = pack_bf16x2(v[4], v[5]);
+            w.w = pack_bf16x2(v[6], v[7]);
+            *reinterpret_cast<uint4*>(p.C + m * p.ldc + n) = w;
+          }
         }
       }
     }

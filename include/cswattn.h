@@ -126,6 +126,35 @@ cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long lon
                              int gate_channels, const void* w_gate, const void* dgate, void* dx,
                              float* dw_gate, void* stream);
 
+/* The QKV projection fused with the prologue: page section "1. GPT 모델
+ * (nanochat/gpt.py)", where the block input is projected to the query, key
+ * and value heads by bias-free Linear layers before RoPE, QK normalisation
+ * and the value residual. With the stacked weight w_qkv ((n_head +
+ * 2 n_kv_head) * head_dim rows, C columns; rows: the query heads, then the
+ * key heads, then the value heads, each head_dim rows):
+ *   y = x[..., :C] w_qkv^T, rounded to bf16, split into q (B, T, n_head, D),
+ *   k and v (B, T, n_kv_head, D);
+ *   q, k: written raw (attn_bwd needs them); q_out, k_out, rstd_q, rstd_k,
+ *   v_out as attn_prologue computes them from (q, k, v, ve, gate).
+ * x: (B, T, x_stride) bf16, columns [0, C) read; C and x_stride multiples
+ * of 8. bf16 layers only; ve and gate only when has_ve. One kernel: the
+ * product on the tensor cores with RMSNorm, RoPE and the value residual in
+ * its epilogue. */
+cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                                 const void* w_qkv, const void* ve, const void* gate, void* q, void* k,
+                                 void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                 void* stream);
+
+/* Backward of the projection (same page section), given attn_bwd's dQ, dK,
+ * dV (gradients of the raw q, k, v):
+ *   dx     = dQ w_q + dK w_k + dV w_v         (B, T, C), bf16, row stride C
+ *   dw_qkv = [dQ dK dV]^T x[..., :C]           ((n_head + 2 n_kv_head) D, C), float32
+ * Six tensor-core matrix products (cswattn_gemm_bf16). x, x_stride, C,
+ * w_qkv as for attn_qkv_prologue; bf16 layers only. */
+cswattn_status attn_qkv_bwd(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                            const void* w_qkv, const void* dQ, const void* dK, const void* dV, void* dx,
+                            float* dw_qkv, void* stream);
+
 /* Forward: O_i = sum_j softmax_j(scale * q_out_i . k_out_j) v_out_j over the
  * causal window, and lse_i = log sum_j exp(scale * q_out_i . k_out_j).
  * Page section "5. 플래시 어텐션 통합" (causal call with window_size).

@@ -248,3 +248,16 @@ def test_checked_build_compiles_and_exports_the_same_symbols():
     checked = ctypes.CDLL(path)
     for n in declared_functions():
         assert hasattr(checked, n), n
+
+
+def test_qkv_entry_point_validation(lib):
+    ptrs = [256 * (i + 1) for i in range(12)]
+    spec = cs.LayerSpec(1, 16, 2, 1, 128, 16, has_ve=False)
+    f32 = cs.LayerSpec(1, 16, 2, 1, 64, 16, has_ve=False, dtype="f32")
+    qp = lib.attn_qkv_prologue
+    assert qp(ctypes.byref(f32.c()), ptrs[0], 64, 64, *ptrs[1:11], None) == cs.ERR_UNSUPPORTED
+    assert qp(ctypes.byref(spec.c()), ptrs[0], 64, 60, *ptrs[1:11], None) == cs.ERR_INVALID_ARG  # C % 8
+    assert qp(ctypes.byref(spec.c()), ptrs[0], 32, 64, *ptrs[1:11], None) == cs.ERR_INVALID_ARG  # stride < C
+    qb = lib.attn_qkv_bwd
+    assert qb(ctypes.byref(f32.c()), ptrs[0], 64, 64, *ptrs[1:7], None) == cs.ERR_UNSUPPORTED
+    assert qb(ctypes.byref(spec.c()), ptrs[0], 64, 60, *ptrs[1:7], None) == cs.ERR_INVALID_ARG
