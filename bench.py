@@ -443,6 +443,8 @@ def run_ours(args):
             line["decode"] = decode_bench(w, dev, peaks, steps=args.steps, warmup=args.warmup,
                                           peak_src=peak_src)
         if solo and not args.no_muon:
+            line["qkv_projection"] = qkv_bench(w, dev, peaks, peak_src, steps=args.steps, warmup=args.warmup)
+        if solo and not args.no_muon:
             line["muon_ns"] = muon_bench(dev, peaks, peak_src, steps=args.steps, warmup=args.warmup)
         if solo and not args.no_other_configs:
             del st
@@ -597,6 +599,60 @@ def muon_bench(dev, peaks, peak_src, steps=20, warmup=5):
     return out
 
 
+def qkv_bench(w, dev, peaks, peak_src, steps=20, warmup=5):
+    """The step before the attention path at the workload's layer shape: the
+    QKV projection of the block input (model dim = n_head * head_dim) fused
+    with the prologue, and its backward (dx, dW), device time per call."""
+    import torch
+
+    import causal_sliding_window_rope_b200 as cs
+    B, T, H, Hk, D = w.B, w.T, w.H, w.Hk, w.D
+    C = H * D
+    g = torch.Generator().manual_seed(4323)
+    bf = torch.bfloat16
+    spec = cs.LayerSpec(B, T, H, Hk, D, w.windows[0], has_ve=True, rope_base=w.rope_base, eps=w.eps)
+    x = torch.randn(B, T, C, generator=g).to(bf).to(dev)
+    wq = (torch.randn((H + 2 * Hk) * D, C, generator=g) / C ** 0.5).to(bf).to(dev)
+    ve = torch.randn(B, T, Hk, D, generator=g).to(bf).to(dev)
+    gate = torch.randn(B, T, Hk, generator=g).to(bf).to(dev)
+    buf = cs.LayerBuffers(spec, device=dev)
+    q = torch.empty(B, T, H, D, dtype=bf, device=dev)
+    k = torch.empty(B, T, Hk, D, dtype=bf, device=dev)
+    dx = torch.empty(B, T, C, dtype=bf, device=dev)
+    dw = torch.empty((H + 2 * Hk) * D, C, dtype=torch.float32, device=dev)
+
+    def fwd():
+        cs.attn_qkv_prologue(spec, x, C, wq, ve, gate, q, k, buf.q_out, buf.k_out, buf.v_out,
+                             buf.rstd_q, buf.rstd_k)
+
+    def bwd():
+        cs.attn_qkv_bwd(spec, x, C, wq, q, k, buf.v_out, dx, dw)  # any bf16 gradients of that shape
+
+    out = {}
+    flops = 2.0 * B * T * C * (H + 2 * Hk) * D
+    stream = torch.cuda.current_stream(dev)
+    for name, fn, fl in (("fwd", fwd, flops), ("bwd", bwd, 2 * flops)):
+        for _ in range(max(warmup, 3)):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / steps
+        out[name] = {"ms_per_call": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
+    cs.cswattn_sync_status()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    return {"workload": f"QKV projection of the layer input (B={B} T={T} C={C} -> {H}+2x{Hk} heads of {D}) "
+                        f"fused with the prologue (fwd), and its backward dx, dW (bwd)",
+            **out, "roofline": {"kernel": "qkv fused product", "bound": "tensor",
+                                "achieved": out["fwd"]["tflops"], "peak": peak, "unit": "TFLOP/s",
+                                "frac": round(out["fwd"]["tflops"] / peak, 4),
+                                "peak_source": f"{peak_src} bf16_tflops"}}
+
+
 def traffic_for(kind):
     """DRAM bytes per launch from a committed ncu capture, if the kernel's
     source still matches the one the counters were taken on; else None."""
@@ -723,7 +779,8 @@ def main():
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the device-timed summary of the other bf16 workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-muon", action="store_true", help="skip the Newton-Schulz measurement")
+    ap.add_argument("--no-muon", action="store_true",
+                    help="skip the Newton-Schulz and QKV-projection measurements")
     ap.add_argument("--muon-only", action="store_true",
                     help="profiling case: only the Newton-Schulz measurement")
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")
