@@ -331,3 +331,49 @@ def qkv_projection_bwd(x, w_qkv, dq, dk, dv):
     dy = np.concatenate([_f64(dq).reshape(B * T, -1), _f64(dk).reshape(B * T, -1),
                          _f64(dv).reshape(B * T, -1)], axis=1)
     return (dy @ w).reshape(B, T, C), dy.T @ x.reshape(B * T, C)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) projection
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(v):
+    """Nearest FP8 E4M3 value (OCP 8-bit floating point: 1 sign, 4 exponent
+    bits with bias 7, 3 mantissa bits; largest finite 448, smallest subnormal
+    2^-9), ties to even, magnitudes above 448 saturated to 448."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    out = np.zeros_like(a)
+    sub = a < 2.0 ** -6                      # subnormal range: steps of 2^-9
+    out[sub] = np.round(a[sub] / 2.0 ** -9) * 2.0 ** -9   # numpy rounds halves to even
+    nrm = ~sub
+    e = np.floor(np.log2(np.where(nrm, a, 1.0)))
+    step = 2.0 ** (e - 3)                    # 3 mantissa bits below the leading one
+    out[nrm] = (np.round(a / step) * step)[nrm]
+    out = np.minimum(out, E4M3_MAX)
+    return np.sign(v) * out
+
+
+def fp8_tensor_scale(x):
+    """Tensor-wise scale of a tensor for E4M3: amax / 448 in float32 (1 when
+    the tensor is zero)."""
+    amax = np.float32(np.max(np.abs(np.asarray(x, dtype=np.float32))))
+    return np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(E4M3_MAX))
+
+
+def quantize_e4m3(x, scale):
+    """E4M3 values of x / scale, the division in float32 (returns float64
+    copies of the FP8 values)."""
+    return e4m3_round(np.asarray(x, dtype=np.float32) / np.float32(scale))
+
+
+def qkv_projection_fp8(x, w_qkv, H, Hk, D):
+    """The QKV projection with both operands quantized to E4M3 with
+    tensor-wise scales (a Float8Linear with tensor-wise scaling):
+    y = (Q(x / sx) Q(w / sw)^T) sx sw. Returns q, k, v and (sx, sw)."""
+    sx, sw = fp8_tensor_scale(x), fp8_tensor_scale(w_qkv)
+    xq = quantize_e4m3(x, sx) * np.float64(sx)
+    wq = quantize_e4m3(w_qkv, sw) * np.float64(sw)
+    q, k, v = qkv_projection(xq, wq, H, Hk, D)
+    return q, k, v, (float(sx), float(sw))

@@ -534,3 +534,40 @@ def test_qkv_projection_gradients_match_central_differences():
         wm[o, c] -= h
         fd = (loss(x, wp) - loss(x, wm)) / (2 * h)
         assert abs(fd - dw[o, c]) <= 1e-6 * max(1.0, abs(dw[o, c])), ("w", o, c)
+
+
+# ---------------------------------------------------------------- FP8 E4M3
+
+def test_e4m3_values_from_the_format_definition():
+    """Codes worked from the E4M3 layout (bias 7, 3 mantissa bits): the
+    largest finite value, the subnormals, exact values, ties to even and
+    saturation."""
+    cases = {448.0: 448.0, 500.0: 448.0, -1e6: -448.0, 2.0 ** -9: 2.0 ** -9, 2.0 ** -10: 0.0,
+             3 * 2.0 ** -10: 2.0 ** -8, 1.0: 1.0, 1.0625: 1.0, 1.1875: 1.25, 1.125: 1.125,
+             17.0: 16.0, 19.0: 20.0, -2.75: -2.75, 0.3: 0.3125, 240.0: 240.0, 232.0: 224.0}
+    for v, want in cases.items():
+        assert oracle.e4m3_round(v) == want, (v, oracle.e4m3_round(v), want)
+
+
+def test_e4m3_matches_torch_float8_conversion():
+    """Against torch's float8_e4m3fn conversion (a library routine the oracle
+    does not use) on values inside the finite range."""
+    v = np.concatenate([rnd(20000, 110) * 30, rnd(5000, 111) * 0.01, np.linspace(-448, 448, 4001)])
+    t = torch.tensor(v, dtype=torch.float32).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(oracle.e4m3_round(np.float32(v).astype(np.float64)), t)
+
+
+def test_fp8_projection_is_the_projection_of_the_dequantized_operands():
+    B, T, C, H, Hk, D = 1, 6, 16, 2, 1, 8
+    x = rnd((B, T, C), 112)
+    w = rnd(((H + 2 * Hk) * D, C), 113) / 4
+    q, k, v, (sx, sw) = oracle.qkv_projection_fp8(x, w, H, Hk, D)
+    assert sx == np.float32(np.abs(np.float32(x)).max() / np.float32(448))
+    xq = oracle.e4m3_round(np.float32(x) / np.float32(sx)) * sx
+    wq = oracle.e4m3_round(np.float32(w) / np.float32(sw)) * sw
+    assert np.all(np.abs(np.float32(x) / np.float32(sx)) <= 448.0001)
+    rq, rk, rv = oracle.qkv_projection(xq, wq, H, Hk, D)
+    np.testing.assert_array_equal(q, rq)
+    # quantization error of the operands is small against the unquantized projection
+    fq, _, _ = oracle.qkv_projection(x, w, H, Hk, D)
+    assert np.linalg.norm(q - fq) / np.linalg.norm(fq) < 0.1
