@@ -628,10 +628,17 @@ def qkv_bench(w, dev, peaks, peak_src, steps=20, warmup=5):
     def bwd():
         cs.attn_qkv_bwd(spec, x, C, wq, q, k, buf.v_out, dx, dw)  # any bf16 gradients of that shape
 
+    scales = torch.empty(2, dtype=torch.float32, device=dev)
+    ws8 = torch.empty(cs.attn_qkv_fp8_workspace_bytes(spec, C), dtype=torch.uint8, device=dev)
+
+    def fwd_fp8():
+        cs.attn_qkv_prologue_fp8(spec, x, C, wq, ve, gate, q, k, buf.q_out, buf.k_out, buf.v_out,
+                                 buf.rstd_q, buf.rstd_k, scales, ws8)
+
     out = {}
     flops = 2.0 * B * T * C * (H + 2 * Hk) * D
     stream = torch.cuda.current_stream(dev)
-    for name, fn, fl in (("fwd", fwd, flops), ("bwd", bwd, 2 * flops)):
+    for name, fn, fl in (("fwd", fwd, flops), ("bwd", bwd, 2 * flops), ("fwd_fp8", fwd_fp8, flops)):
         for _ in range(max(warmup, 3)):
             fn()
         torch.cuda.synchronize(dev)
@@ -645,8 +652,12 @@ def qkv_bench(w, dev, peaks, peak_src, steps=20, warmup=5):
         out[name] = {"ms_per_call": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
     cs.cswattn_sync_status()
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    # E4M3 call: amax, quantization and the fused product; against the FP8
+    # tensor peak taken as twice the bf16 one (the nominal dense ratio).
+    out["fwd_fp8"]["frac_of_fp8_peak"] = round(out["fwd_fp8"]["tflops"] / (2 * peak), 4)
     return {"workload": f"QKV projection of the layer input (B={B} T={T} C={C} -> {H}+2x{Hk} heads of {D}) "
-                        f"fused with the prologue (fwd), and its backward dx, dW (bwd)",
+                        f"fused with the prologue (fwd; fwd_fp8 with E4M3 operands and tensor-wise "
+                        f"scales, quantization included), and its backward dx, dW (bwd)",
             **out, "roofline": {"kernel": "qkv fused product", "bound": "tensor",
                                 "achieved": out["fwd"]["tflops"], "peak": peak, "unit": "TFLOP/s",
                                 "frac": round(out["fwd"]["tflops"] / peak, 4),

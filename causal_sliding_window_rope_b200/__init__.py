@@ -30,7 +30,7 @@ F32, BF16 = 0, 1
 
 # Every symbol the header declares; the CPU tests check the library exports them.
 EXPORTS = ("attn_prologue", "attn_prologue_gated", "attn_gate_bwd", "attn_qkv_prologue",
-           "attn_qkv_bwd", "attn_fwd",
+           "attn_qkv_fp8_workspace_bytes", "attn_qkv_prologue_fp8", "attn_qkv_bwd", "attn_fwd",
            "attn_bwd_workspace_bytes", "attn_bwd", "attn_bwd_noalloc",
            "attn_decode_workspace_bytes", "attn_decode", "cswattn_gemm_bf16",
            "muon_ns_workspace_bytes", "muon_newton_schulz",
@@ -75,6 +75,10 @@ def lib():
         L.attn_gate_bwd.argtypes = [lp, vp, ll, ci, vp, vp, vp, fp, vp]
         L.attn_qkv_prologue.argtypes = [lp, vp, ll, ci] + [vp] * 8 + [fp, fp, vp]
         L.attn_qkv_prologue.restype = ci
+        L.attn_qkv_fp8_workspace_bytes.argtypes = [lp, ci]
+        L.attn_qkv_fp8_workspace_bytes.restype = sz
+        L.attn_qkv_prologue_fp8.argtypes = [lp, vp, ll, ci] + [vp] * 8 + [fp, fp, fp, vp, sz, vp]
+        L.attn_qkv_prologue_fp8.restype = ci
         L.attn_qkv_bwd.argtypes = [lp, vp, ll, ci] + [vp] * 5 + [fp, vp]
         L.attn_qkv_bwd.restype = ci
         cf = ctypes.c_float
@@ -189,6 +193,23 @@ def attn_qkv_prologue(spec: LayerSpec, x, C, w_qkv, ve, gate, q, k, q_out, k_out
     _check(lib().attn_qkv_prologue(ctypes.byref(layer), _ptr(x), int(x.shape[-1]), int(C), _ptr(w_qkv),
                                    _ptr(ve), _ptr(gate), _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out),
                                    _ptr(v_out), _ptr(rstd_q), _ptr(rstd_k), _stream(stream)))
+
+
+def attn_qkv_fp8_workspace_bytes(spec: LayerSpec, C) -> int:
+    layer = spec.c()
+    return int(lib().attn_qkv_fp8_workspace_bytes(ctypes.byref(layer), int(C)))
+
+
+def attn_qkv_prologue_fp8(spec: LayerSpec, x, C, w_qkv, ve, gate, q, k, q_out, k_out, v_out, rstd_q,
+                          rstd_k, scales, workspace, workspace_bytes=None, stream=None):
+    """attn_qkv_prologue with both operands quantized to E4M3 with tensor-wise
+    scales (written to `scales`); `workspace` holds the codes afterwards."""
+    layer = spec.c()
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(lib().attn_qkv_prologue_fp8(ctypes.byref(layer), _ptr(x), int(x.shape[-1]), int(C), _ptr(w_qkv),
+                                       _ptr(ve), _ptr(gate), _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out),
+                                       _ptr(v_out), _ptr(rstd_q), _ptr(rstd_k), _ptr(scales), _ptr(workspace),
+                                       int(nbytes), _stream(stream)))
 
 
 def attn_qkv_bwd(spec: LayerSpec, x, C, w_qkv, dQ, dK, dV, dx, dw_qkv, stream=None):

@@ -25,6 +25,7 @@
 #include "gate.cuh"
 #include "gemm_sm100.cuh"
 #include "qkv_sm100.cuh"
+#include "fp8.cuh"
 
 using namespace cswattn;
 
@@ -177,20 +178,21 @@ cswattn_status make_map(CUtensorMap* map, const void* base, int outer, int T, in
   return CSWATTN_OK;
 }
 
-// Tensor map of a row-major bf16 matrix of `rows` rows of `inner`
-// contiguous elements, `ld` elements apart, viewed as 2-D (inner, rows);
-// a box is box_inner x box_rows (128B swizzle, box_inner = 64), out-of-range
-// elements read as zero.
+// Tensor map of a row-major bf16 (or, with `bytes`, 8-bit) matrix of
+// `rows` rows of `inner` contiguous elements, `ld` elements apart, viewed as
+// 2-D (inner, rows); a box is box_inner x box_rows (128B swizzle: 128-byte
+// box rows), out-of-range elements read as zero.
 cswattn_status make_map_2d(CUtensorMap* map, const void* base, long long inner, long long rows, long long ld,
-                           int box_inner, int box_rows) {
+                           int box_inner, int box_rows, bool bytes = false) {
   EncodeTiledFn enc;
   cswattn_status s = get_encoder(&enc);
   if (s != CSWATTN_OK) return s;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * (bytes ? 1 : 2)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSWATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -1244,17 +1246,45 @@ cswattn_status muon_newton_schulz(int m, int n, const float* coeffs, int steps, 
   return CSWATTN_OK;
 }
 
-cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long long x_stride, int C,
-                                 const void* w_qkv, const void* ve, const void* gate, void* q, void* k,
-                                 void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
-                                 void* stream) {
-  const NvtxRange nvtx_range("attn_qkv_prologue");
+}  // extern "C"
+
+namespace {
+
+// Workspace of the FP8 projection: the two operands' amax bit patterns, then
+// the E4M3 codes of x (B*T x C) and of W ((H + 2 Hk) D x C).
+struct Fp8Workspace {
+  unsigned int* amax;
+  uint8_t *x8, *w8;
+  size_t bytes;
+};
+
+Fp8Workspace carve_fp8(const Shape& s, int C, void* base) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  Fp8Workspace w;
+  size_t off = 0;
+  w.amax = reinterpret_cast<unsigned int*>(p + off);
+  off += 256;
+  w.x8 = p + off;
+  off += pad256(static_cast<size_t>(s.B) * s.T * C);
+  w.w8 = p + off;
+  off += pad256(static_cast<size_t>(s.H + 2 * s.Hk) * s.D * C);
+  w.bytes = off;
+  return w;
+}
+
+// The fused projection; with `f8` (workspace and scales) the operands are
+// first quantized to E4M3 with tensor-wise scales.
+cswattn_status qkv_impl(const cswattn_layer* layer, const void* x, long long x_stride, int C, const void* w_qkv,
+                        const void* ve, const void* gate, void* q, void* k, void* q_out, void* k_out, void* v_out,
+                        float* rstd_q, float* rstd_k, float* scales, void* workspace, size_t workspace_bytes,
+                        bool f8, void* stream) {
   Shape s;
   cswattn_status st = check_layer(layer, &s);
   if (st != CSWATTN_OK) return st;
-  if (!s.bf16) return fail(CSWATTN_ERR_UNSUPPORTED, "attn_qkv_prologue supports bf16 layers only");
+  if (!s.bf16) return fail(CSWATTN_ERR_UNSUPPORTED, "the QKV projection supports bf16 layers only");
   if (C < 1 || C % 8 != 0 || x_stride < C || x_stride % 8 != 0)
     return fail(CSWATTN_ERR_INVALID_ARG, "C must be a positive multiple of 8 and x_stride >= C a multiple of 8");
+  if (f8 && C % 16 != 0) return fail(CSWATTN_ERR_INVALID_ARG, "the FP8 projection needs C a multiple of 16");
   const long long BT = static_cast<long long>(s.B) * s.T;
   if (BT > 65535ll * qkv::kBM) return fail(CSWATTN_ERR_UNSUPPORTED, "too many tokens (%lld)", BT);
   CHECK_PTR(x, 16);
@@ -1270,18 +1300,32 @@ cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long
     CHECK_PTR(ve, 16);
     CHECK_PTR(gate, 2);
   }
+  Fp8Workspace fw{};
+  if (f8) {
+    CHECK_PTR(scales, 4);
+    CHECK_PTR(workspace, 256);
+    fw = carve_fp8(s, C, workspace);
+    if (workspace_bytes < fw.bytes)
+      return fail(CSWATTN_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes, fw.bytes);
+  }
   const int nh = s.H + 2 * s.Hk;
   CUtensorMap mx, mw, mq, mk, mqo, mko, mvo;
-  if ((st = make_map_2d(&mx, x, C, BT, x_stride, 64, qkv::kBM)) != CSWATTN_OK) return st;
-  if ((st = make_map_2d(&mw, w_qkv, C, static_cast<long long>(nh) * s.D, C, 64, s.D)) != CSWATTN_OK) return st;
+  if (f8) {
+    if ((st = make_map_2d(&mx, fw.x8, C, BT, C, 128, qkv::kBM, true)) != CSWATTN_OK) return st;
+    if ((st = make_map_2d(&mw, fw.w8, C, static_cast<long long>(nh) * s.D, C, 128, s.D, true)) != CSWATTN_OK)
+      return st;
+  } else {
+    if ((st = make_map_2d(&mx, x, C, BT, x_stride, 64, qkv::kBM)) != CSWATTN_OK) return st;
+    if ((st = make_map_2d(&mw, w_qkv, C, static_cast<long long>(nh) * s.D, C, 64, s.D)) != CSWATTN_OK) return st;
+  }
   if ((st = make_map_3d(&mq, q, BT, s.H, s.D, qkv::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map_3d(&mk, k, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map_3d(&mqo, q_out, BT, s.H, s.D, qkv::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map_3d(&mko, k_out, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map_3d(&mvo, v_out, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
-  if ((st = s.D == 64 ? set_smem(qkv::qkv_kernel<64>, qkv::kSmemBytes) : set_smem(qkv::qkv_kernel<128>, qkv::kSmemBytes)) !=
-      CSWATTN_OK)
-    return st;
+  auto kern = s.D == 64 ? (f8 ? qkv::qkv_kernel<64, true> : qkv::qkv_kernel<64, false>)
+                        : (f8 ? qkv::qkv_kernel<128, true> : qkv::qkv_kernel<128, false>);
+  if ((st = set_smem(kern, qkv::kSmemBytes)) != CSWATTN_OK) return st;
   qkv::Params qp;
   qp.BT = static_cast<int>(BT);
   qp.T = s.T;
@@ -1295,17 +1339,63 @@ cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long
   qp.gate = static_cast<const __nv_bfloat16*>(gate);
   qp.rstd_q = rstd_q;
   qp.rstd_k = rstd_k;
+  qp.scales = f8 ? scales : nullptr;
   qp.wait_ns = g_wait_ns.load();
   const dim3 grid(static_cast<unsigned>(nh), static_cast<unsigned>((BT + qkv::kBM - 1) / qkv::kBM));
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   {
     ScopedTiming tm(CSWATTN_K_PROLOGUE, cs);
-    if (s.D == 64)
-      launch_pdl(qkv::qkv_kernel<64>, grid, dim3(qkv::kThreads), qkv::kSmemBytes, cs, mx, mw, mq, mk, mqo, mko, mvo, qp);
-    else
-      launch_pdl(qkv::qkv_kernel<128>, grid, dim3(qkv::kThreads), qkv::kSmemBytes, cs, mx, mw, mq, mk, mqo, mko, mvo, qp);
+    if (f8) {
+      // Tensor-wise scales, then the E4M3 codes of both operands.
+      Fp8QuantParams fq;
+      fq.a = static_cast<const __nv_bfloat16*>(x);
+      fq.rows_a = BT;
+      fq.lda = x_stride;
+      fq.b = static_cast<const __nv_bfloat16*>(w_qkv);
+      fq.rows_b = static_cast<long long>(nh) * s.D;
+      fq.cols = C;
+      fq.amax_bits = fw.amax;
+      fq.a8 = fw.x8;
+      fq.b8 = fw.w8;
+      fq.scales = scales;
+      const cudaError_t e = cudaMemsetAsync(fw.amax, 0, 2 * sizeof(unsigned int), cs);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+      const long long n8 = (BT + fq.rows_b) * (C / 8);  // 8-element vectors
+      const unsigned g = static_cast<unsigned>(std::min<long long>((n8 + kFp8Threads - 1) / kFp8Threads, 148 * 8));
+      fp8_amax_kernel<<<g, kFp8Threads, 0, cs>>>(fq);  // ordinary launch: strictly after the memset
+      launch_pdl(fp8_quant_kernel, dim3(g), dim3(kFp8Threads), 0, cs, fq);
+    }
+    launch_pdl(kern, grid, dim3(qkv::kThreads), qkv::kSmemBytes, cs, mx, mw, mq, mk, mqo, mko, mvo, qp);
   }
   return launched("QKV projection launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                                 const void* w_qkv, const void* ve, const void* gate, void* q, void* k,
+                                 void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                 void* stream) {
+  const NvtxRange nvtx_range("attn_qkv_prologue");
+  return qkv_impl(layer, x, x_stride, C, w_qkv, ve, gate, q, k, q_out, k_out, v_out, rstd_q, rstd_k, nullptr,
+                  nullptr, 0, false, stream);
+}
+
+size_t attn_qkv_fp8_workspace_bytes(const cswattn_layer* layer, int C) {
+  Shape s;
+  if (check_layer(layer, &s) != CSWATTN_OK || C < 1) return 0;
+  return carve_fp8(s, C, nullptr).bytes;
+}
+
+cswattn_status attn_qkv_prologue_fp8(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                                     const void* w_qkv, const void* ve, const void* gate, void* q, void* k,
+                                     void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                     float* scales, void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("attn_qkv_prologue_fp8");
+  return qkv_impl(layer, x, x_stride, C, w_qkv, ve, gate, q, k, q_out, k_out, v_out, rstd_q, rstd_k, scales,
+                  workspace, workspace_bytes, true, stream);
 }
 
 cswattn_status attn_qkv_bwd(const cswattn_layer* layer, const void* x, long long x_stride, int C,

@@ -9,6 +9,11 @@
 //   y = x W^T with W = [W_q; W_k; W_v] ((H + 2 Hk) D x C), per head
 //   q (raw, bf16) and q~ = RoPE(RMSNorm(q)), likewise k; v_eff = v + 3 s ve.
 //
+// FP8 variant (section "3. 정밀도 관리": Float8Linear with tensor-wise
+// scaling): x and W arrive as E4M3 codes with one scale each, the products
+// are tcgen05.mma kind::f8f6f4 (K = 32 per instruction, 128-element chunks),
+// and the accumulator is multiplied by the two scales before the epilogue.
+//
 // One CTA per (128-token tile, head): the head's D output columns are one
 // N = D tile of the product, so each epilogue thread holds a whole head row
 // (RMSNorm and the RoPE pairs (i, i + D/2) are in-thread). Warp 0 loads
@@ -46,6 +51,7 @@ struct Params {
   const __nv_bfloat16* gate;     // (B*T, Hk) logits
   float* rstd_q;                 // (B*T, H)
   float* rstd_k;                 // (B*T, Hk)
+  const float* scales;           // FP8 variant: scale of x, scale of W
   unsigned long long wait_ns;
 };
 
@@ -64,10 +70,11 @@ __device__ __forceinline__ void stage_row(uint8_t* tile, int r, const float* v) 
   }
 }
 
-// tmX: x as (C, B*T), 64 x 128 boxes. tmW: W as (C, (H+2Hk) D), 64 x HD
-// boxes. tmQ/tmK/tmQo/tmKo/tmVo: the outputs as (D, heads, B*T), 64 x 1 x
-// 128 boxes.
-template <int HD>
+// tmX: x as (C, B*T), 128-byte x 128-row boxes. tmW: W as (C, (H+2Hk) D),
+// 128-byte x HD-row boxes (64 bf16 or 128 E4M3 channels per box).
+// tmQ/tmK/tmQo/tmKo/tmVo: the outputs as (D, heads, B*T), 64 x 1 x 128
+// boxes.
+template <int HD, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     qkv_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -88,7 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   const int hh = static_cast<int>(blockIdx.x);  // stacked head: q heads, then k, then v
   const int m0 = static_cast<int>(blockIdx.y) * kBM;
-  const int nk = (p.C + kBK - 1) / kBK;
+  constexpr int kChunk = FP8 ? 2 * kBK : kBK;  // channels per stage (128 bytes per row)
+  const int nk = (p.C + kChunk - 1) / kChunk;
   const int kind = hh < p.H ? 0 : (hh < p.H + p.Hk ? 1 : 2);
   const int head = kind == 0 ? hh : (kind == 1 ? hh - p.H : hh - p.H - p.Hk);
   if (!check_bounds(m0 < p.BT && hh < p.H + 2 * p.Hk && nk >= 1)) return;  // checked build
@@ -125,8 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, wc)) break;
         uint8_t* st = smem + s * kStageBytes;
         mbar_expect_tx(&full[s], kXBytes + HD * kBK * 2);
-        tma_load_2d(&tmX, &full[s], st, kc * kBK, m0);
-        tma_load_2d(&tmW, &full[s], st + kXBytes, kc * kBK, hh * HD);
+        tma_load_2d(&tmX, &full[s], st, kc * kChunk, m0);
+        tma_load_2d(&tmW, &full[s], st + kXBytes, kc * kChunk, hh * HD);
         ++issued[s];
       }
       for (int s = 0; s < kStages; ++s)
@@ -135,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t id = idesc_bf16(128, HD, 0, 0);  // x W^T: both K-major
+      constexpr uint32_t id = FP8 ? idesc_e4m3(128, HD, 0, 0) : idesc_bf16(128, HD, 0, 0);  // x W^T: K-major
       const uint32_t s0 = smem_u32(smem);
       for (int kc = 0; kc < nk; ++kc) {
         const int s = kc % kStages, use = kc / kStages;
@@ -143,10 +151,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t da = sdesc_sw128(s0 + s * kStageBytes, 16, 1024);
         const uint64_t db = sdesc_sw128(s0 + s * kStageBytes + kXBytes, 16, 1024);
+        // Four K-steps of 32 bytes per 128-byte row: 16 bf16 or 32 E4M3 channels each.
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_ss(tmem, da + static_cast<uint64_t>(kk * 2), db + static_cast<uint64_t>(kk * 2), id,
-                 (kc > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          if constexpr (FP8)
+            mma_ss_f8(tmem, da + static_cast<uint64_t>(kk * 2), db + static_cast<uint64_t>(kk * 2), id,
+                      (kc > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_ss(tmem, da + static_cast<uint64_t>(kk * 2), db + static_cast<uint64_t>(kk * 2), id,
+                   (kc > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(&empty[s]);
       }
       mma_commit(acc_full);  // also the drain: every issued product completes before it fires
@@ -172,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool got = mbar_wait(acc_full, 0, wc);
     if (__all_sync(0xffffffffu, got)) {
       tc_fence_after();
+      const float sxw = FP8 ? p.scales[0] * p.scales[1] : 1.f;
       float y[HD];
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
@@ -180,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i)  // the projection as stored (bf16)
-          y[32 * c + i] = __bfloat162float(__float2bfloat16_rn(__uint_as_float(a[i])));
+          y[32 * c + i] = __bfloat162float(__float2bfloat16_rn(__uint_as_float(a[i]) * sxw));
       }
       uint8_t* raw_tile = smem;                   // raw q or k rows (HD / 64 panels)
       uint8_t* out_tile = smem + 2 * kBM * 128;   // q~, k~ or v_eff rows

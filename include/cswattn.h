@@ -145,6 +145,31 @@ cswattn_status attn_qkv_prologue(const cswattn_layer* layer, const void* x, long
                                  void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
                                  void* stream);
 
+/* Bytes of device scratch attn_qkv_prologue_fp8 needs for this layer and C:
+ * 256 bytes of amax state, then the E4M3 codes of x (B*T*C bytes, padded to
+ * 256) and of w_qkv ((n_head + 2 n_kv_head) * head_dim * C bytes, padded).
+ * 0 for an invalid layer or C < 1. */
+size_t attn_qkv_fp8_workspace_bytes(const cswattn_layer* layer, int C);
+
+/* The FP8 variant of attn_qkv_prologue: page section "3. 정밀도 관리
+ * (nanochat/common.py)", where --fp8 turns the Linear layers into
+ * Float8Linear with tensor-wise scaling. Each operand t of the projection
+ * (x[..., :C] and w_qkv) gets one scale s_t = amax|t| / 448 (1 for an
+ * all-zero tensor) and is replaced by s_t * E4M3(t / s_t) (round to nearest
+ * even, saturated to +-448, the division in float32); the product runs on
+ * the tensor cores in E4M3 with float32 accumulation and is multiplied by
+ * s_x s_w, then rounded to bf16 and handed to the same prologue epilogue.
+ * scales: 2 floats, device, written (s_x, s_w). workspace: device, 256-byte
+ * aligned, at least attn_qkv_fp8_workspace_bytes; the codes are left in it
+ * (x's at byte 256, w's after them). C a multiple of 16; otherwise as
+ * attn_qkv_prologue. Three launches: the amax reduction, the quantization,
+ * the fused projection. The backward is attn_qkv_bwd on the bf16 x and
+ * w_qkv (the quantization passes gradients straight through). */
+cswattn_status attn_qkv_prologue_fp8(const cswattn_layer* layer, const void* x, long long x_stride, int C,
+                                     const void* w_qkv, const void* ve, const void* gate, void* q, void* k,
+                                     void* q_out, void* k_out, void* v_out, float* rstd_q, float* rstd_k,
+                                     float* scales, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Backward of the projection (same page section), given attn_bwd's dQ, dK,
  * dV (gradients of the raw q, k, v):
  *   dx     = dQ w_q + dK w_k + dV w_v         (B, T, C), bf16, row stride C

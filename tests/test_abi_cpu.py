@@ -261,3 +261,26 @@ def test_qkv_entry_point_validation(lib):
     qb = lib.attn_qkv_bwd
     assert qb(ctypes.byref(f32.c()), ptrs[0], 64, 64, *ptrs[1:7], None) == cs.ERR_UNSUPPORTED
     assert qb(ctypes.byref(spec.c()), ptrs[0], 64, 60, *ptrs[1:7], None) == cs.ERR_INVALID_ARG
+
+
+def test_qkv_fp8_entry_point_validation(lib):
+    """Host checks of the FP8 projection and its workspace size: 256 bytes of
+    amax state, then the x codes (B*T*C bytes) and the weight codes
+    ((H + 2 Hk) D C bytes), each padded to 256."""
+    ptrs = [256 * (i + 1) for i in range(13)]
+    spec = cs.LayerSpec(2, 100, 6, 2, 128, 16, has_ve=False)
+    pad = lambda n: (n + 255) // 256 * 256
+    C = 96
+    assert lib.attn_qkv_fp8_workspace_bytes(ctypes.byref(spec.c()), C) == \
+        256 + pad(2 * 100 * C) + pad(10 * 128 * C)
+    assert lib.attn_qkv_fp8_workspace_bytes(ctypes.byref(spec.c()), 0) == 0
+    ws = lib.attn_qkv_fp8_workspace_bytes(ctypes.byref(spec.c()), C)
+    qp = lib.attn_qkv_prologue_fp8
+    f32 = cs.LayerSpec(2, 100, 6, 2, 64, 16, has_ve=False, dtype="f32")
+    assert qp(ctypes.byref(f32.c()), ptrs[0], C, C, *ptrs[1:12], ptrs[12], ws, None) == cs.ERR_UNSUPPORTED
+    # C a multiple of 8 but not of 16: E4M3 rows must be whole 16-byte units
+    assert qp(ctypes.byref(spec.c()), ptrs[0], 104, 104, *ptrs[1:12], ptrs[12], ws, None) == cs.ERR_INVALID_ARG
+    # workspace one byte short
+    assert qp(ctypes.byref(spec.c()), ptrs[0], C, C, *ptrs[1:12], ptrs[12], ws - 1, None) == cs.ERR_INVALID_ARG
+    # workspace not 256-byte aligned
+    assert qp(ctypes.byref(spec.c()), ptrs[0], C, C, *ptrs[1:12], 16, ws, None) == cs.ERR_INVALID_ARG
