@@ -666,18 +666,18 @@ cswattn_status check_decode_layer(const cswattn_layer* layer, Shape* s) {
   if (s->g > dec::kMaxGroup)
     return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports up to %d query heads per KV head (got %d)",
                 dec::kMaxGroup, s->g);
-  if (s->B > 65535 || s->Hk > 65535)  // grid dimensions of the split-KV kernel
-    return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports B, n_kv_head <= 65535");
+  if (s->B > 65535 || dec::decode_splits(s->T, s->W) > 65535)  // grid dimensions of the split-KV kernel
+    return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports B <= 65535 and at most 65535 key chunks");
   return CSWATTN_OK;
 }
 
 template <int D>
 cswattn_status launch_decode(const Shape& s, const CUtensorMap& mk, const CUtensorMap& mv,
                              const dec::AttnParams& ap, const dec::CombineParams& cp, cudaStream_t st) {
-  constexpr int kSmem = dec::decode_attn_smem<D>();
+  constexpr int kSmem = dec::DecSmem<D>::kBytes;
   cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem);
   if (e != CSWATTN_OK) return e;
-  launch_pdl(dec::decode_attn_kernel<D>, dim3(ap.nsplit, s.Hk, s.B), dim3(dec::kThreads), kSmem, st, mk, mv, ap);
+  launch_pdl(dec::decode_attn_kernel<D>, dim3(s.Hk, ap.nsplit, s.B), dim3(dec::kThreads), kSmem, st, mk, mv, ap);
   launch_pdl(dec::decode_combine_kernel<D>, dim3(s.B * s.H), dim3(D), 0, st, cp);
   return CSWATTN_OK;
 }
@@ -1153,8 +1153,8 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   if (workspace_bytes < w.bytes)
     return fail(CSWATTN_ERR_INVALID_ARG, "decode workspace too small: %zu < %zu bytes", workspace_bytes, w.bytes);
   CUtensorMap mk, mv;
-  if ((st = make_map(&mk, k_cache, s.B, s.T, s.Hk, dec::kChunk, s.D)) != CSWATTN_OK) return st;
-  if ((st = make_map(&mv, v_cache, s.B, s.T, s.Hk, dec::kChunk, s.D)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mk, k_cache, s.B, s.T, s.Hk, dec::kKeys, s.D)) != CSWATTN_OK) return st;
+  if ((st = make_map(&mv, v_cache, s.B, s.T, s.Hk, dec::kKeys, s.D)) != CSWATTN_OK) return st;
   dec::AttnParams ap;
   ap.B = s.B;
   ap.T = s.T;

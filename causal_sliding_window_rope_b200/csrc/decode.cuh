@@ -12,16 +12,20 @@
 //
 // The step reads the window of the K/V cache once: it is bound by HBM
 // bandwidth, not by the tensor cores (one query row per head). Two kernels:
-//   decode_attn: split-KV. CTA = (64-key chunk of the window, KV head,
-//     sequence), small enough that several CTAs per SM keep their copies in
-//     flight: TMA brings the chunk's K and V rows (128B-swizzled panels)
-//     into shared memory while the CTA computes the new token's prologue
-//     (its query rows of this KV head; the chunk holding row p also its key
-//     and value rows, which it writes to the caches and over the staged
-//     row); two threads per key score it against the g query
-//     heads of the group (half of head_dim each), the CTA reduces the chunk's
-//     max and sum per head, and each thread accumulates two columns of P V
-//     over half of the keys; the partial (max, sum, O) goes to the workspace;
+//   decode_attn: split-KV. CTA = (128-key chunk of the window, KV head,
+//     sequence), 128 threads. TMA brings the chunk's K and V rows
+//     (128B-swizzled panels, 32 KB each at head_dim 128) into shared memory
+//     while the CTA computes the new token's prologue (the group's query
+//     rows, in bf16 as the prologue stores them, into a 16-slot operand tile;
+//     the chunk holding row p also its key and value rows, which it writes
+//     to the caches and over the staged row). Both products run on the
+//     tensor cores with the 16 head slots as N: S^T = K Q^T (M = 128 keys)
+//     into TMEM; one thread per key reads its scores, masks, and the CTA
+//     reduces the chunk's max and sum per head; the probabilities go to
+//     shared memory as the bf16 operand P^T; O^T = V^T P^T (M = head_dim,
+//     V read MN-major) into TMEM; one thread per column of O writes the
+//     partial (max, sum, O) to the workspace. Three CTAs per SM keep their
+//     tile copies in flight.
 //   decode_combine: one CTA per (sequence, query head) merges the chunks'
 //     partials (rescaled by exp(m_s - M)) into O and lse.
 // A cache length outside [0, T) is reported through the status word
@@ -36,17 +40,18 @@ constexpr unsigned int kStatusRange = 8u;
 
 namespace dec {
 
-constexpr int kChunk = 64;      // keys per split
-constexpr int kThreads = 128;
+constexpr int kKeys = 128;      // keys per split (one CTA)
+constexpr int kThreads = 128;   // one thread per key, then one per column of O
 constexpr int kMaxGroup = 16;   // query heads per KV head handled by one CTA
-constexpr int kPanel = kChunk * 128;  // kChunk rows x 128 bytes
+constexpr int kSlots = 16;      // head slots: N of both tensor-core products
+constexpr int kPanel = kKeys * 128;  // kKeys rows x 128 bytes
 
-// Number of kChunk-key chunks a window of W keys (in a cache of T rows) can
+// Number of kKeys-key chunks a window of W keys (in a cache of T rows) can
 // straddle: the chunks are aligned to absolute positions.
 __host__ __device__ inline int decode_splits(int T, int W) {
   const int w = W < T ? W : T;
-  const int n = (w + kChunk - 1) / kChunk + 1;
-  const int cap = (T + kChunk - 1) / kChunk;
+  const int n = (w + kKeys - 1) / kKeys + 1;
+  const int cap = (T + kKeys - 1) / kKeys;
   return n < cap ? n : cap;
 }
 
@@ -123,32 +128,58 @@ struct NewToken {
   }
 };
 
-// Shared memory of decode_attn_kernel<D> (dynamic, with 1 KB of alignment slack).
+// Shared memory of decode_attn_kernel<D> (dynamic, 1 KB alignment slack).
+// The two products' B operands are 16-row, K-major, 128B-swizzled tiles of
+// 2 KB panels: Q (head slot x D) and P^T (head slot x 128 keys).
 template <int D>
-constexpr int decode_attn_smem() {
-  return 4 * kPanel + (kMaxGroup * D + kMaxGroup * kChunk + kMaxGroup * D + kMaxGroup * 6 + D) * 4 + 1024;
+struct DecSmem {
+  static constexpr int kTile = (D / 64) * kPanel;     // K or V: kKeys rows, D/64 swizzled panels
+  static constexpr int kSPanel = kSlots * 128;        // 2 KB: 16 rows x 128 bytes
+  static constexpr int kOffV = kTile;
+  // V always spans two panels: the second product reads 128 rows of V^T
+  // (at D = 64 the second panel is never loaded and its rows are unused).
+  static constexpr int kOffQ = kOffV + 2 * kPanel;    // bf16 q~ rows, D/64 panels
+  static constexpr int kOffP = kOffQ + (D / 64) * kSPanel;  // bf16 P^T, 2 panels (keys 0-63, 64-127)
+  static constexpr int kOffRed = kOffP + 2 * kSPanel;  // float [16][4] warp partials
+  static constexpr int kOffStat = kOffRed + kSlots * 4 * 4;  // float [16] chunk max
+  static constexpr int kOffCS = kOffStat + kSlots * 4;       // float [D/2] cos, [D/2] sin
+  static constexpr int kOffBar = kOffCS + D * 4;             // 4 mbarriers, TMEM slot, abort flag
+  static constexpr int kBytes = kOffBar + 64 + 1024;
+  static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "operand tiles need 1024-byte alignment");
+};
+
+// Byte offset of element (row, col) of a 128B-swizzled K-major tile of
+// 16-row panels (64 bf16 columns per panel).
+__device__ __forceinline__ int slot_tile_ofs(int row, int col) {
+  return (col >> 6) * (kSlots * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                const __grid_constant__ CUtensorMap tmV,
                                                                const AttnParams p) {
-  static_assert(kThreads == 2 * kChunk && kThreads == D || kThreads == 2 * D, "thread mapping");
+  using SM = DecSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align1024(smem_raw);
-  uint8_t* sK = smem;                   // 2 panels
-  uint8_t* sV = smem + 2 * kPanel;      // 2 panels
-  float* sq = reinterpret_cast<float*>(smem + 4 * kPanel);  // [g][D], scaled by c log2(e)
-  float* sp = sq + kMaxGroup * D;                            // [g][kChunk] scores -> probabilities
-  float* so = sp + kMaxGroup * kChunk;                       // [g][D] second half of P V
-  float* red = so + kMaxGroup * D;                           // [g][4] warp partials
-  float* stat = red + kMaxGroup * 4;                         // [g][2] max, sum
-  float* cs = stat + kMaxGroup * 2;                          // [D/2] cos(p omega_i)
-  float* sn = cs + D / 2;                                    // [D/2] sin(p omega_i)
-  __shared__ uint64_t bar;
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + SM::kOffV;
+  uint8_t* sQ = smem + SM::kOffQ;
+  uint8_t* sP = smem + SM::kOffP;
+  float* red = reinterpret_cast<float*>(smem + SM::kOffRed);
+  float* stat = reinterpret_cast<float*>(smem + SM::kOffStat);
+  float* cs = reinterpret_cast<float*>(smem + SM::kOffCS);
+  float* sn = cs + D / 2;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kOffBar);
+  uint64_t* bar_k = bars;      // K tile landed
+  uint64_t* bar_v = bars + 1;  // V tile landed
+  uint64_t* bar_s = bars + 2;  // S^T = K Q^T done
+  uint64_t* bar_o = bars + 3;  // O^T = V^T P^T done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 5);
 
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // KV head fastest: the CTAs reading the same cache rows run side by side.
+  const int hk = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int g = p.g;
   pdl_launch_dependents();
   pdl_wait();
@@ -156,11 +187,12 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
   const bool in_range = pos >= 0 && pos < p.T;
   if (!in_range && split == 0 && hk == 0 && tid == 0) atomicOr(&g_status, kStatusRange);
   const int lo = in_range ? max(0, pos - p.W + 1) : 0;
-  const int c0 = (lo / kChunk) * kChunk + split * kChunk;
+  const int c0 = (lo / kKeys) * kKeys + split * kKeys;
+  // A chunk with c0 <= pos holds at least one key of [lo, pos] (c0 <= lo + kKeys - 1).
   const bool work = in_range && c0 <= pos;
-  const bool owns_new = work && pos < c0 + kChunk;  // this chunk holds the new token's row
+  const bool owns_new = work && pos < c0 + kKeys;  // this chunk holds the new token's row
   auto part = [&](int h) { return (static_cast<size_t>(b) * p.H + h) * p.nsplit + split; };
-  if (!check_bounds(b < p.B && hk < p.Hk && split < p.nsplit && (hk + 1) * g <= p.H)) return;
+  if (!check_bounds(b < p.B && hk < p.Hk && split < p.nsplit && (hk + 1) * g <= p.H && g <= kSlots)) return;
   if (!work) {
     // Empty chunk: a partial that the combine step ignores.
     for (int i = tid; i < g * D; i += blockDim.x) p.part_o[part(hk * g + i / D) * D + i % D] = 0.f;
@@ -171,30 +203,46 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
     return;
   }
   if (tid == 0) {
-    mbar_init(&bar, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
     fence_barrier_init();
-    fence_proxy_async_smem();
-    mbar_expect_tx(&bar, 4 * kPanel);
-    // Rows past T read as zero; rows past pos are masked below.
-    tma_load_4d(&tmK, &bar, sK, 0, hk, c0, b);
-    tma_load_4d(&tmK, &bar, sK + kPanel, 64, hk, c0, b);
-    tma_load_4d(&tmV, &bar, sV, 0, hk, c0, b);
-    tma_load_4d(&tmV, &bar, sV + kPanel, 64, hk, c0, b);
+    // Rows past T read as zero. Rows outside [lo, pos] may hold anything:
+    // their scores are masked, and their V rows are zeroed before P V.
+    mbar_expect_tx(bar_k, SM::kTile);
+#pragma unroll
+    for (int pn = 0; pn < D / 64; ++pn) tma_load_4d(&tmK, bar_k, sK + pn * kPanel, 64 * pn, hk, c0, b);
+    mbar_expect_tx(bar_v, SM::kTile);
+#pragma unroll
+    for (int pn = 0; pn < D / 64; ++pn) tma_load_4d(&tmV, bar_v, sV + pn * kPanel, 64 * pn, hk, c0, b);
   }
-  // The new token's prologue at position pos: its g query rows of this KV
-  // head (into sq, scaled by c log2(e)), and, in the chunk that holds row
-  // pos, its key and value rows (written to the caches and, after the chunk
-  // has landed, over row pos - c0 of the staged tiles).
-  using NT = NewToken<D>;
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 32);  // columns 0-15: S^T (lane = key), 16-31: O^T (lane = column of O)
+    tmem_relinquish();
+  }
+  // The new token's prologue at position pos while the tiles land.
   for (int i = tid; i < D / 2; i += blockDim.x) {
     float sv_, cv_;
     sincosf(static_cast<float>(pos) * p.omega[i], &sv_, &cv_);
     cs[i] = cv_;
     sn[i] = sv_;
   }
+  for (int i = tid; i < (kSlots - g) * (D / 8); i += blockDim.x) {  // unused head slots: zero rows
+    const int row = g + i / (D / 8), col = (i % (D / 8)) * 8;
+    *reinterpret_cast<uint4*>(sQ + slot_tile_ofs(row, col)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.wait_ns};
+
+  // q~ rows of the group (bf16, as the prologue stores them) into the Q
+  // tile; in the chunk holding row pos, k~ and v_eff to the caches (and,
+  // once the tiles have landed, over row pos - c0 of the staged tiles).
+  using NT = NewToken<D>;
   const int sub = tid % NT::LPR, grp = tid / NT::LPR;
   constexpr int kRowsPerPass = kThreads / NT::LPR;
+  static_assert(NT::HV == 8, "one 16-byte chunk per half");
   float kl[NT::HV], kh2[NT::HV];
   bool have_k = false, have_v = false;
   for (int base = 0; base < g + 2; base += kRowsPerPass) {
@@ -205,11 +253,13 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
     NT::row(p, b, kind, kind == 0 ? hk * g + rr : hk, sub, valid, cs, sn, yl, yh);
     if (!valid) continue;
     if (kind == 0) {
-#pragma unroll
-      for (int i = 0; i < NT::HV; ++i) {
-        sq[rr * D + sub * NT::HV + i] = yl[i] * p.scale_log2;
-        sq[rr * D + NT::HALF + sub * NT::HV + i] = yh[i] * p.scale_log2;
-      }
+      uint4 u;
+      u = make_uint4(pack_bf16x2(yl[0], yl[1]), pack_bf16x2(yl[2], yl[3]), pack_bf16x2(yl[4], yl[5]),
+                     pack_bf16x2(yl[6], yl[7]));
+      *reinterpret_cast<uint4*>(sQ + slot_tile_ofs(rr, sub * 8)) = u;
+      u = make_uint4(pack_bf16x2(yh[0], yh[1]), pack_bf16x2(yh[2], yh[3]), pack_bf16x2(yh[4], yh[5]),
+                     pack_bf16x2(yh[6], yh[7]));
+      *reinterpret_cast<uint4*>(sQ + slot_tile_ofs(rr, NT::HALF + sub * 8)) = u;
     } else {
       const size_t crow = ((static_cast<size_t>(b) * p.T + pos) * p.Hk + hk) * D + sub * NT::HV;
       __nv_bfloat16* cache = kind == 1 ? p.kc : p.vc;
@@ -224,163 +274,143 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(const __grid_cons
       have_v = kind == 2;
     }
   }
-  __syncthreads();
-  {
-    bool ok = mbar_try_wait(&bar, 0);
-    const uint64_t t0 = globaltimer();
-    while (!ok) {
-      ok = mbar_try_wait(&bar, 0);
-      if (!ok && globaltimer() - t0 > p.wait_ns) {
-        atomicOr(&g_status, kStatusTimeout);
-        drain_wait(&bar, 0);  // the tile copies land before the CTA exits
-        break;
-      }
-    }
-    if (!__syncthreads_and(ok)) return;
-  }
-  if (have_k || have_v) {
-    // Row pos of the staged tile (bf16, 128B-swizzled panels) gets the new
-    // token's values: the copy brought in whatever the cache held there.
+  // Row pos of a staged tile (bf16, 128B-swizzled panels) takes the new
+  // token's values: the copy brought in whatever the cache held there.
+  auto put_row = [&](uint8_t* tile) {
     const int rr = pos - c0;
-    uint8_t* tile = have_k ? sK : sV;
     auto put = [&](int d0, const float (&x)[NT::HV]) {
-      uint4 u;
-      uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+      const uint4 u = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                 pack_bf16x2(x[6], x[7]));
       *reinterpret_cast<uint4*>(tile + (d0 >> 6) * kPanel + rr * 128 + ((((d0 & 63) >> 3) ^ (rr & 7)) << 4)) = u;
     };
-    static_assert(NT::HV == 8, "one 16-byte chunk per half");
     put(sub * NT::HV, kl);
     put(NT::HALF + sub * NT::HV, kh2);
-  }
-  __syncthreads();
+  };
 
-  // Scores (log2 units): threads 2r and 2r+1 take key r = tid / 2, each half
-  // of its columns (one 128-byte panel of D = 128, half a panel of D = 64).
-  const int r = tid >> 1, half = tid & 1;
-  const int j = c0 + r;
-  const bool key_ok = j >= lo && j <= pos;
-  {
-    constexpr int kChunks = D / 16;  // 16-byte chunks per half row
-    float acc[kMaxGroup];
+  bool issued_s = false, issued_o = false;
+  bool ok = mbar_wait(bar_k, 0, wc);
+  if (ok && have_k) put_row(sK);
+  fence_proxy_async_smem();  // Q tile and the new K row, to the tensor cores' proxy
+  ok = __syncthreads_and(ok);
+  if (ok && tid == 0) {
+    // S^T (128 keys x 16 slots) = K Q^T, K = D in steps of 16.
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16(128, kSlots, 0, 0);
+    const uint32_t k0 = smem_u32(sK), q0 = smem_u32(sQ);
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) acc[h] = 0.f;
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t da = sdesc_sw128(k0 + (kk >> 2) * kPanel, 16, 1024) + static_cast<uint64_t>((kk & 3) * 2);
+      const uint64_t db = sdesc_sw128(q0 + (kk >> 2) * SM::kSPanel, 16, 1024) + static_cast<uint64_t>((kk & 3) * 2);
+      mma_ss(tmem, da, db, id, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(bar_s);
+    issued_s = true;
+  }
+  ok = ok && mbar_wait(bar_v, 0, wc);
+  if (ok) {
+    // Thread t owns row t of the V tile: rows outside [lo, pos] become zero
+    // (probability 0 times a NaN would still be NaN in the product).
+    const int j = c0 + tid;
+    if (j < lo || j > pos) {
 #pragma unroll
-    for (int cc = 0; cc < kChunks; ++cc) {
-      const int c = half * kChunks + cc;  // 16-byte chunk of the row
-      const uint8_t* row = sK + (c >> 3) * kPanel + r * 128;
-      const uint4 u = *reinterpret_cast<const uint4*>(row + (((c & 7) ^ (r & 7)) << 4));
-      const __nv_bfloat162* kv = reinterpret_cast<const __nv_bfloat162*>(&u);
-      float kf[8];
+      for (int pn = 0; pn < D / 64; ++pn)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(kv[e]);
-        kf[2 * e] = f.x;
-        kf[2 * e + 1] = f.y;
-      }
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(sV + pn * kPanel + tid * 128 + ((c ^ (tid & 7)) << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);  // chunk order rotated per row: no bank conflicts
+    }
+    if (have_v) put_row(sV);
+  }
+  ok = ok && mbar_wait(bar_s, 0, wc);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    // Thread = key (TMEM lane): its scores in log2 units, masked by a select
+    // (rows outside (pos - W, pos] may hold anything, NaN included).
+    tc_fence_after();
+    uint32_t sr[kSlots];
+    tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16), sr);
+    tmem_ld_wait();
+    const int r = tid, j = c0 + r;
+    const bool key_ok = j >= lo && j <= pos;
+    float sc[kSlots];
 #pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= g) break;
-        const float4 qa = *reinterpret_cast<const float4*>(sq + h * D + c * 8);
-        const float4 qb = *reinterpret_cast<const float4*>(sq + h * D + c * 8 + 4);
-        acc[h] = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], acc[h]))));
-        acc[h] = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], acc[h]))));
+    for (int h = 0; h < kSlots; ++h) {
+      sc[h] = key_ok ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
+      if (h < g) {
+        float m = sc[h];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((tid & 31) == 0) red[h * 4 + warp] = m;
       }
     }
-    // Whole-row scores, then the chunk max per head.
+    __syncthreads();
+    if (tid < g) stat[tid] = fmaxf(fmaxf(red[tid * 4], red[tid * 4 + 1]), fmaxf(red[tid * 4 + 2], red[tid * 4 + 3]));
+    __syncthreads();
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      if (h >= g) break;
-      float s = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 1);
-      s = key_ok ? s : -INFINITY;
-      if (half == 0) sp[h * kChunk + r] = s;
-      float m = s;
+    for (int h = 0; h < kSlots; ++h) {
+      // Probabilities (masked keys: exp2(-inf) = 0; unused slots: 0) as the
+      // bf16 B operand P^T of the second product.
+      const float e = h < g ? exp2f(sc[h] - stat[h]) : 0.f;
+      *reinterpret_cast<__nv_bfloat16*>(sP + slot_tile_ofs(h, r)) = __float2bfloat16_rn(e);
+      if (h < g) {
+        float sum = e;
 #pragma unroll
-      for (int o = 16; o >= 2; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) red[h * 4 + warp] = m;
+        for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if ((tid & 31) == 0) red[h * 4 + warp] = sum;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid < g) {
+      p.part_ml[part(hk * g + tid) * 2] = stat[tid];
+      p.part_ml[part(hk * g + tid) * 2 + 1] = (red[tid * 4] + red[tid * 4 + 1]) + (red[tid * 4 + 2] + red[tid * 4 + 3]);
+    }
+    if (tid == 0) {
+      // O^T (D x 16 slots) = V^T P^T, K = 128 keys in steps of 16. V^T is
+      // the V tile read MN-major (64-column panels kPanel apart); at D = 64
+      // the second 64 rows of the product read other shared memory and are
+      // never loaded back.
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16(128, kSlots, 1, 0);
+      const uint32_t v0 = smem_u32(sV), p0 = smem_u32(sP);
+      const uint64_t dv = sdesc_sw128(v0, kPanel, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kKeys / 16; ++kk) {
+        const uint64_t db = sdesc_sw128(p0 + (kk >> 2) * SM::kSPanel, 16, 1024) + static_cast<uint64_t>((kk & 3) * 2);
+        mma_ss(tmem + kSlots, dv + static_cast<uint64_t>((kk * 16 * 128) >> 4), db, id, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_o);
+      issued_o = true;
+    }
+    ok = __syncthreads_and(mbar_wait(bar_o, 0, wc));
+    if (ok) {
+      // Thread = column d of O (TMEM lane): the group's partial outputs.
+      tc_fence_after();
+      uint32_t orr[kSlots];
+      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + kSlots, orr);
+      tmem_ld_wait();
+      const int d = tid;
+      if (d < D) {
+#pragma unroll
+        for (int h = 0; h < kSlots; ++h)
+          if (h < g) p.part_o[part(hk * g + h) * D + d] = __uint_as_float(orr[h]);
+      }
     }
   }
+  tc_fence_before();
   __syncthreads();
-  if (tid < g) stat[tid * 2] = fmaxf(fmaxf(red[tid * 4], red[tid * 4 + 1]), fmaxf(red[tid * 4 + 2], red[tid * 4 + 3]));
-  __syncthreads();
-  // Probabilities relative to the chunk max (thread tid < kChunk: key tid),
-  // and their sum per head.
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h) {
-    if (h >= g) break;
-    const float m = stat[h * 2];
-    float e = 0.f;
-    if (tid < kChunk) {
-      const int jj = c0 + tid;
-      e = (jj >= lo && jj <= pos) ? exp2f(sp[h * kChunk + tid] - m) : 0.f;
-      sp[h * kChunk + tid] = e;
-    }
-    float s = e;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) red[h * 4 + warp] = s;
+  if (!ok && tid == 0) {
+    // A wait ran out: the copies and products in flight land before the
+    // CTA exits and frees its TMEM.
+    drain_wait(bar_k, 0);
+    drain_wait(bar_v, 0);
+    if (issued_s) drain_wait(bar_s, 0);
+    if (issued_o) drain_wait(bar_o, 0);
   }
   __syncthreads();
-  if (tid < g) {
-    stat[tid * 2 + 1] = (red[tid * 4] + red[tid * 4 + 1]) + (red[tid * 4 + 2] + red[tid * 4 + 3]);
-    p.part_ml[part(hk * g + tid) * 2] = stat[tid * 2];
-    p.part_ml[part(hk * g + tid) * 2 + 1] = stat[tid * 2 + 1];
-  }
-  // P V: thread (column pair cp, key part kh) sums its part of the keys for
-  // columns 2cp, 2cp+1. Rows past pos are never read (they may hold anything);
-  // rows before the window start are earlier tokens' rows, weighted by 0.
-  {
-    constexpr int kPairs = D / 2;
-    constexpr int kKeyParts = kThreads / kPairs;  // 2 (D = 128) or 4 (D = 64)
-    constexpr int kKeys = kChunk / kKeyParts;
-    const int cp = tid % kPairs, kh = tid / kPairs;
-    const int d = 2 * cp, pan = d >> 6, ch = (d & 63) >> 3, el = d & 7;
-    float o0[kMaxGroup], o1[kMaxGroup];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) o0[h] = o1[h] = 0.f;
-#pragma unroll 8
-    for (int rr = 0; rr < kKeys; ++rr) {
-      const int row = kh * kKeys + rr;
-      if (c0 + row > pos) break;
-      const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
-          sV + pan * kPanel + row * 128 + ((ch ^ (row & 7)) << 4) + el * 2));
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= g) break;
-        const float pr = sp[h * kChunk + row];
-        o0[h] = fmaf(pr, v.x, o0[h]);
-        o1[h] = fmaf(pr, v.y, o1[h]);
-      }
-    }
-    // Sum the key parts through shared memory (part 0 collects).
-    for (int q = 1; q < kKeyParts; ++q) {
-      if (kh == q) {
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-          if (h >= g) break;
-          so[h * D + d] = o0[h];
-          so[h * D + d + 1] = o1[h];
-        }
-      }
-      __syncthreads();
-      if (kh == 0) {
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-          if (h >= g) break;
-          o0[h] += so[h * D + d];
-          o1[h] += so[h * D + d + 1];
-        }
-      }
-      __syncthreads();
-    }
-    if (kh == 0) {
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= g) break;
-        *reinterpret_cast<float2*>(p.part_o + part(hk * g + h) * D + d) = make_float2(o0[h], o1[h]);
-      }
-    }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
   }
 }
 

@@ -265,7 +265,7 @@ cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const
 
 /* Bytes of device scratch attn_decode needs for this layer (layer->T is the
  * cache capacity): per query head, the partial results of the split-KV
- * chunks (max, sum and head_dim partial outputs per 64-key chunk), each part
+ * chunks (max, sum and head_dim partial outputs per 128-key chunk), each part
  * padded to 256 bytes. 0 for an invalid or unsupported layer. */
 size_t attn_decode_workspace_bytes(const cswattn_layer* layer);
 

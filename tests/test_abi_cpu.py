@@ -127,9 +127,9 @@ def test_workspace_size_and_check(lib):
 def test_decode_validation(lib):
     spec = cs.LayerSpec(2, 256, 12, 4, 128, 100, has_ve=True)
     n = cs.attn_decode_workspace_bytes(spec)
-    # per 64-key chunk (max, sum) and partial O of every query head; a window
-    # of 100 keys can straddle ceil(100/64) + 1 = 3 chunks
-    rows, chunks = 2 * 12, 3
+    # per 128-key chunk (max, sum) and partial O of every query head; a window
+    # of 100 keys can straddle ceil(100/128) + 1 = 2 chunks (the cache has 2)
+    rows, chunks = 2 * 12, 2
     def pad(x):
         return (x + 255) // 256 * 256
     assert n == pad(rows * chunks * 2 * 4) + pad(rows * chunks * 128 * 4)

@@ -76,6 +76,8 @@ CASES = [
     (2, 129, 3, 3, 64, 64, True, [5, 128]),
     (1, 513, 16, 1, 128, 1, True, [400]),
     (2, 1000, 8, 2, 128, 384, True, [383, 999]),
+    (2, 700, 8, 1, 64, 300, True, [299, 650]),     # group of 8
+    (1, 400, 10, 2, 128, 400, False, [399]),       # group of 5: three unused head slots
 ]
 
 
