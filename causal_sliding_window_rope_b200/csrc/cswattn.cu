@@ -647,7 +647,7 @@ struct DecodeWorkspace {
 
 DecodeWorkspace carve_decode(const Shape& s, void* base) {
   DecodeWorkspace w;
-  w.nsplit = dec::decode_splits(s.T, s.W);
+  w.nsplit = dec::decode_nsplit(s.B, s.Hk, s.T, s.W);
   const size_t rows = static_cast<size_t>(s.B) * s.H;
   uint8_t* p = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -666,7 +666,7 @@ cswattn_status check_decode_layer(const cswattn_layer* layer, Shape* s) {
   if (s->g > dec::kMaxGroup)
     return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports up to %d query heads per KV head (got %d)",
                 dec::kMaxGroup, s->g);
-  if (s->B > 65535 || dec::decode_splits(s->T, s->W) > 65535)  // grid dimensions of the split-KV kernel
+  if (s->B > 65535 || dec::decode_nsplit(s->B, s->Hk, s->T, s->W) > 65535)  // grid of the split-KV kernel
     return fail(CSWATTN_ERR_UNSUPPORTED, "attn_decode supports B <= 65535 and at most 65535 key chunks");
   return CSWATTN_OK;
 }
@@ -677,8 +677,10 @@ cswattn_status launch_decode(const Shape& s, const CUtensorMap& mk, const CUtens
   constexpr int kSmem = dec::DecSmem<D>::kBytes;
   cswattn_status e = set_smem(dec::decode_attn_kernel<D>, kSmem);
   if (e != CSWATTN_OK) return e;
-  launch_pdl(dec::decode_attn_kernel<D>, dim3(s.Hk, ap.nsplit, s.B), dim3(dec::kThreads), kSmem, st, mk, mv, ap);
-  launch_pdl(dec::decode_combine_kernel<D>, dim3(s.B * s.H), dim3(D), 0, st, cp);
+  launch_pdl(dec::decode_attn_kernel<D>, dim3(s.Hk, ap.nsplit, s.B), dim3(dec::kDecThreads), kSmem, st, mk, mv,
+             ap);
+  // With one split per (sequence, KV head) the attention kernel writes O and lse itself.
+  if (ap.nsplit > 1) launch_pdl(dec::decode_combine_kernel<D>, dim3(s.B * s.H), dim3(D), 0, st, cp);
   return CSWATTN_OK;
 }
 
@@ -1163,6 +1165,8 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   ap.W = s.W;
   ap.g = s.g;
   ap.nsplit = w.nsplit;
+  ap.nmax = dec::decode_nmax(w.nsplit, s.T, s.W);
+  ap.tmem_cols = dec::decode_tmem_cols(ap.nmax);
   ap.scale_log2 = s.scale * 1.4426950408889634f;
   ap.has_ve = layer->has_ve;
   ap.eps = layer->eps;
@@ -1177,6 +1181,8 @@ cswattn_status attn_decode(const cswattn_layer* layer, const void* q, const void
   ap.vc = static_cast<__nv_bfloat16*>(v_cache);
   ap.part_ml = w.part_ml;
   ap.part_o = w.part_o;
+  ap.O = static_cast<__nv_bfloat16*>(O);
+  ap.lse = lse;
   ap.wait_ns = g_wait_ns.load();
   dec::CombineParams cp;
   cp.B = s.B;

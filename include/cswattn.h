@@ -264,9 +264,11 @@ cswattn_status attn_bwd_noalloc(const cswattn_layer* layer, const void* q, const
                                 void* dgate, void* stream);
 
 /* Bytes of device scratch attn_decode needs for this layer (layer->T is the
- * cache capacity): per query head, the partial results of the split-KV
- * chunks (max, sum and head_dim partial outputs per 128-key chunk), each part
- * padded to 256 bytes. 0 for an invalid or unsupported layer. */
+ * cache capacity): per query head, the partial results of the splits of the
+ * window (max, sum and head_dim partial outputs per split), each part padded
+ * to 256 bytes. A sequence's window is split only while B * n_kv_head is
+ * below 148 (one split per SM), into at most one split per 128-key chunk it
+ * can straddle. 0 for an invalid or unsupported layer. */
 size_t attn_decode_workspace_bytes(const cswattn_layer* layer);
 
 /* Decode step with a key/value cache: page section "6. 추론 엔진

@@ -127,8 +127,9 @@ def test_workspace_size_and_check(lib):
 def test_decode_validation(lib):
     spec = cs.LayerSpec(2, 256, 12, 4, 128, 100, has_ve=True)
     n = cs.attn_decode_workspace_bytes(spec)
-    # per 128-key chunk (max, sum) and partial O of every query head; a window
-    # of 100 keys can straddle ceil(100/128) + 1 = 2 chunks (the cache has 2)
+    # per split (max, sum) and partial O of every query head; 2 x 4 (sequence,
+    # KV head) pairs would take 18 splits to cover 148 SMs, but a window of
+    # 100 keys straddles at most 2 chunks of 128 (and the cache has 2)
     rows, chunks = 2 * 12, 2
     def pad(x):
         return (x + 255) // 256 * 256
