@@ -461,6 +461,17 @@ def run_ours(args):
 DECODE_BATCH = 32  # sequences generating together
 
 
+def decode_launches(B, Hk, T, W):
+    """Kernels one attn_decode call launches: the attention kernel, and the
+    combine kernel when a sequence's window is split (the library splits only
+    while B * n_kv_head is below the 148 SMs, at most once per 128-key chunk
+    the window can straddle)."""
+    chunks = min(-(-min(W, T) // 128) + 1, -(-T // 128))
+    splits = 1 if B * Hk >= 148 else min(148 // (B * Hk), chunks)
+    splits = max(splits, -(-chunks // 31))
+    return 1 + (splits > 1)
+
+
 def decode_bench(w, dev, peaks, steps=20, warmup=5, peak_src="measured"):
     """One generation step over the workload's layer stack with a KV cache
     (attn_decode per layer): DECODE_BATCH sequences whose caches hold T-1
@@ -520,7 +531,7 @@ def decode_bench(w, dev, peaks, steps=20, warmup=5, peak_src="measured"):
                         f"holding {T - 1} tokens, windows {w.windows}",
             "ms_per_step": round(ms, 4), "tokens_per_s": round(B / (ms * 1e-3), 1),
             "kernel_ms_per_step": round(kt["decode"][0] / steps, 4),
-            "launches_per_step": kt["decode"][1] // steps * 2,
+            "launches_per_step": sum(decode_launches(B, Hk, T, W) for W in w.windows),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": nbytes,
                          "peak_source": f"{peak_src} hbm_gbs"}}
