@@ -566,32 +566,51 @@ cswattn_status check_gemm(const GemmArgs& g) {
   return CSWATTN_OK;
 }
 
-template <bool AMN, bool BMN>
-void launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& gp, dim3 grid, cudaStream_t st) {
-  launch_pdl(gemm::gemm_kernel<AMN, BMN>, grid, dim3(gemm::kThreads), gemm::kSmemBytes, st, ma, mb, gp);
+// Tile width of a product: 256 columns when that still gives at least one
+// tile per SM (148), else 128 (more, smaller tiles fill the SMs better).
+int gemm_bn(int M, int N) {
+  const long long t256 = static_cast<long long>((M + gemm::kBM - 1) / gemm::kBM) * ((N + 255) / 256);
+  return t256 >= 148 ? 256 : 128;
 }
 
-// Validated product, tensor maps built before the launch; nothing is
-// enqueued when a check fails.
+template <bool AMN, bool BMN, int BN>
+cswattn_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& gp, int M, int N,
+                             cudaStream_t st, bool prepare_only) {
+  constexpr int kSmem = gemm::Geo<BN>::kSmemBytes;
+  const cswattn_status e = set_smem(gemm::gemm_kernel<AMN, BMN, BN>, kSmem);
+  if (e != CSWATTN_OK || prepare_only) return e;
+  const dim3 grid((N + BN - 1) / BN, (M + gemm::kBM - 1) / gemm::kBM);
+  launch_pdl(gemm::gemm_kernel<AMN, BMN, BN>, grid, dim3(gemm::kThreads), kSmem, st, ma, mb, gp);
+  return CSWATTN_OK;
+}
+
+template <int BN>
+cswattn_status launch_gemm_bn(int which, const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& gp,
+                              int M, int N, cudaStream_t st, bool prepare_only) {
+  switch (which) {
+    case 0: return launch_gemm_t<false, false, BN>(ma, mb, gp, M, N, st, prepare_only);
+    case 1: return launch_gemm_t<false, true, BN>(ma, mb, gp, M, N, st, prepare_only);
+    case 2: return launch_gemm_t<true, false, BN>(ma, mb, gp, M, N, st, prepare_only);
+    default: return launch_gemm_t<true, true, BN>(ma, mb, gp, M, N, st, prepare_only);
+  }
+}
+
+// Validated product, tensor maps built and shared-memory limits set before
+// the launch; nothing is enqueued when a check fails.
 cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st) {
   cswattn_status e = check_gemm(g);
   if (e != CSWATTN_OK) return e;
+  if ((g.M + gemm::kBM - 1) / gemm::kBM > 65535) return fail(CSWATTN_ERR_UNSUPPORTED, "M too large");
+  const int bn = gemm_bn(g.M, g.N);
   CUtensorMap ma, mb;
-  // K-major operand: (K, rows) with 64 x 128 boxes; MN-major: (rows, K) with 64 x 64 boxes.
+  // K-major operand: (K, rows) with 64 x rows boxes; MN-major: (rows, K) with 64 x 64 boxes.
   if ((e = g.a_mn ? make_map_2d(&ma, g.A, g.M, g.K, g.lda, 64, 64) : make_map_2d(&ma, g.A, g.K, g.M, g.lda, 64, 128)) !=
       CSWATTN_OK)
     return e;
-  if ((e = g.b_mn ? make_map_2d(&mb, g.B, g.N, g.K, g.ldb, 64, 64) : make_map_2d(&mb, g.B, g.K, g.N, g.ldb, 64, 128)) !=
+  if ((e = g.b_mn ? make_map_2d(&mb, g.B, g.N, g.K, g.ldb, 64, 64) : make_map_2d(&mb, g.B, g.K, g.N, g.ldb, 64, bn)) !=
       CSWATTN_OK)
     return e;
   const int which = (g.a_mn ? 2 : 0) + (g.b_mn ? 1 : 0);
-  switch (which) {
-    case 0: e = set_smem(gemm::gemm_kernel<false, false>, gemm::kSmemBytes); break;
-    case 1: e = set_smem(gemm::gemm_kernel<false, true>, gemm::kSmemBytes); break;
-    case 2: e = set_smem(gemm::gemm_kernel<true, false>, gemm::kSmemBytes); break;
-    default: e = set_smem(gemm::gemm_kernel<true, true>, gemm::kSmemBytes); break;
-  }
-  if (e != CSWATTN_OK) return e;
   gemm::Params gp;
   gp.M = g.M;
   gp.N = g.N;
@@ -604,17 +623,15 @@ cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st) {
   gp.C32 = g.c_f32 ? static_cast<float*>(g.C) : nullptr;
   gp.ldc = g.ldc;
   gp.wait_ns = g_wait_ns.load();
-  const dim3 grid((g.N + gemm::kBN - 1) / gemm::kBN, (g.M + gemm::kBM - 1) / gemm::kBM);
-  if (grid.y > 65535) return fail(CSWATTN_ERR_UNSUPPORTED, "M too large");
+  e = bn == 256 ? launch_gemm_bn<256>(which, ma, mb, gp, g.M, g.N, st, true)
+                : launch_gemm_bn<128>(which, ma, mb, gp, g.M, g.N, st, true);
+  if (e != CSWATTN_OK) return e;
   {
     ScopedTiming tm(CSWATTN_K_GEMM, st);
-    switch (which) {
-      case 0: launch_gemm_t<false, false>(ma, mb, gp, grid, st); break;
-      case 1: launch_gemm_t<false, true>(ma, mb, gp, grid, st); break;
-      case 2: launch_gemm_t<true, false>(ma, mb, gp, grid, st); break;
-      default: launch_gemm_t<true, true>(ma, mb, gp, grid, st); break;
-    }
+    e = bn == 256 ? launch_gemm_bn<256>(which, ma, mb, gp, g.M, g.N, st, false)
+                  : launch_gemm_bn<128>(which, ma, mb, gp, g.M, g.N, st, false);
   }
+  if (e != CSWATTN_OK) return e;
   return launched("matrix product launch");
 }
 

@@ -11,28 +11,36 @@
 // X^T X is A_MN = B_MN = true with A = B = X, and X B is A_MN = false,
 // B_MN = true. bf16 inputs and D, bf16 (or float32) C, float32 accumulation.
 //
-// One CTA per 128 x 128 tile of C. Warp 0 (one thread) loads 64-wide K
-// chunks of both operands by TMA into a 6-stage ring (128B swizzle: a
-// K-major chunk is one panel of 128 rows x 64 K, an MN-major chunk two
-// panels of 64 K-rows x 64 elements); warp 1 owns the 128-column TMEM
-// accumulator and issues 4 MMAs (M = N = 128, K = 16) per chunk; warps 2-5
-// read the accumulator (thread = row of the tile), apply alpha and beta D
-// and store the row. Out-of-range rows, columns and K entries of a partial
-// tile read as zero and are not stored.
+// One CTA per 128 x BN tile of C (BN = 128 or 256: the wider tile halves the
+// operand bytes per product, which bound the narrow one). Warp 0 (one
+// thread) loads 64-wide K chunks of both operands by TMA into a ring (128B
+// swizzle: a K-major chunk is one panel of 128 or BN rows x 64 K, an
+// MN-major chunk panels of 64 K-rows x 64 elements); warp 1 owns the
+// BN-column TMEM accumulator and issues 4 MMAs (M = 128, N = BN, K = 16)
+// per chunk; warps 2-5 read the accumulator (thread = row of the tile),
+// apply alpha and beta D and store the row. Out-of-range rows, columns and
+// K entries of a partial tile read as zero and are not stored.
 #pragma once
 #include "common.cuh"
 
 namespace cswattn {
 namespace gemm {
 
-constexpr int kBM = 128, kBN = 128, kBK = 64;
+constexpr int kBM = 128, kBK = 64;
 constexpr int kThreads = 192;
-constexpr int kStages = 6;
-constexpr int kOpBytes = kBM * kBK * 2;   // 16 KB per operand per stage
-constexpr int kStageBytes = 2 * kOpBytes;
-constexpr int kOffBar = kStages * kStageBytes;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+constexpr int kOpBytesA = kBM * kBK * 2;  // 16 KB: 128 rows x 64 K
+constexpr int kPanelMN = 64 * kBK * 2;     // 8 KB: an MN-major panel, 64 K-rows x 64 elements
+
+// Ring geometry of a BN-wide tile: 192 KB of stages either way.
+template <int BN>
+struct Geo {
+  static constexpr int kOpBytesB = BN * kBK * 2;
+  static constexpr int kStageBytes = kOpBytesA + kOpBytesB;
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kOffBar = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 
 struct Params {
   int M, N, K;
@@ -45,15 +53,15 @@ struct Params {
   unsigned long long wait_ns;
 };
 
-// TMA loads of one K chunk of an operand: rows r0.. of the tile, K from k0.
-// K-major: one 128-row x 64-K panel. MN-major: two 64-K-row panels of 64
-// M/N elements.
-template <bool MN>
+// TMA loads of one K chunk of an operand of `rows` rows (128 or BN): rows r0..
+// of the tile, K from k0. K-major: one rows x 64-K panel. MN-major: rows/64
+// panels of 64 K-rows x 64 elements.
+template <bool MN, int ROWS>
 __device__ __forceinline__ void load_operand(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int r0,
                                              int k0) {
   if constexpr (MN) {
-    tma_load_2d(map, bar, dst, r0, k0);
-    tma_load_2d(map, bar, dst + kOpBytes / 2, r0 + 64, k0);
+#pragma unroll
+    for (int pn = 0; pn < ROWS / 64; ++pn) tma_load_2d(map, bar, dst + pn * kPanelMN, r0 + 64 * pn, k0);
   } else {
     tma_load_2d(map, bar, dst, k0, r0);
   }
@@ -63,29 +71,31 @@ __device__ __forceinline__ void load_operand(const CUtensorMap* map, uint64_t* b
 // units) of its K-step kk (16 K entries).
 template <bool MN>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
-  return MN ? sdesc_sw128(saddr, kOpBytes / 2, 1024)  // 64-element chunks 8 KB apart
-            : sdesc_sw128(saddr, 16, 1024);           // 128-byte rows, 8-row groups
+  return MN ? sdesc_sw128(saddr, kPanelMN, 1024)  // 64-element chunks 8 KB apart
+            : sdesc_sw128(saddr, 16, 1024);      // 128-byte rows, 8-row groups
 }
 template <bool MN>
 __device__ __forceinline__ uint64_t kstep_ofs(int kk) {
   return static_cast<uint64_t>((MN ? kk * 16 * 128 : kk * 32) >> 4);
 }
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
+  using G = Geo<BN>;
+  constexpr int kStages = G::kStages, kStageBytes = G::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   pdl_launch_dependents();
   uint8_t* smem = smem_align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::kOffBar);
   uint64_t* full = bars;                // [kStages]
   uint64_t* empty = bars + kStages;     // [kStages]
   uint64_t* acc_full = bars + 2 * kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kStages + 2);
   const int warp = warp_id(), lane = lane_id();
-  const int n0 = static_cast<int>(blockIdx.x) * kBN, m0 = static_cast<int>(blockIdx.y) * kBM;
+  const int n0 = static_cast<int>(blockIdx.x) * BN, m0 = static_cast<int>(blockIdx.y) * kBM;
   const int nk = (p.K + kBK - 1) / kBK;
   if (!check_bounds(m0 < p.M && n0 < p.N && nk >= 1)) return;  // checked build
 
@@ -99,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -114,14 +124,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------ TMA producer
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
-      int issued[kStages] = {0, 0, 0, 0, 0, 0};
+      int issued[kStages] = {};
       for (int kc = 0; kc < nk; ++kc) {
         const int s = kc % kStages, use = kc / kStages;
         if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, wc)) break;
         uint8_t* st = smem + s * kStageBytes;
         mbar_expect_tx(&full[s], kStageBytes);
-        load_operand<A_MN>(&tmA, &full[s], st, m0, kc * kBK);
-        load_operand<B_MN>(&tmB, &full[s], st + kOpBytes, n0, kc * kBK);
+        load_operand<A_MN, kBM>(&tmA, &full[s], st, m0, kc * kBK);
+        load_operand<B_MN, BN>(&tmB, &full[s], st + kOpBytesA, n0, kc * kBK);
         ++issued[s];
       }
       for (int s = 0; s < kStages; ++s)
@@ -130,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t id = idesc_bf16(128, 128, A_MN ? 1 : 0, B_MN ? 1 : 0);
+      constexpr uint32_t id = idesc_bf16(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
       const uint32_t s0 = smem_u32(smem);
       bool ok = true;
       for (int kc = 0; ok && kc < nk; ++kc) {
@@ -141,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint64_t da = operand_desc<A_MN>(s0 + s * kStageBytes);
-        const uint64_t db = operand_desc<B_MN>(s0 + s * kStageBytes + kOpBytes);
+        const uint64_t db = operand_desc<B_MN>(s0 + s * kStageBytes + kOpBytesA);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
           mma_ss(tmem, da + kstep_ofs<A_MN>(kk), db + kstep_ofs<B_MN>(kk), id, (kc > 0 || kk > 0) ? 1u : 0u);
@@ -159,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__all_sync(0xffffffffu, got)) {
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         uint32_t a[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c * 32, a);
         tmem_ld_wait();
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, BN);
   }
 }
 

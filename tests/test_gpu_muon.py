@@ -33,8 +33,11 @@ def rel(a, b):
 
 @pytest.mark.parametrize("a_mn,b_mn", [(False, False), (False, True), (True, False), (True, True)])
 # Every contiguous extent a multiple of 8 (16-byte rows); tiles ragged
-# against the 128 x 128 output tile and the 64-wide K chunk.
-@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (296, 136, 200), (136, 8, 24), (640, 384, 1000)])
+# against the 128 x 128 output tile and the 64-wide K chunk; the last shape
+# has enough tiles (17 x 9 = 153 >= 148 SMs) for the 128 x 256 tile, ragged
+# in all three extents.
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (296, 136, 200), (136, 8, 24), (640, 384, 1000),
+                                   (2056, 2200, 200)])
 def test_gemm_layouts_and_ragged_tiles(M, N, K, a_mn, b_mn):
     A = bf16((K, M) if a_mn else (M, K), 1 + M)
     B = bf16((K, N) if b_mn else (N, K), 2 + N)
