@@ -1335,11 +1335,13 @@ cswattn_status qkv_impl(const cswattn_layer* layer, const void* x, long long x_s
   CUtensorMap mx, mw, mq, mk, mqo, mko, mvo;
   if (f8) {
     if ((st = make_map_2d(&mx, fw.x8, C, BT, C, 128, qkv::kBM, true)) != CSWATTN_OK) return st;
-    if ((st = make_map_2d(&mw, fw.w8, C, static_cast<long long>(nh) * s.D, C, 128, s.D, true)) != CSWATTN_OK)
+    if ((st = make_map_2d(&mw, fw.w8, C, static_cast<long long>(nh) * s.D, C, 128, qkv::kNH * s.D, true)) !=
+        CSWATTN_OK)
       return st;
   } else {
     if ((st = make_map_2d(&mx, x, C, BT, x_stride, 64, qkv::kBM)) != CSWATTN_OK) return st;
-    if ((st = make_map_2d(&mw, w_qkv, C, static_cast<long long>(nh) * s.D, C, 64, s.D)) != CSWATTN_OK) return st;
+    if ((st = make_map_2d(&mw, w_qkv, C, static_cast<long long>(nh) * s.D, C, 64, qkv::kNH * s.D)) != CSWATTN_OK)
+      return st;
   }
   if ((st = make_map_3d(&mq, q, BT, s.H, s.D, qkv::kBM)) != CSWATTN_OK) return st;
   if ((st = make_map_3d(&mk, k, BT, s.Hk, s.D, qkv::kBM)) != CSWATTN_OK) return st;
@@ -1364,7 +1366,8 @@ cswattn_status qkv_impl(const cswattn_layer* layer, const void* x, long long x_s
   qp.rstd_k = rstd_k;
   qp.scales = f8 ? scales : nullptr;
   qp.wait_ns = g_wait_ns.load();
-  const dim3 grid(static_cast<unsigned>(nh), static_cast<unsigned>((BT + qkv::kBM - 1) / qkv::kBM));
+  const dim3 grid(static_cast<unsigned>((nh + qkv::kNH - 1) / qkv::kNH),
+                  static_cast<unsigned>((BT + qkv::kBM - 1) / qkv::kBM));
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   {
     ScopedTiming tm(CSWATTN_K_PROLOGUE, cs);

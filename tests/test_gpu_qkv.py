@@ -46,6 +46,7 @@ def gpu_prologue(spec, x, C, w, ve, gate):
     (2, 300, 256, 6, 2, 128, 130, True),
     (1, 257, 96, 4, 4, 64, 257, True),
     (1, 200, 64, 2, 1, 128, 50, False),
+    (1, 130, 128, 3, 1, 128, 64, True),   # 5 stacked heads: a (q, k) pair and a lone value head
 ])
 def test_qkv_prologue_and_backward_match_oracle(B, T, C, H, Hk, D, W, has_ve):
     spec = cs.LayerSpec(B, T, H, Hk, D, W, has_ve=has_ve, dtype="bf16")
@@ -100,6 +101,7 @@ def e4m3_decode(codes):
     (2, 300, 256, 6, 2, 128, 130, True),
     (1, 257, 400, 4, 4, 64, 257, True),   # C = 3 x 128 + 16: a ragged last chunk
     (1, 200, 64, 2, 1, 128, 50, False),
+    (1, 130, 128, 3, 1, 64, 64, True),    # 5 stacked heads: a (q, k) pair and a lone value head
 ])
 def test_qkv_prologue_fp8_matches_oracle(B, T, C, H, Hk, D, W, has_ve):
     """Page section "3. 정밀도 관리" (Float8Linear, tensor-wise scaling): the
