@@ -579,7 +579,9 @@ cswattn_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const
   constexpr int kSmem = gemm::Geo<BN>::kSmemBytes;
   const cswattn_status e = set_smem(gemm::gemm_kernel<AMN, BMN, BN>, kSmem);
   if (e != CSWATTN_OK || prepare_only) return e;
-  const dim3 grid((N + BN - 1) / BN, (M + gemm::kBM - 1) / gemm::kBM);
+  // Persistent: at most one CTA per SM (148), each walking its share of the tiles.
+  const long long tiles = static_cast<long long>((N + BN - 1) / BN) * ((M + gemm::kBM - 1) / gemm::kBM);
+  const dim3 grid(static_cast<unsigned>(std::min<long long>(tiles, 148)));
   launch_pdl(gemm::gemm_kernel<AMN, BMN, BN>, grid, dim3(gemm::kThreads), kSmem, st, ma, mb, gp);
   return CSWATTN_OK;
 }

@@ -11,15 +11,18 @@
 // X^T X is A_MN = B_MN = true with A = B = X, and X B is A_MN = false,
 // B_MN = true. bf16 inputs and D, bf16 (or float32) C, float32 accumulation.
 //
-// One CTA per 128 x BN tile of C (BN = 128 or 256: the wider tile halves the
-// operand bytes per product, which bound the narrow one). Warp 0 (one
+// Tiles of 128 x BN of C (BN = 128 or 256: the wider tile halves the operand
+// bytes per product, which bound the narrow one), at most one CTA per SM,
+// each walking tiles blockIdx.x, blockIdx.x + gridDim.x, ... Warp 0 (one
 // thread) loads 64-wide K chunks of both operands by TMA into a ring (128B
 // swizzle: a K-major chunk is one panel of 128 or BN rows x 64 K, an
-// MN-major chunk panels of 64 K-rows x 64 elements); warp 1 owns the
-// BN-column TMEM accumulator and issues 4 MMAs (M = 128, N = BN, K = 16)
-// per chunk; warps 2-5 read the accumulator (thread = row of the tile),
-// apply alpha and beta D and store the row. Out-of-range rows, columns and
-// K entries of a partial tile read as zero and are not stored.
+// MN-major chunk panels of 64 K-rows x 64 elements), running ahead across
+// tiles; warp 1 owns two BN-column TMEM accumulators and issues 4 MMAs
+// (M = 128, N = BN, K = 16) per chunk into the one of the current tile;
+// warps 2-5 read the other accumulator back (thread = row of the tile),
+// apply alpha and beta D and store the row, so a tile's epilogue overlaps
+// the next tile's products. Out-of-range rows, columns and K entries of a
+// partial tile read as zero and are not stored.
 #pragma once
 #include "common.cuh"
 
@@ -89,27 +92,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   uint8_t* smem = smem_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::kOffBar);
-  uint64_t* full = bars;                // [kStages]
-  uint64_t* empty = bars + kStages;     // [kStages]
-  uint64_t* acc_full = bars + 2 * kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kStages + 2);
+  uint64_t* full = bars;                      // [kStages]
+  uint64_t* empty = bars + kStages;           // [kStages]
+  uint64_t* acc_full = bars + 2 * kStages;    // [2] accumulator b holds a finished tile
+  uint64_t* acc_empty = bars + 2 * kStages + 2;  // [2] accumulator b read back (4 epilogue warps)
+  uint64_t* mma_drain = bars + 2 * kStages + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kStages + 6);
   const int warp = warp_id(), lane = lane_id();
-  const int n0 = static_cast<int>(blockIdx.x) * BN, m0 = static_cast<int>(blockIdx.y) * kBM;
   const int nk = (p.K + kBK - 1) / kBK;
-  if (!check_bounds(m0 < p.M && n0 < p.N && nk >= 1)) return;  // checked build
+  const int ntn = (p.N + BN - 1) / BN;
+  const int ntiles = ((p.M + kBM - 1) / kBM) * ntn;
+  // Tiles of this CTA: blockIdx.x, + gridDim.x, ... (row-major over the
+  // tile grid, so the CTAs in flight share rows of A and columns of B).
+  const int my_tiles = static_cast<int>(blockIdx.x) < ntiles
+                           ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                           : 0;
+  if (!check_bounds(my_tiles >= 1 && nk >= 1)) return;  // checked build
+  auto tile_origin = [&](int li, int& m0, int& n0) {
+    const int t = static_cast<int>(blockIdx.x) + li * static_cast<int>(gridDim.x);
+    m0 = (t / ntn) * kBM;
+    n0 = (t % ntn) * BN;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);  // two accumulators: tile i in columns (i & 1) * BN
     tmem_relinquish();
   }
   tc_fence_before();
@@ -121,18 +141,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer (chunks of all the CTA's tiles)
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
       int issued[kStages] = {};
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % kStages, use = kc / kStages;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, wc)) break;
-        uint8_t* st = smem + s * kStageBytes;
-        mbar_expect_tx(&full[s], kStageBytes);
-        load_operand<A_MN, kBM>(&tmA, &full[s], st, m0, kc * kBK);
-        load_operand<B_MN, BN>(&tmB, &full[s], st + kOpBytesA, n0, kc * kBK);
-        ++issued[s];
+      bool ok = true;
+      for (int li = 0; ok && li < my_tiles; ++li) {
+        int m0, n0;
+        tile_origin(li, m0, n0);
+        for (int kc = 0; kc < nk; ++kc) {
+          const int g = li * nk + kc, s = g % kStages, use = g / kStages;
+          if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, wc))) break;
+          uint8_t* st = smem + s * kStageBytes;
+          mbar_expect_tx(&full[s], kStageBytes);
+          load_operand<A_MN, kBM>(&tmA, &full[s], st, m0, kc * kBK);
+          load_operand<B_MN, BN>(&tmB, &full[s], st + kOpBytesA, n0, kc * kBK);
+          ++issued[s];
+        }
       }
       for (int s = 0; s < kStages; ++s)
         if (issued[s] > 0) drain_wait(&full[s], (issued[s] - 1) & 1);
@@ -143,35 +168,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id = idesc_bf16(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
       const uint32_t s0 = smem_u32(smem);
       bool ok = true;
-      for (int kc = 0; ok && kc < nk; ++kc) {
-        const int s = kc % kStages, use = kc / kStages;
-        if (!mbar_wait(&full[s], use & 1, wc)) {
-          ok = false;
-          break;
-        }
+      for (int li = 0; ok && li < my_tiles; ++li) {
+        const int b = li & 1, u = li >> 1;
+        if (u > 0 && !(ok = mbar_wait(&acc_empty[b], (u - 1) & 1, wc))) break;
         tc_fence_after();
-        const uint64_t da = operand_desc<A_MN>(s0 + s * kStageBytes);
-        const uint64_t db = operand_desc<B_MN>(s0 + s * kStageBytes + kOpBytesA);
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * BN);
+        for (int kc = 0; kc < nk; ++kc) {
+          const int g = li * nk + kc, s = g % kStages, use = g / kStages;
+          if (!(ok = mbar_wait(&full[s], use & 1, wc))) break;
+          tc_fence_after();
+          const uint64_t da = operand_desc<A_MN>(s0 + s * kStageBytes);
+          const uint64_t db = operand_desc<B_MN>(s0 + s * kStageBytes + kOpBytesA);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_ss(tmem, da + kstep_ofs<A_MN>(kk), db + kstep_ofs<B_MN>(kk), id, (kc > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&empty[s]);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_ss(acc, da + kstep_ofs<A_MN>(kk), db + kstep_ofs<B_MN>(kk), id, (kc > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&acc_full[b]);
       }
-      mma_commit(acc_full);  // also the drain: every issued product completes before it fires
-      drain_wait(acc_full, 0);
+      mma_commit(mma_drain);  // every product issued above completes before it fires
+      drain_wait(mma_drain, 0);
     }
   } else {
     // -------------------------------------------------- epilogue (warps 2-5)
     const int quad = warp & 3;  // TMEM lanes 32 quad .. 32 quad + 31
     const int r = quad * 32 + lane;
-    const int m = m0 + r;
-    const bool got = mbar_wait(acc_full, 0, wc);
-    if (__all_sync(0xffffffffu, got)) {
+    for (int li = 0; li < my_tiles; ++li) {
+      const int b = li & 1, u = li >> 1;
+      const bool got = mbar_wait(&acc_full[b], u & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
+      int m0, n0;
+      tile_origin(li, m0, n0);
+      const int m = m0 + r;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t a[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c * 32, a);
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + b * BN + c * 32, a);
         tmem_ld_wait();
         if (m >= p.M) continue;
 #pragma unroll
@@ -182,8 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = p.alpha * __uint_as_float(a[q * 8 + e]);
           if (p.beta != 0.f) {
-            const uint4 u = *reinterpret_cast<const uint4*>(p.D + m * p.ldd + n);
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+            const uint4 uu = *reinterpret_cast<const uint4*>(p.D + m * p.ldd + n);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&uu);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(h2[e]);
@@ -205,6 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // Accumulator b is read: the MMA issuer may start tile li + 2 in it.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
 
@@ -212,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
