@@ -41,7 +41,7 @@ constexpr int kWBytes = kNH * 128 * kBK * 2;  // 32 KB: up to 2 x 128 weight row
 constexpr int kStageBytes = kXBytes + kWBytes;
 constexpr int kHeadStage = 4 * kBM * 128;     // output staging of one head: raw and final rows, 2 panels each
 static_assert(kNH * kHeadStage <= kStages * kStageBytes, "output staging fits in the ring");
-constexpr int kOffTab = kStages * kStageBytes;         // cos/sin table [128][64] x 2, float32
+constexpr int kOffTab = kStages * kStageBytes;         // cos/sin table [64][128] x 2, float32
 constexpr int kOffBar = kOffTab + 2 * kBM * 64 * 4;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* staged = bars + 2 * kStages + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kStages + 3);
-  float* tcos = reinterpret_cast<float*>(smem + kOffTab);  // [128][64]
+  float* tcos = reinterpret_cast<float*>(smem + kOffTab);  // [64 frequencies][128 rows]: a warp's rows in distinct banks
   float* tsin = tcos + kBM * 64;
   const int warp = warp_id(), lane = lane_id();
   const int nh = p.H + 2 * p.Hk;
@@ -185,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < HALF; ++i) {
         float sn, cs;
         sincosf(t * p.omega[i], &sn, &cs);
-        tcos[r * 64 + i] = cs;
-        tsin[r * 64 + i] = sn;
+        tcos[i * kBM + r] = cs;
+        tsin[i * kBM + r] = sn;
       }
     }
     const bool got = mbar_wait(acc_full, 0, wc);
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float rstd = rsqrtf(ss / static_cast<float>(HD) + p.eps);
 #pragma unroll
           for (int i = 0; i < HALF; ++i) {
-            const float cs = tcos[r * 64 + i], sn = tsin[r * 64 + i];
+            const float cs = tcos[i * kBM + r], sn = tsin[i * kBM + r];
             const float nl = y[i] * rstd, nh2 = y[i + HALF] * rstd;
             y[i] = fmaf(nl, cs, -nh2 * sn);
             y[i + HALF] = fmaf(nl, sn, nh2 * cs);
