@@ -144,7 +144,18 @@ __host__ __device__ inline size_t epilogue_stage_bytes(int tok, int H, int Hk, i
 
 template <int VEC>
 __device__ __forceinline__ void load_f32(const float* src, float (&x)[VEC]) {
-  if constexpr (VEC % 4 == 0) {
+  if constexpr (VEC == 8) {
+    // Two 16-byte chunks per lane, the lanes 32 bytes apart: a lane whose
+    // chunk pair starts in the upper 128 bytes of a 256-byte span (address
+    // bit 7) reads its second chunk first, so each load instruction of a
+    // quarter warp covers 128 distinct bytes of banks (no conflicts).
+    const int sw = static_cast<int>((reinterpret_cast<uintptr_t>(src) >> 7) & 1);
+    const float4 a = *reinterpret_cast<const float4*>(src + 4 * sw);
+    const float4 b = *reinterpret_cast<const float4*>(src + 4 - 4 * sw);
+    const float4 lo = sw ? b : a, hi = sw ? a : b;
+    x[0] = lo.x; x[1] = lo.y; x[2] = lo.z; x[3] = lo.w;
+    x[4] = hi.x; x[5] = hi.y; x[6] = hi.z; x[7] = hi.w;
+  } else if constexpr (VEC % 4 == 0) {
 #pragma unroll
     for (int i = 0; i < VEC; i += 4) {
       float4 u = *reinterpret_cast<const float4*>(src + i);
@@ -170,7 +181,7 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
   constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
 
-  __shared__ __align__(16) TokenTable<HALF> tab;
+  __shared__ __align__(16) TokenTable<HALF, HV> tab;
   __shared__ uint64_t s_bar;
   extern __shared__ __align__(128) uint8_t stage_smem[];
 
@@ -294,7 +305,7 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
 
     // RoPE^-1 on this lane's pairs (kind 2 rows skip it below).
     float cv[HV], sv[HV], nl[HV], nh[HV];
-    tab.template load<HV>(tt, sub * HV, cv, sv);
+    tab.load(tt, sub * HV, cv, sv);
 #pragma unroll
     for (int i = 0; i < HV; ++i) {
       nl[i] = fmaf(dl[i], cv[i], dh[i] * sv[i]);

@@ -139,11 +139,21 @@ __device__ __forceinline__ float row_sum(float v) {
 
 // Per-CTA token table of the row kernels: the CTA's ntt (at most
 // kPrologueTok) consecutive tokens (b, t), and cos/sin(t * omega_i) for each.
-template <int HALF>
+// A lane reads the HV pairs sub*HV .. sub*HV + HV - 1 as 16-byte chunks;
+// with HV a multiple of 4 the pairs are stored chunk-major (chunk q of every
+// lane, then chunk q + 1), so the lanes of a quarter warp read one
+// contiguous 128-byte span (no bank conflicts).
+template <int HALF, int HV>
 struct TokenTable {
+  static constexpr bool kChunked = HV % 4 == 0;
   float cos_[kPrologueTok][HALF];
   float sin_[kPrologueTok][HALF];
   int b[kPrologueTok], t[kPrologueTok];
+
+  __device__ static int pos(int i) {
+    if constexpr (kChunked) return (((i % HV) >> 2) * (HALF / HV) + i / HV) * 4 + (i & 3);
+    else return i;
+  }
 
   // Tokens tok0 .. tok0 + ntt - 1, all of them below B*T.
   __device__ void fill(long long tok0, int T, const float* omega, int ntt) {
@@ -157,24 +167,24 @@ struct TokenTable {
       const int t_ = static_cast<int>((tok0 + tt) % T);
       float sn, cs;
       sincosf(static_cast<float>(t_) * omega[i], &sn, &cs);
-      cos_[tt][i] = cs;
-      sin_[tt][i] = sn;
+      cos_[tt][pos(i)] = cs;
+      sin_[tt][pos(i)] = sn;
     }
   }
-  // cos and sin of the VEC consecutive pairs starting at pair0 (16-byte loads).
-  template <int VEC>
-  __device__ void load(int tt, int pair0, float (&c)[VEC], float (&s)[VEC]) const {
-    if constexpr (VEC % 4 == 0) {
+  // cos and sin of the HV consecutive pairs starting at pair0 = sub * HV.
+  __device__ void load(int tt, int pair0, float (&c)[HV], float (&s)[HV]) const {
+    if constexpr (kChunked) {
 #pragma unroll
-      for (int i = 0; i < VEC; i += 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(&cos_[tt][pair0 + i]);
-        const float4 s4 = *reinterpret_cast<const float4*>(&sin_[tt][pair0 + i]);
-        c[i] = c4.x; c[i + 1] = c4.y; c[i + 2] = c4.z; c[i + 3] = c4.w;
-        s[i] = s4.x; s[i + 1] = s4.y; s[i + 2] = s4.z; s[i + 3] = s4.w;
+      for (int q = 0; q < HV / 4; ++q) {
+        const int at = (q * (HALF / HV) + pair0 / HV) * 4;
+        const float4 c4 = *reinterpret_cast<const float4*>(&cos_[tt][at]);
+        const float4 s4 = *reinterpret_cast<const float4*>(&sin_[tt][at]);
+        c[4 * q] = c4.x; c[4 * q + 1] = c4.y; c[4 * q + 2] = c4.z; c[4 * q + 3] = c4.w;
+        s[4 * q] = s4.x; s[4 * q + 1] = s4.y; s[4 * q + 2] = s4.z; s[4 * q + 3] = s4.w;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) {
+      for (int i = 0; i < HV; ++i) {
         c[i] = cos_[tt][pair0 + i];
         s[i] = sin_[tt][pair0 + i];
       }
@@ -242,7 +252,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   constexpr int HV = RL::HV, LPR = RL::LPR, HALF = RL::HALF;
   constexpr int ROWS_PER_PASS = kPrologueThreads / LPR;
 
-  __shared__ __align__(16) TokenTable<HALF> tab;
+  __shared__ __align__(16) TokenTable<HALF, HV> tab;
   __shared__ uint64_t s_bar;
   extern __shared__ __align__(128) uint8_t stage_smem[];
 
@@ -379,7 +389,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
     }
     // RoPE on the pairs (i, i + D/2) held by this lane.
     float cv[HV], sv[HV], yl[HV], yh[HV];
-    tab.template load<HV>(tt, sub * HV, cv, sv);
+    tab.load(tt, sub * HV, cv, sv);
 #pragma unroll
     for (int i = 0; i < HV; ++i) {
       const float nl = xl[i] * rstd, nh = xh[i] * rstd;
