@@ -368,6 +368,16 @@ def run_ours(args):
             dist.barrier()
             dist.destroy_process_group()
         return
+    if args.qkv_only:
+        # Profiling case: only the QKV-projection measurement at the workload's layer shape.
+        if rank == 0:
+            peaks, peak_src = load_peaks()
+            print(json.dumps({"qkv_projection": qkv_bench(cs.WORKLOADS[args.config], dev, peaks, peak_src,
+                                                          steps=args.steps, warmup=args.warmup)}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     w = cs.WORKLOADS[args.config]
     if args.single_layer is not None:
@@ -646,10 +656,33 @@ def qkv_bench(w, dev, peaks, peak_src, steps=20, warmup=5):
         cs.attn_qkv_prologue_fp8(spec, x, C, wq, ve, gate, q, k, buf.q_out, buf.k_out, buf.v_out,
                                  buf.rstd_q, buf.rstd_k, scales, ws8)
 
+    # The value-embedding gate's projection (gate logits from the first
+    # GATE_CHANNELS channels of x; the page does not give the channel count,
+    # a parameter of the call), against the prologue given the logits.
+    GATE_CHANNELS = 32
+    w_gate = (torch.randn(Hk, GATE_CHANNELS, generator=g) / GATE_CHANNELS ** 0.5).to(bf).to(dev)
+    gate_out = torch.empty(B, T, Hk, dtype=bf, device=dev)
+    dgx = torch.empty(B, T, GATE_CHANNELS, dtype=bf, device=dev)
+    dwg = torch.empty(Hk, GATE_CHANNELS, dtype=torch.float32, device=dev)
+
+    v_in = torch.randn(B, T, Hk, D, generator=g).to(bf).to(dev)
+
+    def prologue_plain():
+        cs.attn_prologue(spec, q, k, v_in, ve, gate, buf.q_out, buf.k_out, buf.v_out, buf.rstd_q, buf.rstd_k)
+
+    def prologue_gated():
+        cs.attn_prologue_gated(spec, q, k, v_in, ve, x, GATE_CHANNELS, w_gate, gate_out, buf.q_out,
+                               buf.k_out, buf.v_out, buf.rstd_q, buf.rstd_k)
+
+    def gate_bwd():
+        cs.attn_gate_bwd(spec, x, GATE_CHANNELS, w_gate, gate, dgx, dwg)
+
     out = {}
     flops = 2.0 * B * T * C * (H + 2 * Hk) * D
     stream = torch.cuda.current_stream(dev)
-    for name, fn, fl in (("fwd", fwd, flops), ("bwd", bwd, 2 * flops), ("fwd_fp8", fwd_fp8, flops)):
+    for name, fn, fl in (("fwd", fwd, flops), ("bwd", bwd, 2 * flops), ("fwd_fp8", fwd_fp8, flops),
+                         ("prologue", prologue_plain, 0.0), ("prologue_gated", prologue_gated, 0.0),
+                         ("gate_bwd", gate_bwd, 0.0)):
         for _ in range(max(warmup, 3)):
             fn()
         torch.cuda.synchronize(dev)
@@ -660,7 +693,9 @@ def qkv_bench(w, dev, peaks, peak_src, steps=20, warmup=5):
         b.record(stream)
         torch.cuda.synchronize(dev)
         ms = a.elapsed_time(b) / steps
-        out[name] = {"ms_per_call": round(ms, 4), "tflops": round(fl / (ms * 1e-3) / 1e12, 1)}
+        out[name] = {"ms_per_call": round(ms, 4)}
+        if fl > 0:
+            out[name]["tflops"] = round(fl / (ms * 1e-3) / 1e12, 1)
     cs.cswattn_sync_status()
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     # E4M3 call: amax, quantization and the fused product; against the FP8
@@ -668,7 +703,9 @@ def qkv_bench(w, dev, peaks, peak_src, steps=20, warmup=5):
     out["fwd_fp8"]["frac_of_fp8_peak"] = round(out["fwd_fp8"]["tflops"] / (2 * peak), 4)
     return {"workload": f"QKV projection of the layer input (B={B} T={T} C={C} -> {H}+2x{Hk} heads of {D}) "
                         f"fused with the prologue (fwd; fwd_fp8 with E4M3 operands and tensor-wise "
-                        f"scales, quantization included), and its backward dx, dW (bwd)",
+                        f"scales, quantization included), and its backward dx, dW (bwd); the prologue "
+                        f"given the gate logits, with them projected from x[..., :{GATE_CHANNELS}] "
+                        f"(prologue_gated), and that projection's backward (gate_bwd); inputs L2-warm",
             **out, "roofline": {"kernel": "qkv fused product", "bound": "tensor",
                                 "achieved": out["fwd"]["tflops"], "peak": peak, "unit": "TFLOP/s",
                                 "frac": round(out["fwd"]["tflops"] / peak, 4),
@@ -803,6 +840,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-muon", action="store_true",
                     help="skip the Newton-Schulz and QKV-projection measurements")
+    ap.add_argument("--qkv-only", action="store_true",
+                    help="profiling case: only the QKV-projection measurement")
     ap.add_argument("--muon-only", action="store_true",
                     help="profiling case: only the Newton-Schulz measurement")
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurement")

@@ -885,22 +885,35 @@ cswattn_status attn_gate_bwd(const cswattn_layer* layer, const void* x, long lon
   gp.x_stride = x_stride;
   gp.Hk = s.Hk;
   gp.C = gate_channels;
-  gp.dw_blocks = s.Hk * ((gate_channels + 31) / 32);
+  gp.dw_blocks = s.Hk * ((gate_channels + 31) / 32) * kGateCluster;
   gp.x = x;
   gp.w = w_gate;
   gp.dgate = dgate;
   gp.dx = dx;
   gp.dw = dw_gate;
-  const long long dx_blocks = (gp.ntok * gate_channels + kGateDwThreads - 1) / kGateDwThreads;
+  // dx blocks rounded up to whole clusters (the extra blocks have no entries).
+  long long dx_blocks = (gp.ntok * gate_channels + kGateDwThreads - 1) / kGateDwThreads;
+  dx_blocks = (dx_blocks + kGateCluster - 1) / kGateCluster * kGateCluster;
   if (gp.dw_blocks + dx_blocks > 0x7fffffffll) return fail(CSWATTN_ERR_UNSUPPORTED, "gate backward too large");
-  const dim3 grid(static_cast<unsigned>(gp.dw_blocks + dx_blocks));
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(gp.dw_blocks + dx_blocks));
+  cfg.blockDim = dim3(kGateDwThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kGateCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   {
-    ScopedTiming tm(CSWATTN_K_GATE_BWD, cs);
-    if (s.bf16)
-      launch_pdl(gate_bwd_kernel<__nv_bfloat16>, grid, dim3(kGateDwThreads), 0, cs, gp);
-    else
-      launch_pdl(gate_bwd_kernel<float>, grid, dim3(kGateDwThreads), 0, cs, gp);
+    ScopedTiming tm(CSWATTN_K_GATE_BWD, cfg.stream);
+    const cudaError_t e = s.bf16 ? cudaLaunchKernelEx(&cfg, gate_bwd_kernel<__nv_bfloat16>, gp)
+                                 : cudaLaunchKernelEx(&cfg, gate_bwd_kernel<float>, gp);
+    if (e != cudaSuccess) return cuda_fail(e, "gate backward launch");
   }
   return launched("gate backward launch");
 }

@@ -7,22 +7,27 @@
 // Given dgate = dL/dgate (the attention backward's dgate output):
 //   dx[b,t,c] = sum_h dgate[b,t,h] w[h,c]          (B, T, C)
 //   dw[h,c]   = sum_{b,t} dgate[b,t,h] x[b,t,c]    (Hk, C), float32
-// One launch does both. The dw blocks each own 32 channels of one head and
-// sum over all tokens in a fixed order (32 token lanes, then a tree over the
-// lanes), so dw is deterministic; the dx blocks take 1024 (token, channel)
-// entries each.
+// One launch does both. A cluster of kGateCluster dw blocks owns 32
+// channels of one head: block r of the cluster sums tokens r*32 + lane + 256 i
+// over its 32 token lanes (a tree over the lanes), and the cluster's block 0
+// adds the blocks' partials from their shared memory in rank order, so dw is
+// deterministic and needs no scratch memory; the dx blocks take 1024
+// (token, channel) entries each.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "prologue.cuh"
 
 namespace cswattn {
 
 constexpr int kGateDwThreads = 1024;  // 32 channels x 32 token lanes (dx: 1024 entries)
+constexpr int kGateCluster = 8;       // dw blocks per (head, 32 channels), one cluster
 
 struct GateBwdParams {
   long long ntok;      // B * T
   long long x_stride;  // elements between consecutive tokens of x
   int Hk, C;
-  int dw_blocks;       // Hk * ceil(C / 32)
+  int dw_blocks;       // Hk * ceil(C / 32) * kGateCluster
   const void* x;       // (B, T, x_stride), layer dtype
   const void* w;       // (Hk, C), layer dtype
   const void* dgate;   // (B, T, Hk), layer dtype
@@ -37,9 +42,14 @@ __global__ void __launch_bounds__(kGateDwThreads) gate_bwd_kernel(const GateBwdP
   pdl_wait();
   const int blk = static_cast<int>(blockIdx.x);
   if (blk < p.dw_blocks) {
-    // ---- dw[h, c0 + lane]: token lane `tl` sums tokens tl, tl + 32, ...
+    // ---- dw[h, c0 + lane]: token lane `tl` of cluster block `rank` sums
+    // tokens rank*32 + tl, + 32*kGateCluster, ...
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
     const int cblocks = (p.C + 31) / 32;
-    const int h = blk / cblocks, c0 = (blk % cblocks) * 32;
+    const int grp = blk / kGateCluster;
+    const int h = grp / cblocks, c0 = (grp % cblocks) * 32;
     const int lane = threadIdx.x & 31, tl = threadIdx.x >> 5;
     const int c = c0 + lane;
     float acc = 0.f;
@@ -47,7 +57,7 @@ __global__ void __launch_bounds__(kGateDwThreads) gate_bwd_kernel(const GateBwdP
       const T* x = static_cast<const T*>(p.x);
       const T* dg = static_cast<const T*>(p.dgate);
 #pragma unroll 4
-      for (long long n = tl; n < p.ntok; n += 32)
+      for (long long n = rank * 32 + tl; n < p.ntok; n += 32 * kGateCluster)
         acc = fmaf(Vec16<T>::scalar(dg, n * p.Hk + h), Vec16<T>::scalar(x, n * p.x_stride + c), acc);
     }
     red[tl][lane] = acc;
@@ -56,7 +66,13 @@ __global__ void __launch_bounds__(kGateDwThreads) gate_bwd_kernel(const GateBwdP
       if (tl < s) red[tl][lane] += red[tl + s][lane];
       __syncthreads();
     }
-    if (tl == 0 && c < p.C) p.dw[static_cast<size_t>(h) * p.C + c] = red[0][lane];
+    cluster.sync();  // every block's partial in its red[0]
+    if (rank == 0 && tl == 0 && c < p.C) {
+      float sum = 0.f;
+      for (int r = 0; r < kGateCluster; ++r) sum += cluster.map_shared_rank(&red[0][0], r)[lane];
+      p.dw[static_cast<size_t>(h) * p.C + c] = sum;
+    }
+    cluster.sync();  // the partials stay until block 0 has read them
   } else {
     // ---- dx: one (token, channel) entry per thread
     const long long e = static_cast<long long>(blk - p.dw_blocks) * kGateDwThreads + threadIdx.x;

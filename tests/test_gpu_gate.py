@@ -66,3 +66,29 @@ def test_gated_prologue_and_gate_backward_f32():
     got, ref = run_case(2, 40, 4, 2, 16, 9, 24, 10, "f32", seed=66)
     for k in ref:
         assert max_abs(got[k], ref[k]) <= 1e-4, (k, max_abs(got[k], ref[k]))
+
+
+def test_gate_backward_is_deterministic_and_matches_at_d24_shape():
+    """dw_gate is summed in a fixed order (token lanes, then the cluster's
+    blocks in rank order): two calls give the same bits. At the d24 layer
+    shape (B*T = 8192 tokens, 4 KV heads, 32 and 40 gate channels: a
+    partial channel group), dx and dw against the oracle."""
+    B, T, Hk = 4, 2048, 4
+    g = torch.Generator().manual_seed(71)
+    for C in (32, 40):
+        spec = cs.LayerSpec(B, T, 12, Hk, 128, 1024, has_ve=True, dtype="bf16")
+        x = torch.randn(B, T, 1536, generator=g).to(torch.bfloat16)
+        w = (torch.randn(Hk, C, generator=g) / C ** 0.5).to(torch.bfloat16)
+        dgate = (0.1 * torch.randn(B, T, Hk, generator=g)).to(torch.bfloat16)
+        xd, wd, dgd = x.cuda(), w.cuda(), dgate.cuda()
+        runs = []
+        for _ in range(2):
+            dx = torch.empty(B, T, C, dtype=torch.bfloat16, device="cuda")
+            dw = torch.empty(Hk, C, dtype=torch.float32, device="cuda")
+            cs.attn_gate_bwd(spec, xd, C, wd, dgd, dx, dw)
+            runs.append((dx, dw))
+        cs.cswattn_sync_status()
+        assert torch.equal(runs[0][1], runs[1][1]) and torch.equal(runs[0][0], runs[1][0])
+        rdx, rdw = oracle.gate_bwd(f64(x), f64(w), C, f64(dgate))
+        assert rel_frob(f64(runs[0][0]), rdx) <= 2e-2
+        assert rel_frob(f64(runs[0][1]), rdw) <= 2e-2

@@ -161,3 +161,28 @@ def test_qkv_prologue_fp8_zero_input():
     assert torch.count_nonzero(q).item() == 0 and torch.count_nonzero(k).item() == 0
     coef = 3.0 / (1.0 + np.exp(-f64(gate)))
     assert rel_frob(f64(buf.v_out), coef[..., None] * f64(ve)) <= TOL
+
+
+def test_qkv_prologue_fp8_full_size_d24():
+    """The d24 layer's projection with E4M3 operands (C = 1536, 12 query and
+    4 KV heads, B*T = 8192 tokens): both scales bit-exact, the raw
+    projections and the prologue outputs against the oracle."""
+    B, T, C, H, Hk, D = 4, 2048, 1536, 12, 4, 128
+    spec = cs.LayerSpec(B, T, H, Hk, D, 1024, has_ve=True, dtype="bf16")
+    x, w, ve, gate, _ = draw(B, T, C, H, Hk, D, True, seed=49)
+    buf = cs.LayerBuffers(spec)
+    q = torch.empty(B, T, H, D, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(B, T, Hk, D, dtype=torch.bfloat16, device="cuda")
+    scales = torch.zeros(2, dtype=torch.float32, device="cuda")
+    ws = torch.empty(cs.attn_qkv_fp8_workspace_bytes(spec, C), dtype=torch.uint8, device="cuda")
+    cs.attn_qkv_prologue_fp8(spec, x.cuda(), C, w.cuda(), ve.cuda(), gate.cuda(), q, k, buf.q_out, buf.k_out,
+                             buf.v_out, buf.rstd_q, buf.rstd_k, scales, ws)
+    cs.cswattn_sync_status()
+    rq, rk, rv, (sx, sw) = oracle.qkv_projection_fp8(f64(x), f64(w), H, Hk, D)
+    got = scales.cpu().numpy()
+    assert got[0] == np.float32(sx) and got[1] == np.float32(sw)
+    L = oracle.Layer(B, T, H, Hk, D, 1024, True)
+    qt, kt, veff, rsq, rsk = oracle.prologue(L, rq, rk, rv, f64(ve), f64(gate))
+    for name, a, r in (("q", q, rq), ("k", k, rk), ("q_out", buf.q_out, qt), ("k_out", buf.k_out, kt),
+                       ("v_out", buf.v_out, veff), ("rstd_k", buf.rstd_k, rsk)):
+        assert rel_frob(f64(a), r) <= TOL, name
