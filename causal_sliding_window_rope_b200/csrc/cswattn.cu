@@ -547,18 +547,22 @@ struct GemmArgs {
   bool c_f32 = false;  // C is float32 (else bf16)
 };
 
-cswattn_status check_gemm(const GemmArgs& g) {
+// With `operands` false (a segmented product) A, B, lda and ldb are the
+// segments' and are checked per segment by run_gemm.
+cswattn_status check_gemm(const GemmArgs& g, bool operands = true) {
   if (g.M < 1 || g.N < 1 || g.K < 1) return fail(CSWATTN_ERR_INVALID_ARG, "M, N, K must be >= 1");
   if (g.M > (1 << 30) || g.N > (1 << 30) || g.K > (1 << 30)) return fail(CSWATTN_ERR_UNSUPPORTED, "matrix too large");
   if (g.N % 8 != 0) return fail(CSWATTN_ERR_UNSUPPORTED, "N must be a multiple of 8 (got %d)", g.N);
   const long long a_inner = g.a_mn ? g.M : g.K, b_inner = g.b_mn ? g.N : g.K;
-  if (g.lda < a_inner || g.ldb < b_inner || g.ldc < g.N || (g.beta != 0.f && g.ldd < g.N))
+  if ((operands && (g.lda < a_inner || g.ldb < b_inner)) || g.ldc < g.N || (g.beta != 0.f && g.ldd < g.N))
     return fail(CSWATTN_ERR_INVALID_ARG, "a leading dimension is smaller than its row");
-  if (g.lda % 8 || g.ldb % 8 || g.ldc % 8 || (g.beta != 0.f && g.ldd % 8))
+  if ((operands && (g.lda % 8 || g.ldb % 8)) || g.ldc % 8 || (g.beta != 0.f && g.ldd % 8))
     return fail(CSWATTN_ERR_INVALID_ARG, "leading dimensions must be multiples of 8 elements");
   if (g.c_f32 && g.beta != 0.f) return fail(CSWATTN_ERR_UNSUPPORTED, "a float32 C takes no beta D term");
-  CHECK_PTR(g.A, 16);
-  CHECK_PTR(g.B, 16);
+  if (operands) {
+    CHECK_PTR(g.A, 16);
+    CHECK_PTR(g.B, 16);
+  }
   CHECK_PTR(g.C, 16);
   if (g.beta != 0.f) CHECK_PTR(g.D, 16);
   if (g.C == g.A || g.C == g.B) return fail(CSWATTN_ERR_INVALID_ARG, "C must not alias A or B");
@@ -574,46 +578,102 @@ int gemm_bn(int M, int N) {
 }
 
 template <bool AMN, bool BMN, int BN>
-cswattn_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& gp, int M, int N,
-                             cudaStream_t st, bool prepare_only) {
+cswattn_status launch_gemm_t(const gemm::Maps& maps, const gemm::Params& gp, int M, int N, cudaStream_t st,
+                             bool prepare_only) {
   constexpr int kSmem = gemm::Geo<BN>::kSmemBytes;
   const cswattn_status e = set_smem(gemm::gemm_kernel<AMN, BMN, BN>, kSmem);
   if (e != CSWATTN_OK || prepare_only) return e;
   // Persistent: at most one CTA per SM (148), each walking its share of the tiles.
   const long long tiles = static_cast<long long>((N + BN - 1) / BN) * ((M + gemm::kBM - 1) / gemm::kBM);
   const dim3 grid(static_cast<unsigned>(std::min<long long>(tiles, 148)));
-  launch_pdl(gemm::gemm_kernel<AMN, BMN, BN>, grid, dim3(gemm::kThreads), kSmem, st, ma, mb, gp);
+  launch_pdl(gemm::gemm_kernel<AMN, BMN, BN>, grid, dim3(gemm::kThreads), kSmem, st, maps, gp);
   return CSWATTN_OK;
 }
 
 template <int BN>
-cswattn_status launch_gemm_bn(int which, const CUtensorMap& ma, const CUtensorMap& mb, const gemm::Params& gp,
-                              int M, int N, cudaStream_t st, bool prepare_only) {
+cswattn_status launch_gemm_bn(int which, const gemm::Maps& maps, const gemm::Params& gp, int M, int N,
+                              cudaStream_t st, bool prepare_only) {
   switch (which) {
-    case 0: return launch_gemm_t<false, false, BN>(ma, mb, gp, M, N, st, prepare_only);
-    case 1: return launch_gemm_t<false, true, BN>(ma, mb, gp, M, N, st, prepare_only);
-    case 2: return launch_gemm_t<true, false, BN>(ma, mb, gp, M, N, st, prepare_only);
-    default: return launch_gemm_t<true, true, BN>(ma, mb, gp, M, N, st, prepare_only);
+    case 0: return launch_gemm_t<false, false, BN>(maps, gp, M, N, st, prepare_only);
+    case 1: return launch_gemm_t<false, true, BN>(maps, gp, M, N, st, prepare_only);
+    case 2: return launch_gemm_t<true, false, BN>(maps, gp, M, N, st, prepare_only);
+    default: return launch_gemm_t<true, true, BN>(maps, gp, M, N, st, prepare_only);
   }
 }
 
+// Operand segments of one product (see gemm::Maps): segment s has operands
+// A[s], B[s] (along M: B[0] alone) with leading dimensions lda[s], ldb[s],
+// and extent ext[s]: its K (along K) or its rows of M (along M).
+struct GemmSegs {
+  int n = 0;  // 0: the product of the GemmArgs alone
+  bool along_m = false;
+  const void* A[gemm::kMaxSeg] = {};
+  const void* B[gemm::kMaxSeg] = {};
+  long long lda[gemm::kMaxSeg] = {}, ldb[gemm::kMaxSeg] = {};
+  int ext[gemm::kMaxSeg] = {};
+};
+
 // Validated product, tensor maps built and shared-memory limits set before
-// the launch; nothing is enqueued when a check fails.
-cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st) {
-  cswattn_status e = check_gemm(g);
+// the launch; nothing is enqueued when a check fails. With segments, g holds
+// the whole product's M, N, K, layouts and output (its A, B, lda, ldb are
+// not used).
+cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st, const GemmSegs* sg = nullptr) {
+  cswattn_status e = check_gemm(g, sg == nullptr);
   if (e != CSWATTN_OK) return e;
   if ((g.M + gemm::kBM - 1) / gemm::kBM > 65535) return fail(CSWATTN_ERR_UNSUPPORTED, "M too large");
+  GemmSegs one;
+  if (!sg) {
+    one.n = 1;
+    one.A[0] = g.A;
+    one.B[0] = g.B;
+    one.lda[0] = g.lda;
+    one.ldb[0] = g.ldb;
+    one.ext[0] = g.K;
+    sg = &one;
+  }
+  if (sg->n < 1 || sg->n > gemm::kMaxSeg) return fail(CSWATTN_ERR_INVALID_ARG, "1 to 3 operand segments");
   const int bn = gemm_bn(g.M, g.N);
-  CUtensorMap ma, mb;
-  // K-major operand: (K, rows) with 64 x rows boxes; MN-major: (rows, K) with 64 x 64 boxes.
-  if ((e = g.a_mn ? make_map_2d(&ma, g.A, g.M, g.K, g.lda, 64, 64) : make_map_2d(&ma, g.A, g.K, g.M, g.lda, 64, 128)) !=
-      CSWATTN_OK)
-    return e;
-  if ((e = g.b_mn ? make_map_2d(&mb, g.B, g.N, g.K, g.ldb, 64, 64) : make_map_2d(&mb, g.B, g.K, g.N, g.ldb, 64, bn)) !=
-      CSWATTN_OK)
-    return e;
-  const int which = (g.a_mn ? 2 : 0) + (g.b_mn ? 1 : 0);
+  gemm::Maps maps;
   gemm::Params gp;
+  gp.nseg = sg->n;
+  gp.along_m = sg->along_m ? 1 : 0;
+  int sum = 0;
+  for (int s = 0; s < sg->n; ++s) {
+    const int ext = sg->ext[s];
+    const int Ms = sg->along_m ? ext : g.M, Ks = sg->along_m ? g.K : ext;
+    if (ext < 1) return fail(CSWATTN_ERR_INVALID_ARG, "an operand segment is empty");
+    if (sg->along_m && s + 1 < sg->n && ext % gemm::kBM != 0)
+      return fail(CSWATTN_ERR_UNSUPPORTED, "along M, every segment but the last spans whole 128-row tiles");
+    CHECK_PTR(sg->A[s], 16);
+    const long long a_inner = g.a_mn ? Ms : Ks;
+    if (sg->lda[s] < a_inner || sg->lda[s] % 8) return fail(CSWATTN_ERR_INVALID_ARG, "segment lda");
+    if ((e = g.a_mn ? make_map_2d(&maps.a[s], sg->A[s], Ms, Ks, sg->lda[s], 64, 64)
+                    : make_map_2d(&maps.a[s], sg->A[s], Ks, Ms, sg->lda[s], 64, 128)) != CSWATTN_OK)
+      return e;
+    if (!sg->along_m || s == 0) {
+      CHECK_PTR(sg->B[s], 16);
+      const long long b_inner = g.b_mn ? g.N : Ks;
+      if (sg->ldb[s] < b_inner || sg->ldb[s] % 8) return fail(CSWATTN_ERR_INVALID_ARG, "segment ldb");
+      if ((e = g.b_mn ? make_map_2d(&maps.b[s], sg->B[s], g.N, Ks, sg->ldb[s], 64, 64)
+                      : make_map_2d(&maps.b[s], sg->B[s], Ks, g.N, sg->ldb[s], 64, bn)) != CSWATTN_OK)
+        return e;
+    } else {
+      maps.b[s] = maps.b[0];
+    }
+    gp.kseg[s] = Ks;
+    gp.mstart[s] = sum;
+    sum += ext;
+  }
+  for (int s = sg->n; s < gemm::kMaxSeg; ++s) {
+    maps.a[s] = maps.a[0];
+    maps.b[s] = maps.b[0];
+    gp.kseg[s] = 0;
+    gp.mstart[s] = sum;
+  }
+  gp.mstart[gemm::kMaxSeg] = sum;
+  if (sum != (sg->along_m ? g.M : g.K))
+    return fail(CSWATTN_ERR_INVALID_ARG, "the segments do not add up to %s", sg->along_m ? "M" : "K");
+  const int which = (g.a_mn ? 2 : 0) + (g.b_mn ? 1 : 0);
   gp.M = g.M;
   gp.N = g.N;
   gp.K = g.K;
@@ -625,13 +685,13 @@ cswattn_status run_gemm(const GemmArgs& g, cudaStream_t st) {
   gp.C32 = g.c_f32 ? static_cast<float*>(g.C) : nullptr;
   gp.ldc = g.ldc;
   gp.wait_ns = g_wait_ns.load();
-  e = bn == 256 ? launch_gemm_bn<256>(which, ma, mb, gp, g.M, g.N, st, true)
-                : launch_gemm_bn<128>(which, ma, mb, gp, g.M, g.N, st, true);
+  e = bn == 256 ? launch_gemm_bn<256>(which, maps, gp, g.M, g.N, st, true)
+                : launch_gemm_bn<128>(which, maps, gp, g.M, g.N, st, true);
   if (e != CSWATTN_OK) return e;
   {
     ScopedTiming tm(CSWATTN_K_GEMM, st);
-    e = bn == 256 ? launch_gemm_bn<256>(which, ma, mb, gp, g.M, g.N, st, false)
-                  : launch_gemm_bn<128>(which, ma, mb, gp, g.M, g.N, st, false);
+    e = bn == 256 ? launch_gemm_bn<256>(which, maps, gp, g.M, g.N, st, false)
+                  : launch_gemm_bn<128>(which, maps, gp, g.M, g.N, st, false);
   }
   if (e != CSWATTN_OK) return e;
   return launched("matrix product launch");
@@ -1456,20 +1516,59 @@ cswattn_status attn_qkv_bwd(const cswattn_layer* layer, const void* x, long long
   const int M = static_cast<int>(BT);
   const long long hq = static_cast<long long>(s.H) * s.D, hk = static_cast<long long>(s.Hk) * s.D;
   const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(w_qkv);
-  // dx = dQ W_q + dK W_k + dV W_v (W_* rows of the stacked weight, MN-major operands).
-  const GemmArgs g[6] = {
-      {M, C, static_cast<int>(hq), false, true, dQ, w, nullptr, hq, C, 0, C, 1.f, 0.f, dx},
-      {M, C, static_cast<int>(hk), false, true, dK, w + hq * C, dx, hk, C, C, C, 1.f, 1.f, dx},
-      {M, C, static_cast<int>(hk), false, true, dV, w + (hq + hk) * C, dx, hk, C, C, C, 1.f, 1.f, dx},
-      // dW_q = dQ^T x, dW_k = dK^T x, dW_v = dV^T x (float32 rows of the stacked gradient).
+  const int nr = static_cast<int>(hq + 2 * hk);  // rows of the stacked weight
+  CHECK_PTR(dQ, 16);
+  CHECK_PTR(dK, 16);
+  CHECK_PTR(dV, 16);
+  CHECK_PTR(x, 16);
+  CHECK_PTR(w_qkv, 16);
+  // dx = dQ W_q + dK W_k + dV W_v: one product whose K is the three segments
+  // (W_* rows of the stacked weight, MN-major), so dx is rounded once.
+  const GemmArgs gx{M, C, nr, false, true, dQ, w, nullptr, hq, C, 0, C, 1.f, 0.f, dx};
+  GemmSegs sx;
+  sx.n = 3;
+  sx.along_m = false;
+  const void* dys[3] = {dQ, dK, dV};
+  const long long lds[3] = {hq, hk, hk};
+  for (int i = 0; i < 3; ++i) {
+    sx.A[i] = dys[i];
+    sx.B[i] = w + (i == 0 ? 0 : (i == 1 ? hq : hq + hk)) * C;
+    sx.lda[i] = lds[i];
+    sx.ldb[i] = C;
+    sx.ext[i] = static_cast<int>(lds[i]);
+  }
+  // dW = [dQ dK dV]^T x (float32 rows of the stacked gradient): one product
+  // with M made of the three segments when the query and key blocks span
+  // whole 128-row tiles, else three products.
+  const GemmArgs gw{nr, C, M, true, true, dQ, x, nullptr, hq, x_stride, 0, C, 1.f, 0.f, dw_qkv, true};
+  GemmSegs sw;
+  sw.n = 3;
+  sw.along_m = true;
+  for (int i = 0; i < 3; ++i) {
+    sw.A[i] = dys[i];
+    sw.lda[i] = lds[i];
+    sw.ext[i] = static_cast<int>(lds[i]);
+  }
+  sw.B[0] = x;
+  sw.ldb[0] = x_stride;
+  const bool w_one = hq % gemm::kBM == 0 && hk % gemm::kBM == 0;
+  const GemmArgs gws[3] = {
       {static_cast<int>(hq), C, M, true, true, dQ, x, nullptr, hq, x_stride, 0, C, 1.f, 0.f, dw_qkv, true},
       {static_cast<int>(hk), C, M, true, true, dK, x, nullptr, hk, x_stride, 0, C, 1.f, 0.f, dw_qkv + hq * C, true},
-      {static_cast<int>(hk), C, M, true, true, dV, x, nullptr, hk, x_stride, 0, C, 1.f, 0.f, dw_qkv + (hq + hk) * C, true},
+      {static_cast<int>(hk), C, M, true, true, dV, x, nullptr, hk, x_stride, 0, C, 1.f, 0.f, dw_qkv + (hq + hk) * C,
+       true},
   };
-  for (const auto& a : g)
-    if ((st = check_gemm(a)) != CSWATTN_OK) return st;
+  if ((st = check_gemm(gx, false)) != CSWATTN_OK) return st;
+  if (w_one) {
+    if ((st = check_gemm(gw, false)) != CSWATTN_OK) return st;
+  } else {
+    for (const auto& a : gws)
+      if ((st = check_gemm(a)) != CSWATTN_OK) return st;
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  for (const auto& a : g)
+  if ((st = run_gemm(gx, cs, &sx)) != CSWATTN_OK) return st;
+  if (w_one) return run_gemm(gw, cs, &sw);
+  for (const auto& a : gws)
     if ((st = run_gemm(a, cs)) != CSWATTN_OK) return st;
   return CSWATTN_OK;
 }

@@ -45,7 +45,22 @@ struct Geo {
   static_assert(kSmemBytes <= 232448, "shared memory per block");
 };
 
+// Up to three operand segments. Along K: the product is the sum over the
+// segments of A_s B_s (each with its own K extent; the chunks of segment s
+// follow those of s - 1 into the same accumulator). Along M: rows
+// [mstart[s], mstart[s+1]) of C take A_s (row m - mstart[s]) with the
+// shared B (maps.b[0]); every segment but the last spans whole 128-row tiles.
+constexpr int kMaxSeg = 3;
+struct Maps {
+  CUtensorMap a[kMaxSeg];
+  CUtensorMap b[kMaxSeg];
+};
+
 struct Params {
+  int nseg;                // 1 .. kMaxSeg
+  int along_m;             // segments concatenated along M (else along K)
+  int kseg[kMaxSeg];       // along K: K extent of each segment
+  int mstart[kMaxSeg + 1]; // along M: first row of each segment, then M
   int M, N, K;
   float alpha, beta;
   const __nv_bfloat16* D;  // (M x N) row-major with ldd, or null when beta == 0
@@ -84,8 +99,7 @@ __device__ __forceinline__ uint64_t kstep_ofs(int kk) {
 
 template <bool A_MN, bool B_MN, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const Params p) {
+    gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
   using G = Geo<BN>;
   constexpr int kStages = G::kStages, kStageBytes = G::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -100,7 +114,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kStages + 6);
   const int warp = warp_id(), lane = lane_id();
-  const int nk = (p.K + kBK - 1) / kBK;
+  // K chunks of a tile (along K: the segments' chunks one after the other).
+  int nk = (p.K + kBK - 1) / kBK;
+  if (!p.along_m) {
+    nk = 0;
+    for (int sg = 0; sg < p.nseg; ++sg) nk += (p.kseg[sg] + kBK - 1) / kBK;
+  }
   const int ntn = (p.N + BN - 1) / BN;
   const int ntiles = ((p.M + kBM - 1) / kBM) * ntn;
   // Tiles of this CTA: blockIdx.x, + gridDim.x, ... (row-major over the
@@ -108,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int my_tiles = static_cast<int>(blockIdx.x) < ntiles
                            ? (ntiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
                            : 0;
-  if (!check_bounds(my_tiles >= 1 && nk >= 1)) return;  // checked build
+  if (!check_bounds(my_tiles >= 1 && nk >= 1 && p.nseg >= 1 && p.nseg <= kMaxSeg)) return;  // checked build
   auto tile_origin = [&](int li, int& m0, int& n0) {
     const int t = static_cast<int>(blockIdx.x) + li * static_cast<int>(gridDim.x);
     m0 = (t / ntn) * kBM;
@@ -142,21 +161,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (chunks of all the CTA's tiles)
-      prefetch_tmap(&tmA);
-      prefetch_tmap(&tmB);
+      for (int sg = 0; sg < p.nseg; ++sg) {
+        prefetch_tmap(&maps.a[sg]);
+        prefetch_tmap(&maps.b[sg]);
+      }
       int issued[kStages] = {};
       bool ok = true;
       for (int li = 0; ok && li < my_tiles; ++li) {
         int m0, n0;
         tile_origin(li, m0, n0);
-        for (int kc = 0; kc < nk; ++kc) {
-          const int g = li * nk + kc, s = g % kStages, use = g / kStages;
+        // Along M: the tile's segment (tiles never straddle two) and its row in it.
+        int sm = 0;
+        if (p.along_m)
+          while (sm + 1 < p.nseg && m0 >= p.mstart[sm + 1]) ++sm;
+        const int ma = p.along_m ? m0 - p.mstart[sm] : m0;
+        int sg = p.along_m ? sm : 0, kc = 0;  // along K: segment sg, its chunk kc
+        for (int c = 0; c < nk; ++c) {
+          if (!p.along_m) {
+            while (kc * kBK >= p.kseg[sg]) {
+              ++sg;
+              kc = 0;
+            }
+          }
+          const int g = li * nk + c, s = g % kStages, use = g / kStages;
           if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, wc))) break;
           uint8_t* st = smem + s * kStageBytes;
           mbar_expect_tx(&full[s], kStageBytes);
-          load_operand<A_MN, kBM>(&tmA, &full[s], st, m0, kc * kBK);
-          load_operand<B_MN, BN>(&tmB, &full[s], st + kOpBytesA, n0, kc * kBK);
+          load_operand<A_MN, kBM>(&maps.a[sg], &full[s], st, ma, kc * kBK);
+          load_operand<B_MN, BN>(&maps.b[p.along_m ? 0 : sg], &full[s], st + kOpBytesA, n0, kc * kBK);
           ++issued[s];
+          ++kc;
         }
       }
       for (int s = 0; s < kStages; ++s)

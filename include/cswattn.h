@@ -174,8 +174,12 @@ cswattn_status attn_qkv_prologue_fp8(const cswattn_layer* layer, const void* x, 
  * dV (gradients of the raw q, k, v):
  *   dx     = dQ w_q + dK w_k + dV w_v         (B, T, C), bf16, row stride C
  *   dw_qkv = [dQ dK dV]^T x[..., :C]           ((n_head + 2 n_kv_head) D, C), float32
- * Six tensor-core matrix products (cswattn_gemm_bf16). x, x_stride, C,
- * w_qkv as for attn_qkv_prologue; bf16 layers only. */
+ * Two tensor-core matrix products (the kernel of cswattn_gemm_bf16 with
+ * operands in three segments): dx in one accumulator over the three weight
+ * blocks (rounded to bf16 once), dw_qkv over the three gradient blocks (three
+ * products when n_head * D or n_kv_head * D is not a multiple of 128). x,
+ * x_stride, C, w_qkv as for attn_qkv_prologue; all pointers 16-byte aligned;
+ * bf16 layers only. */
 cswattn_status attn_qkv_bwd(const cswattn_layer* layer, const void* x, long long x_stride, int C,
                             const void* w_qkv, const void* dQ, const void* dK, const void* dV, void* dx,
                             float* dw_qkv, void* stream);

@@ -47,6 +47,7 @@ def gpu_prologue(spec, x, C, w, ve, gate):
     (1, 257, 96, 4, 4, 64, 257, True),
     (1, 200, 64, 2, 1, 128, 50, False),
     (1, 130, 128, 3, 1, 128, 64, True),   # 5 stacked heads: a (q, k) pair and a lone value head
+    (1, 150, 64, 3, 1, 64, 64, True),     # 3 x 64 query rows: dW as three products, not one
 ])
 def test_qkv_prologue_and_backward_match_oracle(B, T, C, H, Hk, D, W, has_ve):
     spec = cs.LayerSpec(B, T, H, Hk, D, W, has_ve=has_ve, dtype="bf16")
