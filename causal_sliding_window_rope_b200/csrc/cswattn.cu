@@ -581,12 +581,13 @@ template <bool AMN, bool BMN, int BN>
 cswattn_status launch_gemm_t(const gemm::Maps& maps, const gemm::Params& gp, int M, int N, cudaStream_t st,
                              bool prepare_only) {
   constexpr int kSmem = gemm::Geo<BN>::kSmemBytes;
-  const cswattn_status e = set_smem(gemm::gemm_kernel<AMN, BMN, BN>, kSmem);
+  auto kern = gp.nseg > 1 ? gemm::gemm_kernel<AMN, BMN, BN, true> : gemm::gemm_kernel<AMN, BMN, BN, false>;
+  const cswattn_status e = set_smem(kern, kSmem);
   if (e != CSWATTN_OK || prepare_only) return e;
   // Persistent: at most one CTA per SM (148), each walking its share of the tiles.
   const long long tiles = static_cast<long long>((N + BN - 1) / BN) * ((M + gemm::kBM - 1) / gemm::kBM);
   const dim3 grid(static_cast<unsigned>(std::min<long long>(tiles, 148)));
-  launch_pdl(gemm::gemm_kernel<AMN, BMN, BN>, grid, dim3(gemm::kThreads), kSmem, st, maps, gp);
+  launch_pdl(kern, grid, dim3(gemm::kThreads), kSmem, st, maps, gp);
   return CSWATTN_OK;
 }
 

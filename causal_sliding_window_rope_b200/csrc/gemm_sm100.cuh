@@ -97,7 +97,8 @@ __device__ __forceinline__ uint64_t kstep_ofs(int kk) {
   return static_cast<uint64_t>((MN ? kk * 16 * 128 : kk * 32) >> 4);
 }
 
-template <bool A_MN, bool B_MN, int BN>
+// SEG: operands in segments (else one A and one B: maps.a[0], maps.b[0]).
+template <bool A_MN, bool B_MN, int BN, bool SEG>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
   using G = Geo<BN>;
@@ -116,10 +117,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   // K chunks of a tile (along K: the segments' chunks one after the other).
   int nk = (p.K + kBK - 1) / kBK;
-  if (!p.along_m) {
-    nk = 0;
-    for (int sg = 0; sg < p.nseg; ++sg) nk += (p.kseg[sg] + kBK - 1) / kBK;
-  }
+  if (SEG && !p.along_m)
+    nk = (p.kseg[0] + kBK - 1) / kBK + (p.nseg > 1 ? (p.kseg[1] + kBK - 1) / kBK : 0) +
+         (p.nseg > 2 ? (p.kseg[2] + kBK - 1) / kBK : 0);
   const int ntn = (p.N + BN - 1) / BN;
   const int ntiles = ((p.M + kBM - 1) / kBM) * ntn;
   // Tiles of this CTA: blockIdx.x, + gridDim.x, ... (row-major over the
@@ -161,9 +161,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (chunks of all the CTA's tiles)
-      for (int sg = 0; sg < p.nseg; ++sg) {
-        prefetch_tmap(&maps.a[sg]);
-        prefetch_tmap(&maps.b[sg]);
+      // Segment operands by constant index (no dynamic indexing of the
+      // kernel parameters): c1, c2 = first chunk of segments 1 and 2 along K.
+      const int c1 = (p.kseg[0] + kBK - 1) / kBK;
+      const int c2 = c1 + (p.nseg > 1 ? (p.kseg[1] + kBK - 1) / kBK : 0);
+      const int m1 = p.mstart[1], m2 = p.mstart[2];
+      prefetch_tmap(&maps.a[0]);
+      prefetch_tmap(&maps.b[0]);
+      if (SEG && p.nseg > 1) {
+        prefetch_tmap(&maps.a[1]);
+        if (!p.along_m) prefetch_tmap(&maps.b[1]);
+      }
+      if (SEG && p.nseg > 2) {
+        prefetch_tmap(&maps.a[2]);
+        if (!p.along_m) prefetch_tmap(&maps.b[2]);
       }
       int issued[kStages] = {};
       bool ok = true;
@@ -171,26 +182,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         int m0, n0;
         tile_origin(li, m0, n0);
         // Along M: the tile's segment (tiles never straddle two) and its row in it.
-        int sm = 0;
-        if (p.along_m)
-          while (sm + 1 < p.nseg && m0 >= p.mstart[sm + 1]) ++sm;
-        const int ma = p.along_m ? m0 - p.mstart[sm] : m0;
-        int sg = p.along_m ? sm : 0, kc = 0;  // along K: segment sg, its chunk kc
+        int sm = 0, ma = m0;
+        if (SEG && p.along_m) {
+          sm = (p.nseg > 2 && m0 >= m2) ? 2 : ((p.nseg > 1 && m0 >= m1) ? 1 : 0);
+          ma = m0 - (sm == 2 ? m2 : (sm == 1 ? m1 : 0));
+        }
         for (int c = 0; c < nk; ++c) {
-          if (!p.along_m) {
-            while (kc * kBK >= p.kseg[sg]) {
-              ++sg;
-              kc = 0;
-            }
+          // Along K: segment of chunk c and the chunk within it.
+          int sk = 0, kc = c, sb = 0;
+          if constexpr (SEG) {
+            sk = p.along_m ? sm : (c >= c2 && p.nseg > 2 ? 2 : (c >= c1 && p.nseg > 1 ? 1 : 0));
+            kc = p.along_m ? c : c - (sk == 2 ? c2 : (sk == 1 ? c1 : 0));
+            sb = p.along_m ? 0 : sk;
           }
+          const CUtensorMap* mapA = sk == 2 ? &maps.a[2] : (sk == 1 ? &maps.a[1] : &maps.a[0]);
+          const CUtensorMap* mapB = sb == 2 ? &maps.b[2] : (sb == 1 ? &maps.b[1] : &maps.b[0]);
           const int g = li * nk + c, s = g % kStages, use = g / kStages;
           if (use > 0 && !(ok = mbar_wait(&empty[s], (use - 1) & 1, wc))) break;
           uint8_t* st = smem + s * kStageBytes;
           mbar_expect_tx(&full[s], kStageBytes);
-          load_operand<A_MN, kBM>(&maps.a[sg], &full[s], st, ma, kc * kBK);
-          load_operand<B_MN, BN>(&maps.b[p.along_m ? 0 : sg], &full[s], st + kOpBytesA, n0, kc * kBK);
+          load_operand<A_MN, kBM>(mapA, &full[s], st, ma, kc * kBK);
+          load_operand<B_MN, BN>(mapB, &full[s], st + kOpBytesA, n0, kc * kBK);
           ++issued[s];
-          ++kc;
         }
       }
       for (int s = 0; s < kStages; ++s)
