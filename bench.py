@@ -297,13 +297,57 @@ def measure_stack(st, args, world, dist, flush_buf, warmup, steps, with_split=Tr
     return per_step, ktimes
 
 
-def kernel_table(ktimes, w, steps):
+def bwd_parts_of(cs, spec):
+    """Backward parts per key tile, read back from the documented workspace
+    layout: dq accumulator, dK and dV partial slots (parts x (B,T,Hk,D)
+    float32 each), Delta and lse2 ((B,H,Tpad) float32), each padded to 256."""
+    pad = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    ws = cs.attn_bwd_workspace_bytes(spec)
+    B, T, H, Hk, D = spec.B, spec.T, spec.n_head, spec.n_kv_head, spec.head_dim
+    tpad = (T + 63) // 64 * 64
+    for parts in range(1, 9):
+        if pad(B * H * T * D * 4) + 2 * pad(B * T * Hk * D * parts * 4) + 2 * pad(B * H * tpad * 4) == ws:
+            return parts
+    return None
+
+
+def row_bytes(w, cs):
+    """Bytes each row kernel moves per step (all layers), by its design: the
+    prologue reads q, k, v (ve, gate) and writes q~, k~, v_eff and the rstd
+    rows; the preprocess reads O, dO and lse, writes Delta and lse2 and clears
+    the float32 dq accumulator; the epilogue reads the float32 dq~ and the
+    parts' dk~/dv_eff, q, k (ve, gate), rstd, and writes dQ, dK, dV (dve,
+    dgate)."""
+    B, T, H, Hk, D = w.B, w.T, w.H, w.Hk, w.D
+    e = 2  # bf16
+    nq, nk, tok = B * T * H * D, B * T * Hk * D, B * T
+    tpad = (T + 63) // 64 * 64
+    out = {"prologue": 0, "bwd_pre": 0, "bwd_epi": 0}
+    for W, ve in zip(w.windows, w.ve):
+        spec = cs.LayerSpec(B, T, H, Hk, D, W, has_ve=ve, dtype="bf16", rope_base=w.rope_base, eps=w.eps)
+        parts = bwd_parts_of(cs, spec) or 1
+        vb = (nk * e + tok * Hk * e) if ve else 0
+        out["prologue"] += 2 * (nq + 2 * nk) * e + vb + tok * (H + Hk) * 4
+        out["bwd_pre"] += 2 * nq * e + B * H * T * 4 + 2 * B * H * tpad * 4 + nq * 4
+        out["bwd_epi"] += (nq * 4 + 2 * parts * nk * 4 + (nq + nk) * e + tok * (H + Hk) * 4 + vb
+                           + (nq + 2 * nk) * e + ((nk * e + tok * Hk * e) if ve else 0))
+    return out
+
+
+def kernel_table(ktimes, w, steps, cs=None, hbm=None):
     _, flops_fwd, flops_bwd = layer_flops(w)
     kern = {k: {"ms_per_step": round(v[0] / steps, 4), "launches": v[1]}
             for k, v in ktimes.items() if not k.startswith("_")}
     for k, fl in (("fwd", flops_fwd), ("bwd", flops_bwd)):
         if k in ktimes and ktimes[k][0] > 0:
             kern[k]["tflops"] = round(sum(fl) * steps / (ktimes[k][0] * 1e-3) / 1e12, 2)
+    if cs is not None and hbm:
+        for k, nbytes in row_bytes(w, cs).items():
+            if k in ktimes and ktimes[k][0] > 0:
+                gbs = nbytes * steps / (ktimes[k][0] * 1e-3) / 1e9
+                kern[k]["bytes_per_step"] = nbytes
+                kern[k]["gbs"] = round(gbs, 1)
+                kern[k]["frac_hbm"] = round(gbs / hbm, 4)
     if "_pass_ms" in ktimes:
         kern["_pass"] = {"ms_per_step": round(ktimes["_pass_ms"][0] / steps, 4),
                          "note": "second timed pass with an event pair around every kernel"}
@@ -330,7 +374,7 @@ def other_configs(args, dev, peaks, peak_src, flush_buf, cs, synth):
                              "nominal_dense": round(fl / (ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS, 4)},
                          "roofline": roofline({k: v for k, v in kt.items() if not k.startswith("_")},
                                               w, args.steps, peaks, peak_src),
-                         "kernels": kernel_table(kt, w, args.steps)}
+                         "kernels": kernel_table(kt, w, args.steps, cs, peaks.get("hbm_gbs"))}
         del st
         torch.cuda.empty_cache()
     return out
@@ -441,7 +485,7 @@ def run_ours(args):
                 "nominal_dense": round(value / world / NOMINAL_BF16_TFLOPS, 4),
                 "peak_source": peak_src},
             "roofline": roofline(kt, w, args.steps, peaks, peak_src),
-            "kernels": kernel_table(ktimes, w, args.steps),
+            "kernels": kernel_table(ktimes, w, args.steps, cs, peaks.get("hbm_gbs")),
             "gpu_launches": sum(n for _, n in kt.values()),
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": st.h2d, "d2h_bytes_per_step": st.d2h,
@@ -829,8 +873,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", type=int, choices=BF16_CONFIGS, default=DEFAULT_CONFIG,
                     help="workload of the headline line (2: d12, 3: d12 SSSL, 4: d24 GQA SSSL, "
