@@ -54,6 +54,55 @@ constexpr int kRegLo = 80;   // producer / MMA warpgroup
 constexpr int kRegHi = 208;  // each softmax warpgroup
 static_assert(128 * kRegLo + 256 * kRegHi <= kThreads * 168, "register budget");
 
+// Pairs of exponentials (of the 16 per 32-column chunk) taken on the FMA
+// pipe instead of the MUFU unit: pair i when bit i is set.
+constexpr unsigned kPolyPairs = 0x8080u;
+
+// Packed pairs of fp32 values (one 64-bit register pair) for the f32x2
+// arithmetic of sm_100: one instruction per pair of softmax elements.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe (Cody-Waite range reduction and a
+// polynomial): x = n + f with n = rint(x) (the 1.5 * 2^23 rounding trick)
+// and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial whose coefficients were
+// fitted to the relative error on that interval (max 7.5e-5, below half an
+// ulp of bf16), and n is added to the exponent field. x is clamped to -125,
+// so -inf gives 2^-125 (a normal number) rather than 0: far below anything
+// that reaches a row sum beside its maximum's 1.
+__device__ __forceinline__ void exp2_fma_x2(uint64_t x2, float& p0, float& p1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t2 = f2_add(x2, f2_pack(12582912.f, 12582912.f));
+  const uint64_t n2 = f2_add(t2, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f2 = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
+  uint64_t q2 = f2_fma(f2_pack(0.05517132f, 0.05517132f), f2, f2_pack(0.24261054f, 0.24261054f));
+  q2 = f2_fma(q2, f2, f2_pack(0.69326099f, 0.69326099f));
+  q2 = f2_fma(q2, f2, f2_pack(0.99992811f, 0.99992811f));
+  float q0, q1, t0, t1;
+  f2_unpack(q2, q0, q1);
+  f2_unpack(t2, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 struct Params {
   int B, T, H, Hk, W, g, nq, npairs;
   float scale_log2;  // softmax scale * log2(e)
@@ -231,11 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ring(j, 1, s, use);
         const int n = j - lo_t[X];
         if (!mbar_wait(&kv_full[s], use & 1, wc)) return false;
-        if (!mbar_wait(&p_full[X], n & 1, wc)) return false;
-        tc_fence_after();
         const uint64_t vd = dV0 + static_cast<uint64_t>((s * kTileBytes) >> 4);
         const uint32_t o_tmem = tmem + 256u + static_cast<uint32_t>(X) * 128u;
         const uint32_t p_tmem = tmem + static_cast<uint32_t>(X) * 128u;
+        if (!mbar_wait(&p_full[X], n & 1, wc)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
@@ -300,22 +349,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         const int k0 = j * kBM;
         if (k0 + kBM - 1 > q0 || q0 + kBM - 1 - k0 >= p.W) {
+          // Row r keeps the keys k0 + e with a <= e <= b (causal: kj <= qi;
+          // window: qi - kj < W); an empty range keeps none. Chunks that
+          // every lane of the warp keeps whole are skipped.
+          int a = max(qi - p.W + 1 - k0, 0);
+          const int b = min(qi - k0, kBM - 1);
+          unsigned span = static_cast<unsigned>(b - a);
+          if (b < a) {
+            a = 1 << 20;
+            span = 0u;
+          }
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 4; ++c) {
+            if (__all_sync(0xffffffffu, a <= 32 * c && 32 * c + 31 <= b)) continue;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kj = k0 + c * 32 + i;
-              if (kj > qi || qi - kj >= p.W) sv[c][i] = __float_as_uint(-INFINITY);
-            }
+            for (int i = 0; i < 32; ++i)
+              if (static_cast<unsigned>(32 * c + i - a) > span) sv[c][i] = __float_as_uint(-INFINITY);
+          }
         }
-        // Row max: one chain of three-input maxima per 32-column chunk.
+        // Row max: a tree of three-input maxima per 32-column chunk.
         float mp[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float m = fmax3(__uint_as_float(sv[c][0]), __uint_as_float(sv[c][1]), __uint_as_float(sv[c][2]));
+          float t[11];
 #pragma unroll
-          for (int i = 3; i < 31; i += 2) m = fmax3(m, __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
-          mp[c] = fmaxf(m, __uint_as_float(sv[c][31]));
+          for (int k = 0; k < 10; ++k)
+            t[k] = fmax3(__uint_as_float(sv[c][3 * k]), __uint_as_float(sv[c][3 * k + 1]),
+                         __uint_as_float(sv[c][3 * k + 2]));
+          t[10] = fmaxf(__uint_as_float(sv[c][30]), __uint_as_float(sv[c][31]));
+          mp[c] = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]),
+                        fmaxf(fmax3(t[6], t[7], t[8]), fmaxf(t[9], t[10])));
         }
         float mx = fmax3(mp[0], mp[1], fmaxf(mp[2], mp[3])) * c2;
         float alpha = 1.f;
@@ -340,20 +403,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st_wait();
         }
         const float mu = (m2 == -INFINITY) ? 0.f : m2;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+        // x = c S - mu and the partial row sums, a pair of elements per
+        // f32x2 instruction; four independent accumulator pairs.
+        const uint64_t c2x2 = f2_pack(c2, c2), nmu2 = f2_pack(-mu, -mu);
+        uint64_t ls2[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) ls2[a] = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -mu));
-            const float p1 = ex2(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -mu));
-            ls[i & 3] += p0 + p1;
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sv[c][2 * i]), __uint_as_float(sv[c][2 * i + 1])), c2x2, nmu2);
+            float p0, p1;
+            if ((kPolyPairs >> i) & 1u) {
+              exp2_fma_x2(x2, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            ls2[i & 3] = f2_add(ls2[i & 3], f2_pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tS + c * 16, pk);
         }
-        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        float la, lb, lc, ld;
+        f2_unpack(f2_add(ls2[0], ls2[1]), la, lb);
+        f2_unpack(f2_add(ls2[2], ls2[3]), lc, ld);
+        l = l * alpha + ((la + lb) + (lc + ld));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[X]);
