@@ -16,8 +16,9 @@
 namespace cswattn {
 
 // Row terms of the backward, in the padded layout (B, H, Tpad) with Tpad a
-// multiple of 64: delta = dO.O and lse2 = lse * log2(e); past T, delta = 0
-// and lse2 = +inf (so exp2(s - lse2) = 0 for padding queries).
+// multiple of 64: delta = dO.O and nlse2 = -lse * log2(e) (negated, so that
+// the backward forms c2 s + nlse2 with one fused multiply-add); past T,
+// delta = 0 and nlse2 = -inf (so exp2(c2 s + nlse2) = 0 for padding queries).
 struct PreParams {
   long long rows;  // B * T * H
   int T, H, Tpad;
@@ -26,7 +27,7 @@ struct PreParams {
   const void *O, *dO;
   const float* lse;  // (B, H, T)
   float* delta;      // (B, H, Tpad)
-  float* lse2;       // (B, H, Tpad)
+  float* nlse2;      // (B, H, Tpad)
   float* dq_zero;    // (B, T, H, D) accumulator to clear, or null
 };
 
@@ -107,11 +108,11 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
       const long long b = s_b[tt], t = s_t[tt];
       const long long o = (b * p.H + h) * p.Tpad;
       p.delta[o + t] = acc;
-      p.lse2[o + t] = p.lse[(b * p.H + h) * p.T + t] * 1.4426950408889634f;
+      p.nlse2[o + t] = p.lse[(b * p.H + h) * p.T + t] * -1.4426950408889634f;
       if (t == p.T - 1) {
         for (long long tp = p.T; tp < p.Tpad; ++tp) {
           p.delta[o + tp] = 0.f;
-          p.lse2[o + tp] = INFINITY;
+          p.nlse2[o + tp] = -INFINITY;
         }
       }
     }

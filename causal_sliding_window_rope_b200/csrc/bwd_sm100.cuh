@@ -15,7 +15,8 @@
 // once. Per step (transposed products, keys on the TMEM lanes):
 //   S^T  = K Q^T      (M=128 keys, N=64 queries, K=128 d)   SS MMA
 //   dP^T = V dO^T     (same shape)                         SS MMA
-//   softmax warps: P^T = exp2(c2 S^T - lse2), dS^T = P^T (dP^T - Delta),
+//   softmax warps: P^T = exp2(c2 S^T - lse2), dS^T = P^T (dP^T - Delta)
+//                  (pairs of elements per f32x2 instruction),
 //                  both as bf16 into TMEM (the step's dQ^T columns), and
 //                  dS^T also into shared memory (128B-swizzled)
 //   dV  += P^T dO     (M=128 keys, N=128 d, K=64)           TS MMA (P^T in TMEM)
@@ -65,7 +66,7 @@ constexpr int kOffBar = kOffDQS + 4 * kDQPanel;
 // of 128 rows x 32 float32.
 constexpr int kF32Panel = kBN * 128;
 static_assert(kOffQD + 8 * kF32Panel <= kOffDQS, "write-out staging");
-constexpr int kOffRow = kOffBar + 256;         // per Q stage: lse2[64], delta[64]
+constexpr int kOffRow = kOffBar + 256;         // per Q stage: nlse2[64], delta[64]
 constexpr int kSmemBytes = kOffRow + kQStages * 2 * kBQ * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
@@ -87,7 +88,7 @@ struct Params {
   long long kv_stride;     // elements between the parts' dK/dV partial slots
   float scale_log2;  // c * log2(e)
   float scale;       // c
-  const float* lse2;   // (B,H,Tpad) lse * log2(e), +inf past T
+  const float* nlse2;  // (B,H,Tpad) -lse * log2(e), -inf past T
   const float* delta;  // (B,H,Tpad) dO.O, 0 past T
   float* dq_acc;       // (B,T,H,D), accumulated (must start at zero)
   float* dk_acc;       // [parts] x (B,T,Hk,D) partial sums
@@ -124,8 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_staged = bars + 20;  // dK/dV rows written to shared memory
   uint64_t* dqs_full = bars + 21;   // [2] half of the dQ staging tile written (128 arrivals)
   uint64_t* dqs_free = bars + 23;   // [2] the reduction has read that half
-  float* s_lse2 = reinterpret_cast<float*>(smem + kOffRow);        // [kQStages][64]
-  float* s_delta = s_lse2 + kQStages * kBQ;                         // [kQStages][64]
+  float* s_nlse2 = reinterpret_cast<float*>(smem + kOffRow);       // [kQStages][64]
+  float* s_delta = s_nlse2 + kQStages * kBQ;                        // [kQStages][64]
 
   const int warp = warp_id(), lane = lane_id();
 
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(&tmDO, &q_full[st], od + kQPanel, 64, h, q0, b);
         // Row terms of the step's 64 queries (padded layout: always in range).
         const size_t ro = (static_cast<size_t>(b) * p.H + h) * p.Tpad + q0;
-        bulk_load(s_lse2 + st * kBQ, p.lse2 + ro, kBQ * 4, &q_full[st]);
+        bulk_load(s_nlse2 + st * kBQ, p.nlse2 + ro, kBQ * 4, &q_full[st]);
         bulk_load(s_delta + st * kBQ, p.delta + ro, kBQ * 4, &q_full[st]);
         ++nq[st];
         if (++st == kQStages) {
@@ -340,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0; n < N; ++n, c.next()) {
       const int st = n % kQStages, use = n / kQStages;
       const int q0 = c.q0();
-      // S^T/dP^T of this step, and (same stage barrier as Q/dO) its lse2/Delta.
+      // S^T/dP^T of this step, and (same stage barrier as Q/dO) its nlse2/Delta.
       bool got = mbar_wait(sp_full, n & 1, wc);
       got = got && mbar_wait(&q_full[st], use & 1, wc);
       if (!__all_sync(0xffffffffu, got)) {
@@ -356,33 +357,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(sp_free);  // the MMA warp may overwrite SP now
-      const bool need_mask = (q0 < k0 + kBN - 1) || (q0 + kBQ - 1 - k0 >= p.W);
-      const float4* L2 = reinterpret_cast<const float4*>(s_lse2 + st * kBQ);
+      const float4* NL = reinterpret_cast<const float4*>(s_nlse2 + st * kBQ);
       const float4* DL = reinterpret_cast<const float4*>(s_delta + st * kBQ);
+      const uint64_t c2x2 = f2_pack(c2, c2);
       uint32_t pp[32], dd[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          const float4 l4 = L2[(c * 32 + i) >> 2];
+          const float4 l4 = NL[(c * 32 + i) >> 2];
           const float4 d4 = DL[(c * 32 + i) >> 2];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-          const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = c * 32 + i + e;
-            const int q = q0 + col;
-            float pr = ex2(fmaf(__uint_as_float(sv[c][i + e]), c2, -lv[e]));
-            if (need_mask && (q < kj || q - kj >= p.W)) pr = 0.f;
-            pv[e] = pr;
-            dsv[e] = pr * (__uint_as_float(dv[c][i + e]) - dl[e]);
+          for (int h = 0; h < 2; ++h) {
+            const int e = i + 2 * h;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), c2x2,
+                                       h == 0 ? f2_pack(l4.x, l4.y) : f2_pack(l4.z, l4.w));
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+            const uint64_t ds2 =
+                f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dv[c][e]), __uint_as_float(dv[c][e + 1])),
+                                  h == 0 ? f2_pack(d4.x, d4.y) : f2_pack(d4.z, d4.w)));
+            float p0, p1, s0, s1;
+            f2_unpack(p2, p0, p1);
+            f2_unpack(ds2, s0, s1);
+            pp[c * 16 + e / 2] = pack_bf16x2(p0, p1);
+            dd[c * 16 + e / 2] = pack_bf16x2(s0, s1);
           }
-          pp[c * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
-          pp[c * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-          dd[c * 16 + i / 2] = pack_bf16x2(dsv[0], dsv[1]);
-          dd[c * 16 + i / 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
+      if ((q0 < k0 + kBN - 1) || (q0 + kBQ - 1 - k0 >= p.W)) {
+        // Key row kj sees the queries kj <= q < kj + W: columns [a, b] of
+        // the step. Pairs outside are zeroed (P and dS alike); 16-pair
+        // chunks that every lane of the warp keeps whole are skipped.
+        int a = max(kj - q0, 0);
+        const int bq = min(kj + p.W - 1 - q0, kBQ - 1);
+        unsigned span = static_cast<unsigned>(bq - a);
+        if (bq < a) {
+          a = 1 << 20;
+          span = 0u;
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (__all_sync(0xffffffffu, a <= 32 * c && 32 * c + 31 <= bq)) continue;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const bool k0v = static_cast<unsigned>(32 * c + 2 * i - a) <= span;
+            const bool k1v = static_cast<unsigned>(32 * c + 2 * i + 1 - a) <= span;
+            const uint32_t keep = (k0v ? 0x0000ffffu : 0u) | (k1v ? 0xffff0000u : 0u);
+            pp[c * 16 + i] &= keep;
+            dd[c * 16 + i] &= keep;
+          }
+        }
+      }
       // Buffer db (TMEM dQ^T columns and shared dS^T) was last used by step
       // n-2: wait until that step's dQ^T has been drained and its dQ^T
       // product has read the shared dS^T.

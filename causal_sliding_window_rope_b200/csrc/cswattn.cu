@@ -464,7 +464,7 @@ struct ScopedTiming {
 size_t pad256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Workspace {
-  float *dq_acc, *dk_acc, *dv_acc, *delta, *lse2;
+  float *dq_acc, *dk_acc, *dv_acc, *delta, *nlse2;
   int Tpad;
   size_t bytes;
 };
@@ -506,7 +506,7 @@ Workspace carve(const Shape& s, void* base) {
   off += pad256(nk * 4);
   w.delta = reinterpret_cast<float*>(p + off);
   off += pad256(nr * 4);
-  w.lse2 = reinterpret_cast<float*>(p + off);
+  w.nlse2 = reinterpret_cast<float*>(p + off);
   off += pad256(nr * 4);
   w.Tpad = padded_T(s.T);
   w.bytes = off;
@@ -1095,7 +1095,7 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
   pre.dO = dO;
   pre.lse = lse;
   pre.delta = w.delta;
-  pre.lse2 = w.lse2;
+  pre.nlse2 = w.nlse2;
   // The tensor-core backward accumulates dq~ with reductions: zero it here.
   pre.dq_zero = s.bf16 ? w.dq_acc : nullptr;
 
@@ -1149,7 +1149,7 @@ cswattn_status attn_bwd(const cswattn_layer* layer, const void* q, const void* k
     bp.scale_log2 = s.scale * 1.4426950408889634f;
     bp.scale = s.scale;
     bp.Tpad = w.Tpad;
-    bp.lse2 = w.lse2;
+    bp.nlse2 = w.nlse2;
     bp.delta = w.delta;
     bp.dq_acc = w.dq_acc;
     bp.dk_acc = w.dk_acc;

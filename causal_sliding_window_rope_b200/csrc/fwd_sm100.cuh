@@ -58,27 +58,6 @@ static_assert(128 * kRegLo + 256 * kRegHi <= kThreads * 168, "register budget");
 // pipe instead of the MUFU unit: pair i when bit i is set.
 constexpr unsigned kPolyPairs = 0x8080u;
 
-// Packed pairs of fp32 values (one 64-bit register pair) for the f32x2
-// arithmetic of sm_100: one instruction per pair of softmax elements.
-__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 // 2^x for a pair on the FMA pipe (Cody-Waite range reduction and a
 // polynomial): x = n + f with n = rint(x) (the 1.5 * 2^23 rounding trick)
 // and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial whose coefficients were
