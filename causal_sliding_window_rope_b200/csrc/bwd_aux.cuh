@@ -31,8 +31,10 @@ struct PreParams {
   float* dq_zero;    // (B, T, H, D) accumulator to clear, or null
 };
 
+// Shared-memory bytes of the staged preprocess for `tok` tokens: O and dO
+// rows, then the block's lse values (float32).
 __host__ __device__ inline size_t preprocess_stage_bytes(int tok, int H, int D, int esize) {
-  return 2 * static_cast<size_t>(tok) * H * D * esize;
+  return 2 * static_cast<size_t>(tok) * H * D * esize + static_cast<size_t>(tok) * H * 4;
 }
 
 // One CTA per `tok` consecutive tokens, staged like the prologue (one bulk
@@ -61,6 +63,9 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
     s_t[threadIdx.x] = static_cast<int>(tok % p.T);
   }
   pdl_wait();
+  // The block's lse values, staged next to the rows so that no row waits on
+  // a global load: float32 after the dO rows.
+  float* s_lse = reinterpret_cast<float*>(stage_smem + 2 * static_cast<size_t>(p.tok) * orow * sizeof(T));
   if constexpr (STAGED) {
     T* so = reinterpret_cast<T*>(stage_smem);
     T* sg = so + p.tok * orow;
@@ -72,6 +77,11 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
     }
     ob = so;
     gb = sg;
+    for (int i = threadIdx.x; i < ntt * p.H; i += blockDim.x) {
+      const long long tok = tok0 + i / p.H;
+      const long long b = tok / p.T, t = tok % p.T;
+      s_lse[i] = p.lse[(b * p.H + i % p.H) * p.T + t];
+    }
   }
   if (p.dq_zero) {
     // The block's rows of the dq accumulator (contiguous in (B,T,H,D)).
@@ -108,7 +118,7 @@ __global__ void __launch_bounds__(kPrologueThreads) preprocess_kernel(const PreP
       const long long b = s_b[tt], t = s_t[tt];
       const long long o = (b * p.H + h) * p.Tpad;
       p.delta[o + t] = acc;
-      p.nlse2[o + t] = p.lse[(b * p.H + h) * p.T + t] * -1.4426950408889634f;
+      p.nlse2[o + t] = (STAGED ? s_lse[tt * p.H + h] : p.lse[(b * p.H + h) * p.T + t]) * -1.4426950408889634f;
       if (t == p.T - 1) {
         for (long long tp = p.T; tp < p.Tpad; ++tp) {
           p.delta[o + tp] = 0.f;
@@ -135,12 +145,14 @@ struct EpiParams {
 };
 
 // Shared-memory bytes of the staged epilogue for `tok` tokens: dq~, the dk~
-// and dv_eff partial slots (float32), then q, k and ve (layer dtype).
+// and dv_eff partial slots (float32), then q, k and ve (layer dtype), then
+// the block's rstd_q, rstd_k and gate values (float32).
 __host__ __device__ inline size_t epilogue_stage_bytes(int tok, int H, int Hk, int D, int esize,
                                                        int parts, bool has_ve) {
   return static_cast<size_t>(tok) * D *
-         ((static_cast<size_t>(H) + 2 * static_cast<size_t>(parts) * Hk) * 4 +
-          (static_cast<size_t>(H) + (has_ve ? 2 : 1) * Hk) * esize);
+             ((static_cast<size_t>(H) + 2 * static_cast<size_t>(parts) * Hk) * 4 +
+              (static_cast<size_t>(H) + (has_ve ? 2 : 1) * Hk) * esize) +
+         static_cast<size_t>(tok) * (H + 2 * Hk) * 4;
 }
 
 template <int VEC>
@@ -200,6 +212,12 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
   const T* kb = static_cast<const T*>(p.k) + tok0 * kvrow;
   const T* eb = p.has_ve ? static_cast<const T*>(p.ve) + tok0 * kvrow : nullptr;
   const Stage stage{&s_bar};
+  // Staged row terms (float32): rstd_q [tok][H], rstd_k [tok][Hk], gate
+  // [tok][Hk], after the staged rows.
+  float* s_rterm = reinterpret_cast<float*>(
+      stage_smem + static_cast<size_t>(p.tok) * D *
+                       ((static_cast<size_t>(p.H) + 2 * static_cast<size_t>(p.parts) * p.Hk) * 4 +
+                        (static_cast<size_t>(p.H) + (p.has_ve ? 2 : 1) * p.Hk) * sizeof(T)));
   pdl_launch_dependents();
   tab.fill(tok0, p.T, p.omega, ntt);
   pdl_wait();
@@ -224,6 +242,13 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
       stage.copy(sq, qb, qh);
       stage.copy(sk, kb, kh);
       if (p.has_ve) stage.copy(se, eb, kh);
+    }
+    // rstd_q, rstd_k and the gate logits of the block, after the rows.
+    for (int i = threadIdx.x; i < ntt * p.H; i += blockDim.x) s_rterm[i] = p.rstd_q[tok0 * p.H + i];
+    for (int i = threadIdx.x; i < ntt * p.Hk; i += blockDim.x) {
+      s_rterm[p.tok * p.H + i] = p.rstd_k[tok0 * p.Hk + i];
+      if (p.has_ve)
+        s_rterm[p.tok * (p.H + p.Hk) + i] = Vec16<T>::scalar(p.gate, static_cast<size_t>(tok0) * p.Hk + i);
     }
     dqb = sdq;
     dkb = sdk;
@@ -290,11 +315,17 @@ __global__ void __launch_bounds__(kPrologueThreads) epilogue_kernel(const EpiPar
       if (kind != 2) {
         HVec::load((kind == 0 ? qb : kb) + boff, xl);
         HVec::load((kind == 0 ? qb : kb) + boff + HALF, xh);
-        rs = (kind == 0 ? p.rstd_q : p.rstd_k)[row];
+        if constexpr (STAGED)
+          rs = kind == 0 ? s_rterm[tt * p.H + head] : s_rterm[p.tok * p.H + tt * p.Hk + head];
+        else
+          rs = (kind == 0 ? p.rstd_q : p.rstd_k)[row];
       } else if (p.has_ve) {
         HVec::load(eb + boff, xl);
         HVec::load(eb + boff + HALF, xh);
-        gl = Vec16<T>::scalar(p.gate, row);
+        if constexpr (STAGED)
+          gl = s_rterm[p.tok * (p.H + p.Hk) + tt * p.Hk + head];
+        else
+          gl = Vec16<T>::scalar(p.gate, row);
       } else {
 #pragma unroll
         for (int i = 0; i < HV; ++i) xl[i] = xh[i] = 0.f;

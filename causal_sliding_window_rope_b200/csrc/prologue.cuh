@@ -238,10 +238,12 @@ struct Stage {
   }
 };
 
-// Shared-memory bytes of the staged prologue for `tok` tokens.
+// Shared-memory bytes of the staged prologue for `tok` tokens: q, k, v and
+// ve rows, then the block's gate logits as float32 (with ve).
 __host__ __device__ inline size_t prologue_stage_bytes(int tok, int H, int Hk, int D, int esize,
                                                        bool has_ve) {
-  return static_cast<size_t>(tok) * (H + (has_ve ? 3 : 2) * Hk) * D * esize;
+  return static_cast<size_t>(tok) * (H + (has_ve ? 3 : 2) * Hk) * D * esize +
+         (has_ve ? static_cast<size_t>(tok) * Hk * 4 : 0);
 }
 
 template <typename T, int D, bool STAGED>
@@ -267,6 +269,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const T *vb = static_cast<const T*>(p.v) + tok0 * kvrow;
   const T *eb = p.has_ve ? static_cast<const T*>(p.ve) + tok0 * kvrow : nullptr;
   const Stage stage{&s_bar};
+  // The block's gate logits (value rows), staged next to the rows so that no
+  // row waits on a global load: float32 after the ve rows.
+  float* s_gate = reinterpret_cast<float*>(stage_smem + static_cast<size_t>(p.tok) * (qrow + 3 * kvrow) * sizeof(T));
   pdl_launch_dependents();
   tab.fill(tok0, p.T, p.omega, ntt);
   pdl_wait();
@@ -275,6 +280,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
     T* sk = sq + p.tok * qrow;
     T* sv = sk + p.tok * kvrow;
     T* se = sv + p.tok * kvrow;
+    if (p.has_ve && !p.xg)
+      for (int i = threadIdx.x; i < ntt * p.Hk; i += blockDim.x)
+        s_gate[i] = Vec16<T>::scalar(p.gate, static_cast<size_t>(tok0) * p.Hk + i);
     if (threadIdx.x == 0) {
       const uint32_t qb_ = static_cast<uint32_t>(ntt * qrow * sizeof(T));
       const uint32_t kb_ = static_cast<uint32_t>(ntt * kvrow * sizeof(T));
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
     if (has_e) {
       HVec::load(eb + boff, el);
       HVec::load(eb + boff + HALF, eh);
-      if (!p.xg) gl = Vec16<T>::scalar(p.gate, row);
+      if (!p.xg) gl = STAGED ? s_gate[tt * p.Hk + head] : Vec16<T>::scalar(p.gate, row);
     } else {
 #pragma unroll
       for (int i = 0; i < HV; ++i) el[i] = eh[i] = 0.f;
